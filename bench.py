@@ -1,0 +1,412 @@
+"""Benchmark of the segment-causal attention hot path on B200.
+
+One step = the whole hot path at steady state on one layer's cache:
+  nomas_kv_commit of a finished 3-latent-frame segment (RoPE + INT8
+  quantisation + ring append, evicting the oldest frames of the 18-frame
+  window), then nomas_seg_attn of the next segment (3 latent frames of
+  22x40 = 2640 video tokens + 256 text tokens, 16 heads x 128) over the
+  18-frame INT8 history (15,840 cached tokens): Nk = 18,736 keys.
+The history stays at 18 frames, so every step does the same work.
+
+Metric: seg-attention TFLOP/s = 4*H*D*Nq*Nk FLOP per step / step time
+(QK^T + PV, unpadded, no softmax credit), and ms per layer-step.
+Inputs are synthetic (seeded generator in synth/), shapes from the pages.
+L2 (126 MB) is flushed before every timed step by writing 512 MB; the flush
+is outside the per-step CUDA-event windows.
+
+--impl reference times the CPU oracle (oracle/) as it stands, on a bounded
+sample of the same workload (rank 0 only), as the reference arm.
+With torchrun (N > 1) every rank runs an independent layer cache on its GPU
+(weak scaling, no data-path collective); the time is the max over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+WORKLOAD = "single_gpu_int8_18f"
+HEAD_DIM = 128
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=1000)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--impl", default="nomas", choices=["nomas", "reference"])
+    p.add_argument("--e2e-steps", type=int, default=0, help="end-to-end steps (default: min(steps, 100))")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(path))
+        return d, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_shape(w):
+    F = w["grid_h"] * w["grid_w"]
+    nq = w["cur_frames"] * F + w["n_text"]
+    nc = w["window"] * F
+    nk = nc + nq
+    flop = 4.0 * w["heads"] * HEAD_DIM * nq * nk
+    return F, nq, nc, nk, flop
+
+
+def commit_bytes(w):
+    """Algorithmic bytes of one commit: read K, V BF16; write codes + fp32 scales."""
+    F = w["grid_h"] * w["grid_w"]
+    rows = w["cur_frames"] * F * w["heads"]
+    return rows * 2 * (HEAD_DIM * 2 + HEAD_DIM + 4)
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+        self.t_on = self.t_off = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def mark(self, on: bool):
+        if on:
+            self.t_on = time.time()
+        else:
+            self.t_off = time.time()
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for ts, line in self.lines:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 8:
+                continue
+            if self.t_on is not None and not (self.t_on <= ts <= (self.t_off or ts)):
+                continue
+            rows.append(parts)
+        if not rows:
+            rows = [[x.strip() for x in l.split(",")] for _, l in self.lines if len(l.split(",")) >= 8]
+        if not rows:
+            return None
+        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for name, val in zip(names, r[4:8]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timings (reference arm and cpu_baseline)
+# ---------------------------------------------------------------------------
+
+def oracle_setup(w):
+    import oracle
+    orc = oracle.OracleCache(oracle.MODE_INT8, w["heads"], w["grid_h"], w["grid_w"], w["window"], w["capacity"])
+    oracle.build_history(orc, w["hist_commits"], w["seed"])
+    geo = synth.Geometry(w["heads"], w["grid_h"], w["grid_w"])
+    q, k, v = synth.segment_qkv(geo, w["cur_frames"], w["n_text"], w["seed"], segment=len(w["hist_commits"]))
+    return orc, q, k, v
+
+
+def oracle_rate(orc, q, k, v, w, rows, nthreads):
+    """TFLOP/s of the oracle on `rows` query rows (all heads)."""
+    _, _, _, nk, _ = workload_shape(w)
+    t0 = time.perf_counter()
+    orc.seg_attn(q, k, v, w["cur_frames"], w["n_text"], rows=rows, nthreads=nthreads)
+    dt = time.perf_counter() - t0
+    flop = 4.0 * w["heads"] * HEAD_DIM * len(rows) * nk
+    return flop / dt / 1e12, dt, flop
+
+
+def cpu_baseline(w):
+    import oracle
+    nthreads = oracle.default_threads()
+    orc, q, k, v = oracle_setup(w)
+    _, nq, _, _, _ = workload_shape(w)
+    rng = np.random.default_rng(0)
+    probe = np.sort(rng.choice(nq, 8, replace=False))
+    _, dt, _ = oracle_rate(orc, q, k, v, w, probe, nthreads)
+    n = int(np.clip(8 * 12.0 / max(dt, 1e-3), 8, nq))
+    rows = np.sort(rng.choice(nq, n, replace=False))
+    rate, dt, flop = oracle_rate(orc, q, k, v, w, rows, nthreads)
+    return {"value": rate, "unit": "TFLOP/s", "cores": nthreads, "kind": "oracle",
+            "sample": f"{n} query rows x {w['heads']} heads of the {WORKLOAD} workload (fp64 two-pass softmax over "
+                      f"all {workload_shape(w)[3]} keys), {dt:.1f} s, {flop / 1e9:.1f} GFLOP"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    import oracle
+    w = synth.WORKLOADS[WORKLOAD]
+    nthreads = oracle.default_threads()
+    orc, q, k, v = oracle_setup(w)
+    _, nq, _, nk, flop_step = workload_shape(w)
+    # one step = one query row of every head (bounded so K + W steps end in minutes)
+    budget_s = 150.0
+    rng = np.random.default_rng(1)
+    t0 = time.perf_counter()
+    oracle_rate(orc, q, k, v, w, np.array([0]), nthreads)
+    per_row = time.perf_counter() - t0
+    rows_per_step = int(np.clip(budget_s / max(per_row, 1e-4) / max(args.steps + args.warmup, 1), 1, 64))
+    for _ in range(args.warmup):
+        oracle_rate(orc, q, k, v, w, rng.choice(nq, rows_per_step, replace=False), nthreads)
+    tot_flop = 0.0
+    tot_t = 0.0
+    for _ in range(args.steps):
+        r, dt, fl = oracle_rate(orc, q, k, v, w, np.sort(rng.choice(nq, rows_per_step, replace=False)), nthreads)
+        tot_flop += fl
+        tot_t += dt
+    value = tot_flop / tot_t / 1e12
+    ms_full = flop_step / (value * 1e12) * 1e3
+    F, _, nc, _, _ = workload_shape(w)
+    line = {"metric": "seg_attn_tflops", "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_full, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": WORKLOAD, "heads": w["heads"], "grid": [w["grid_h"], w["grid_w"]],
+                       "history_frames": w["window"], "cache": "int8", "n_video_frames": w["cur_frames"],
+                       "n_text": w["n_text"], "nq": nq, "nk": nk},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": nthreads, "kind": "oracle",
+                             "sample": f"{rows_per_step} query rows x {w['heads']} heads per step; ms_per_step "
+                                       f"extrapolates to all {nq} rows"},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import torch
+    import segment_causal_kv_b200 as nm
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    w = synth.WORKLOADS[WORKLOAD]
+    F, nq, nc, nk, flop_step = workload_shape(w)
+    geo = synth.Geometry(w["heads"], w["grid_h"], w["grid_w"])
+    to_dev = lambda b: torch.from_numpy(np.ascontiguousarray(b).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    cache = nm.KVCache("int8", w["heads"], w["grid_h"], w["grid_w"], w["window"], w["capacity"], device=dev)
+    for s, nf in enumerate(w["hist_commits"]):
+        k, v = synth.history_kv(geo, nf, w["seed"] + rank, s)
+        cache.commit(to_dev(k), to_dev(v), nf)
+    n_seg = len(w["hist_commits"])
+    kf_h, vf_h = synth.history_kv(geo, w["cur_frames"], w["seed"] + rank, n_seg)
+    q_h, k_h, v_h = synth.segment_qkv(geo, w["cur_frames"], w["n_text"], w["seed"] + rank, segment=n_seg + 1)
+    kf, vf, q, k, v = (to_dev(x) for x in (kf_h, vf_h, q_h, k_h, v_h))
+    out = torch.empty((nq, w["heads"], HEAD_DIM), dtype=torch.bfloat16, device=dev)
+    ws = cache.workspace(w["cur_frames"], w["n_text"])
+    flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        cache.commit(kf, vf, w["cur_frames"], stream=stream)
+        cache.seg_attn(q, k, v, w["cur_frames"], w["n_text"], out=out, workspace=ws, stream=stream)
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    if dist:
+        dist.barrier()
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    sampler.mark(True)
+    torch.cuda.synchronize(dev)
+    if dist:
+        dist.barrier()
+    for i in range(K):
+        flush.zero_()
+        ev[i][0].record(stream)
+        cache.commit(kf, vf, w["cur_frames"], stream=stream)
+        ev[i][1].record(stream)
+        cache.seg_attn(q, k, v, w["cur_frames"], w["n_text"], out=out, workspace=ws, stream=stream)
+        ev[i][2].record(stream)
+    torch.cuda.synchronize(dev)
+    if dist:
+        dist.barrier()
+    sampler.mark(False)
+    commit_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K)]
+    attn_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]
+    step_ms_total = sum(commit_ms) + sum(attn_ms)
+    if dist:
+        t = torch.tensor([step_ms_total, sum(attn_ms)], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        step_ms_total, attn_total = float(t[0]), float(t[1])
+    else:
+        attn_total = sum(attn_ms)
+    if cache.device_status(stream) != nm.NOMAS_OK:
+        raise RuntimeError("a kernel reported a timed-out wait")
+
+    # ---- end to end through the public API from pinned host buffers
+    Ke = args.e2e_steps or min(K, 100)
+    host_in = [torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16).pin_memory()
+               for x in (kf_h, vf_h, q_h, k_h, v_h)]
+    dev_in = [torch.empty_like(x, device=dev) for x in host_in]
+    host_out = torch.empty((nq, w["heads"], HEAD_DIM), dtype=torch.bfloat16).pin_memory()
+    h2d = sum(x.numel() * x.element_size() for x in host_in)
+    d2h = host_out.numel() * host_out.element_size()
+
+    def e2e_step():
+        for hsrc, ddst in zip(host_in, dev_in):
+            ddst.copy_(hsrc, non_blocking=True)
+        cache.commit(dev_in[0], dev_in[1], w["cur_frames"], stream=stream)
+        cache.seg_attn(dev_in[2], dev_in[3], dev_in[4], w["cur_frames"], w["n_text"], out=out, workspace=ws,
+                       stream=stream)
+        host_out.copy_(out, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    if dist:
+        dist.barrier()
+    e2e_ms = []
+    for _ in range(Ke):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        e2e_step()
+        b.record(stream)
+        b.synchronize()
+        e2e_ms.append(a.elapsed_time(b))
+    e2e_total = sum(e2e_ms)
+    if dist:
+        t = torch.tensor([e2e_total], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_total = float(t[0])
+    clocks = sampler.stop()
+
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    peaks, peak_src = load_peaks()
+    ms_step = step_ms_total / K
+    value = world * flop_step * K / (step_ms_total * 1e-3) / 1e12
+    attn_avg_ms = attn_total / K
+    achieved = flop_step / (attn_avg_ms * 1e-3) / 1e12
+    peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    peak_burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    cm = statistics.mean(commit_ms)
+    line = {
+        "metric": "seg_attn_tflops",
+        "value": value,
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "heads": w["heads"], "grid": [w["grid_h"], w["grid_w"]],
+                   "history_frames": w["window"], "cache": "int8", "n_video_frames": w["cur_frames"],
+                   "n_text": w["n_text"], "nq": nq, "nk": nk, "flop_per_step": flop_step,
+                   "step": "kv_commit(3 frames) + seg_attn", "l2": "flushed: 512 MB written before each step",
+                   "parallelism": f"replica x{world}"},
+        "attn_ms": attn_avg_ms,
+        "commit_ms": cm,
+        "commit_gbs": commit_bytes(w) / (cm * 1e-3) / 1e9,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": None, "peak_kind": f"bf16 dense, sustained, {peak_src}",
+                     "frac_of_burst": achieved / peak_burst, "frac_of_nominal_2250": achieved / 2250.0,
+                     "kernel": "nomas_seg_attn call (prep + attn_kernel + combine), CUDA events"},
+        "e2e": {"value": world * flop_step * Ke / (e2e_total * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": Ke,
+                "ms_per_step": e2e_total / Ke},
+        # per step: commit, RoPE prep, attention, and the split combine when used
+        "gpu_launches": K * (3 + _combine_launches(cache)),
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        try:
+            line["cpu_baseline"] = cpu_baseline(w)
+        except Exception as e:  # the baseline is reported, never required
+            line["cpu_baseline"] = {"value": None, "error": str(e)}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def _combine_launches(cache) -> int:
+    """1 when the shape uses KV splits (the combine kernel runs), else 0."""
+    ws = cache.workspace_bytes(3, 256)
+    h, F = cache.heads, cache.tokens_per_frame
+    nq = 3 * F + 256
+    qk = 2 * ((h * nq * HEAD_DIM * 2 + 255) // 256 * 256)
+    return 1 if ws > 256 + qk + 256 else 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

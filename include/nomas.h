@@ -1,0 +1,197 @@
+/*
+ * nomas.h -- C ABI of the segment-causal joint attention library (sm_100a).
+ *
+ * One layer of a segment-autoregressive video MMDiT (Hy-Nomas): the current
+ * segment's text and video tokens attend to each other and to a lifelong
+ * key/value cache of earlier segments' video tokens; video positions carry
+ * 3D RoPE. The cache holds either BF16 values (full history) or INT8 codes
+ * with a per-(token, head) fp32 scale and a sliding window of latent frames.
+ *
+ * Sources (page title, section):
+ *  - Hy-Nomas model card, "Segment-Autoregressive Diffusion Transformer":
+ *    segment-wise causal joint attention with 3D RoPE and a per-layer KV
+ *    cache supplying earlier segments; architecture table (16 heads x 128,
+ *    RoPE split [16,56,56] over t/h/w, theta 256); "Attention is causal
+ *    across segments"; cached keys and values are reused; full history
+ *    (max_cache_segments=null) in the standard configuration.
+ *  - same card, "Single-GPU Low-Memory Inference": INT8 KV storage with
+ *    BF16 attention computation; a GPU history budget of 18 latent frames.
+ *  - "Hy-Nomas Explained" blog, "Segment-wise causal joint attention" and
+ *    "Step 3: The Video Latent ...": 22 x 40 = 880 tokens per latent frame.
+ *
+ * Conventions for every call:
+ *  - Pointers named "device" must point to device memory of the current
+ *    CUDA device; the caller owns all memory. The library never allocates
+ *    or frees memory, never synchronises (except nomas_device_status), and
+ *    enqueues work only on the given stream (a cudaStream_t passed as
+ *    void*; NULL means the legacy default stream).
+ *  - Return value: NOMAS_OK (0) or a negative NOMAS_ERR_* code. All
+ *    argument and state validation happens on the host before any launch:
+ *    a call that returns an error has enqueued nothing and changed nothing.
+ *  - BF16 tensors are passed as raw 16-bit patterns; layouts are row-major
+ *    with the last index fastest.
+ *  - Head dimension is fixed at 128 and the RoPE split at [16, 56, 56].
+ *  - RoPE pairs are interleaved (2j, 2j+1) inside each axis block; pair j of
+ *    a block of width d turns by pos * theta^(-2j/d). A video token's
+ *    position is (t, h, w): t = absolute latent-frame index since the last
+ *    nomas_cache_reset, (h, w) its grid cell; tokens of a frame are
+ *    row-major (h, then w). Text tokens are not rotated.
+ *  - A descriptor must not be used from two host threads at once. Device
+ *    work of successive calls is ordered only by the stream(s) the caller
+ *    passes.
+ */
+#ifndef NOMAS_H
+#define NOMAS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ---------------------------------------------------- */
+#define NOMAS_OK 0
+#define NOMAS_ERR_ARG (-1)       /* NULL pointer, bad size, head_dim != 128, ... */
+#define NOMAS_ERR_ALIGN (-2)     /* pointer or stride not 16-byte aligned */
+#define NOMAS_ERR_STATE (-3)     /* descriptor not reset, or changed since */
+#define NOMAS_ERR_CAPACITY (-4)  /* full-history commit beyond capacity_frames */
+#define NOMAS_ERR_WORKSPACE (-5) /* workspace NULL or smaller than required */
+#define NOMAS_ERR_CUDA (-6)      /* a CUDA runtime/driver call failed */
+#define NOMAS_ERR_DEVICE (-7)    /* current device is not sm_100 */
+#define NOMAS_ERR_DEVICE_TIMEOUT (-8) /* a kernel gave up a bounded wait */
+
+/* ---- cache modes ------------------------------------------------------ */
+#define NOMAS_CACHE_BF16 0 /* cached K/V kept as BF16 (K after RoPE) */
+#define NOMAS_CACHE_INT8 1 /* cached K/V as INT8 codes + fp32 per-(token, head) scales */
+
+#define NOMAS_HEAD_DIM 128
+#define NOMAS_MAX_GRID_HW 96 /* grid_h + grid_w limit (RoPE tables travel as launch arguments) */
+
+/*
+ * One layer's K/V cache. The caller fills the configuration fields and the
+ * device pointers, then calls nomas_cache_reset; the library maintains the
+ * state fields afterwards (treat them as read-only).
+ *
+ * Slots: a slot holds one latent frame (grid_h * grid_w tokens). Cache
+ * buffers are head-major:
+ *   k, v      : [heads][capacity_frames * tokens_per_frame][128]
+ *               int8 codes (INT8 mode) or BF16 bits (BF16 mode), device;
+ *               16-byte aligned.
+ *   k_scale,
+ *   v_scale   : fp32 [heads][capacity_frames * tokens_per_frame], device,
+ *               16-byte aligned (INT8 mode; must be NULL in BF16 mode).
+ * window_frames > 0: the cache keeps only the last window_frames committed
+ *   latent frames (FIFO at frame granularity); frame f lives in slot
+ *   f mod window_frames; capacity_frames must equal window_frames.
+ * window_frames == 0: full history; frame f lives in slot f and a commit
+ *   that would pass capacity_frames fails with NOMAS_ERR_CAPACITY.
+ * Eviction is bookkeeping only: an evicted slot is simply overwritten by a
+ * later frame. Because slots fill from 0 and wrap only when full, the
+ * visible history is always slots [0, valid_frames).
+ */
+typedef struct nomas_cache {
+    /* configuration (caller) */
+    int32_t mode;            /* NOMAS_CACHE_BF16 or NOMAS_CACHE_INT8 */
+    int32_t heads;           /* attention heads (16 in Hy-Nomas) */
+    int32_t head_dim;        /* must be 128 */
+    int32_t grid_h, grid_w;  /* latent grid; tokens_per_frame = grid_h * grid_w */
+    int32_t window_frames;   /* history budget in latent frames; 0 = full history */
+    int32_t capacity_frames; /* slots allocated */
+    float rope_theta;        /* 256 in Hy-Nomas */
+    void *k, *v;             /* device, see above */
+    float *k_scale, *v_scale;
+    /* state (library) */
+    int64_t frames_committed; /* absolute index of the next frame to commit */
+    int32_t valid_frames;     /* frames visible to attention (slots [0, valid_frames)) */
+    int32_t head_slot;        /* slot the next committed frame goes to */
+    uint64_t check;           /* reset stamp over the configuration fields */
+} nomas_cache;
+
+/*
+ * nomas_cache_reset -- validate the descriptor and empty the cache.
+ * Host only: sets frames_committed = valid_frames = head_slot = 0 and stamps
+ * the configuration. Cache memory is not touched (no kernel is launched).
+ * Errors: NOMAS_ERR_ARG (c NULL, non-positive sizes, head_dim != 128,
+ * unknown mode, window > 0 with capacity != window, grid_h + grid_w >
+ * NOMAS_MAX_GRID_HW, theta <= 0, scales present in BF16 mode or missing in
+ * INT8 mode), NOMAS_ERR_ALIGN (a buffer not 16-byte aligned).
+ */
+int nomas_cache_reset(nomas_cache *c);
+
+/*
+ * nomas_kv_commit -- append a finished segment's video K/V to the cache
+ * (model card: cached keys and values are reused when generation advances;
+ * single-GPU configuration: INT8 storage and an 18-frame history budget).
+ *
+ * k, v : device, BF16 bits, token-major [n_frames * tokens_per_frame][heads][128];
+ *        consecutive tokens are token_stride elements apart
+ *        (token_stride >= heads * 128, a multiple of 8); 16-byte aligned.
+ *        Only video tokens are committed; text tokens are not cached.
+ * n_frames : latent frames in the segment (>= 0; 0 is a no-op).
+ * Frame i of the segment gets t = frames_committed + i. K is rotated with
+ * 3D RoPE in fp32 (c, s = fp32 roundings of the double-precision cos/sin of
+ * pos * theta^(-2j/d); y0 = fma(x0, c, -rn(x1*s)), y1 = fma(x0, s, rn(x1*c))),
+ * V is not. INT8 mode: per (token, head) row of 128, absmax a, scale =
+ * a / 127 (IEEE fp32 division; 0 when a == 0), code = round-half-even(x /
+ * scale) clamped to [-127, 127]. BF16 mode: round-half-even to BF16.
+ * With a window, frames of this segment that fall out of the window by its
+ * end are not written. Host state is advanced at enqueue time.
+ * Errors: NOMAS_ERR_ARG, NOMAS_ERR_ALIGN, NOMAS_ERR_STATE (descriptor not
+ * reset or configuration changed), NOMAS_ERR_CAPACITY, NOMAS_ERR_CUDA.
+ */
+int nomas_kv_commit(nomas_cache *c, const void *k, const void *v, int64_t token_stride, int32_t n_frames,
+                    void *stream);
+
+/*
+ * nomas_seg_attn_workspace_bytes -- device workspace nomas_seg_attn needs
+ * for this cache state and segment shape (0 on invalid arguments). The
+ * first 256 bytes of a workspace are a status header: zero them once
+ * before first use; the library only sets error bits in it.
+ */
+size_t nomas_seg_attn_workspace_bytes(const nomas_cache *c, int32_t n_video_frames, int32_t n_text);
+
+/*
+ * nomas_seg_attn -- segment-causal joint attention of the current segment
+ * (model card: the current segment attends to all past KV cache and to
+ * itself; attention is causal across segments, bidirectional inside one).
+ *
+ * q, k, v : device, BF16 bits, token-major [Nq][heads][128] with
+ *           Nq = n_video_frames * tokens_per_frame + n_text, video tokens
+ *           first; token_stride elements between tokens (>= heads*128,
+ *           multiple of 8); 16-byte aligned. Video frame i of the segment
+ *           has t = c->frames_committed + i (the segment directly follows
+ *           the committed history).
+ * out     : device, BF16 bits [Nq][heads][128] (contiguous), 16-byte aligned.
+ * lse     : optional device fp32 [heads][Nq]: natural-log sum of exp of the
+ *           scaled scores; NULL to skip.
+ * For each head and query i: out_i = sum_j softmax_j(<R(p_i) q_i, k_j> / sqrt(128)) v_j
+ * over the visible cached tokens (INT8 mode: code * scale) and all Nq
+ * tokens of the current segment (keys rotated with their own positions).
+ * The cache is read only. Q and current K are rounded to BF16 after RoPE,
+ * probabilities are BF16 for the P.V product, accumulation is fp32.
+ * workspace : device, >= nomas_seg_attn_workspace_bytes(...) bytes,
+ *             256-byte aligned, not shared with a call running concurrently.
+ * Errors: NOMAS_ERR_ARG, NOMAS_ERR_ALIGN, NOMAS_ERR_STATE,
+ * NOMAS_ERR_WORKSPACE, NOMAS_ERR_DEVICE, NOMAS_ERR_CUDA.
+ */
+int nomas_seg_attn(const nomas_cache *c, const void *q, const void *k, const void *v, int64_t token_stride,
+                   int32_t n_video_frames, int32_t n_text, void *out, float *lse, void *workspace,
+                   size_t workspace_bytes, void *stream);
+
+/*
+ * nomas_device_status -- synchronise `stream`, read and clear the status
+ * header of a workspace. Returns NOMAS_OK, NOMAS_ERR_DEVICE_TIMEOUT (a
+ * kernel abandoned a bounded wait; its outputs are invalid) or
+ * NOMAS_ERR_CUDA. This is the only call that blocks the host.
+ */
+int nomas_device_status(void *workspace, void *stream);
+
+/* Human-readable name of a status code (static storage). */
+const char *nomas_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NOMAS_H */

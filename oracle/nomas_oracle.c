@@ -131,32 +131,58 @@ static void video_pos(int64_t n, int64_t t0, int gh, int gw, double pos[3]) {
     (void)gh;
 }
 
-/* fp64 rotation of one 128-vector at position pos (exact cos/sin). */
-void orc_rope_rotate_f64(const double *x, const double pos[3], double theta, double *y) {
+/* cos/sin (double) of the 64 pairs at position pos: cs[2p] = cos, cs[2p+1] = sin. */
+static void rope_cs_f64_all(const double pos[3], double theta, double *cs) {
     for (int p = 0; p < ORC_D / 2; ++p) {
         int d, j;
         int ax = pair_axis(p, &d, &j);
         double a = orc_rope_angle(d, j, pos[ax], theta);
-        double c = cos(a), s = sin(a);
+        cs[2 * p] = cos(a);
+        cs[2 * p + 1] = sin(a);
+    }
+}
+
+static void rotate_f64_cs(const double *x, const double *cs, double *y) {
+    for (int p = 0; p < ORC_D / 2; ++p) {
+        double c = cs[2 * p], s = cs[2 * p + 1];
         double x0 = x[2 * p], x1 = x[2 * p + 1];
         y[2 * p] = x0 * c - x1 * s;
         y[2 * p + 1] = x0 * s + x1 * c;
     }
 }
 
-/* fp32 rotation with the commit's exact expression. */
-void orc_rope_rotate_f32(const float *x, const double pos[3], double theta, float *y) {
+/* fp64 rotation of one 128-vector at position pos (exact cos/sin). */
+void orc_rope_rotate_f64(const double *x, const double pos[3], double theta, double *y) {
+    double cs[ORC_D];
+    rope_cs_f64_all(pos, theta, cs);
+    rotate_f64_cs(x, cs, y);
+}
+
+/* fp32 cos/sin of the 64 pairs at position pos (commit table). */
+static void rope_cs_f32_all(const double pos[3], double theta, float *cs) {
     for (int p = 0; p < ORC_D / 2; ++p) {
         int d, j;
         int ax = pair_axis(p, &d, &j);
-        float c, s;
-        orc_rope_cs_f32(d, j, pos[ax], theta, &c, &s);
+        orc_rope_cs_f32(d, j, pos[ax], theta, &cs[2 * p], &cs[2 * p + 1]);
+    }
+}
+
+static void rotate_f32_cs(const float *x, const float *cs, float *y) {
+    for (int p = 0; p < ORC_D / 2; ++p) {
+        float c = cs[2 * p], s = cs[2 * p + 1];
         float x0 = x[2 * p], x1 = x[2 * p + 1];
         float x1s = x1 * s; /* rounded to fp32 (compiled with -ffp-contract=off) */
         float x1c = x1 * c;
         y[2 * p] = fmaf(x0, c, -x1s);
         y[2 * p + 1] = fmaf(x0, s, x1c);
     }
+}
+
+/* fp32 rotation with the commit's exact expression. */
+void orc_rope_rotate_f32(const float *x, const double pos[3], double theta, float *y) {
+    float cs[ORC_D];
+    rope_cs_f32_all(pos, theta, cs);
+    rotate_f32_cs(x, cs, y);
 }
 
 /* ------------------------------------------------------------------ */
@@ -220,13 +246,19 @@ int orc_commit(orc_cache *c, const uint16_t *k, const uint16_t *v, int64_t token
             int64_t n = (int64_t)i * F + r; /* token inside the segment */
             double pos[3];
             video_pos(n, c->frames_committed, c->grid_h, c->grid_w, pos);
+            float csf[ORC_D];
+            double csd[ORC_D];
+            if (c->mode == ORC_MODE_F64)
+                rope_cs_f64_all(pos, c->theta, csd);
+            else
+                rope_cs_f32_all(pos, c->theta, csf);
             for (int h = 0; h < H; ++h) {
                 const uint16_t *kr = k + n * token_stride + (int64_t)h * ORC_D;
                 const uint16_t *vr = v + n * token_stride + (int64_t)h * ORC_D;
                 int64_t row = (int64_t)h * cap_tok + slot * F + r;
                 if (c->mode == ORC_MODE_F64) {
                     for (int e = 0; e < ORC_D; ++e) xd[e] = (double)bf16_to_f32(kr[e]);
-                    orc_rope_rotate_f64(xd, pos, c->theta, yd);
+                    rotate_f64_cs(xd, csd, yd);
                     for (int e = 0; e < ORC_D; ++e) {
                         c->k_f64[row * ORC_D + e] = yd[e];
                         c->v_f64[row * ORC_D + e] = (double)bf16_to_f32(vr[e]);
@@ -234,7 +266,7 @@ int orc_commit(orc_cache *c, const uint16_t *k, const uint16_t *v, int64_t token
                     continue;
                 }
                 for (int e = 0; e < ORC_D; ++e) xf[e] = bf16_to_f32(kr[e]);
-                orc_rope_rotate_f32(xf, pos, c->theta, yf);
+                rotate_f32_cs(xf, csf, yf);
                 if (c->mode == ORC_MODE_BF16) {
                     for (int e = 0; e < ORC_D; ++e) {
                         c->k_bf16[row * ORC_D + e] = orc_f32_to_bf16(yf[e]);
@@ -326,21 +358,32 @@ static void attend_rows_parallel(const key_set *ks, const double *qrot, int64_t 
         for (int t = 0; t < nthreads; ++t) pthread_join(th[t], NULL);
 }
 
-/* Rotated fp64 copy of a segment's tensor for head h (video tokens rotated
- * at t0 + frame, text tokens unchanged). */
-static void rotate_segment(const uint16_t *x, int64_t token_stride, int h, int64_t nv, int64_t nq, int64_t t0,
-                           int gh, int gw, double theta, double *out) {
+/* cos/sin tables of a segment's video tokens: [nv][128] (t0 + frame, h, w). */
+static double *segment_cs(int64_t nv, int64_t t0, int gh, int gw, double theta) {
+    double *cs = (double *)malloc(sizeof(double) * (size_t)(nv > 0 ? nv : 1) * ORC_D);
+    if (!cs) return NULL;
+    for (int64_t n = 0; n < nv; ++n) {
+        double pos[3];
+        video_pos(n, t0, gh, gw, pos);
+        rope_cs_f64_all(pos, theta, cs + n * ORC_D);
+    }
+    return cs;
+}
+
+/* Rotated fp64 copy of rows `rows` (NULL: 0..nrows-1) of a segment's tensor
+ * for head h: video tokens (index < nv) rotated with the tables `cs`, text
+ * tokens unchanged. */
+static void rotate_segment(const uint16_t *x, int64_t token_stride, int h, int64_t nv, const int64_t *rows,
+                           int64_t nrows, const double *cs, double *out) {
     double tmp[ORC_D];
-    for (int64_t n = 0; n < nq; ++n) {
+    for (int64_t r = 0; r < nrows; ++r) {
+        int64_t n = rows ? rows[r] : r;
         const uint16_t *xr = x + n * token_stride + (int64_t)h * ORC_D;
         for (int e = 0; e < ORC_D; ++e) tmp[e] = (double)bf16_to_f32(xr[e]);
-        if (n < nv) {
-            double pos[3];
-            video_pos(n, t0, gh, gw, pos);
-            orc_rope_rotate_f64(tmp, pos, theta, out + n * ORC_D);
-        } else {
-            memcpy(out + n * ORC_D, tmp, sizeof(tmp));
-        }
+        if (n < nv)
+            rotate_f64_cs(tmp, cs + n * ORC_D, out + r * ORC_D);
+        else
+            memcpy(out + r * ORC_D, tmp, sizeof(tmp));
     }
 }
 
@@ -402,12 +445,12 @@ int orc_seg_attn(const orc_cache *c, const uint16_t *q, const uint16_t *k, const
 
     double *keys = (double *)malloc(sizeof(double) * (size_t)(nk > 0 ? nk : 1) * ORC_D);
     double *vals = (double *)malloc(sizeof(double) * (size_t)(nk > 0 ? nk : 1) * ORC_D);
-    double *qall = (double *)malloc(sizeof(double) * (size_t)(nq > 0 ? nq : 1) * ORC_D);
+    double *cs = segment_cs(nv, t0, c->grid_h, c->grid_w, c->theta);
     double *qsel = (double *)malloc(sizeof(double) * (size_t)(n_rows > 0 ? n_rows : 1) * ORC_D);
     double *osel = (double *)malloc(sizeof(double) * (size_t)(n_rows > 0 ? n_rows : 1) * ORC_D);
     double *lsel = (double *)malloc(sizeof(double) * (size_t)(n_rows > 0 ? n_rows : 1));
-    if (!keys || !vals || !qall || !qsel || !osel || !lsel) {
-        free(keys); free(vals); free(qall); free(qsel); free(osel); free(lsel);
+    if (!keys || !vals || !cs || !qsel || !osel || !lsel) {
+        free(keys); free(vals); free(cs); free(qsel); free(osel); free(lsel);
         return -3;
     }
     for (int h = 0; h < H; ++h) {
@@ -417,13 +460,9 @@ int orc_seg_attn(const orc_cache *c, const uint16_t *q, const uint16_t *k, const
             for (int64_t r = 0; r < F; ++r, ++j)
                 cache_row(c, (int64_t)h * cap_tok + (int64_t)s * F + r, keys + j * ORC_D, vals + j * ORC_D);
         }
-        rotate_segment(k, token_stride, h, nv, nq, t0, c->grid_h, c->grid_w, c->theta, keys + nc * ORC_D);
+        rotate_segment(k, token_stride, h, nv, NULL, nq, cs, keys + nc * ORC_D);
         plain_segment(v, token_stride, h, nq, vals + nc * ORC_D);
-        rotate_segment(q, token_stride, h, nv, nq, t0, c->grid_h, c->grid_w, c->theta, qall);
-        for (int64_t r = 0; r < n_rows; ++r) {
-            int64_t i = rows ? rows[r] : r;
-            memcpy(qsel + r * ORC_D, qall + i * ORC_D, sizeof(double) * ORC_D);
-        }
+        rotate_segment(q, token_stride, h, nv, rows, n_rows, cs, qsel);
         key_set ks = {nk, keys, vals};
         attend_rows_parallel(&ks, qsel, n_rows, osel, lsel, nthreads);
         for (int64_t r = 0; r < n_rows; ++r) {
@@ -431,7 +470,7 @@ int orc_seg_attn(const orc_cache *c, const uint16_t *q, const uint16_t *k, const
             if (lse) lse[(int64_t)h * n_rows + r] = lsel[r];
         }
     }
-    free(keys); free(vals); free(qall); free(qsel); free(osel); free(lsel);
+    free(keys); free(vals); free(cs); free(qsel); free(osel); free(lsel);
     return 0;
 }
 
@@ -480,7 +519,9 @@ int orc_full_seq_attn(int n_seg, const uint16_t *const *qs, const uint16_t *cons
         int64_t j = 0, t0 = 0;
         for (int s = 0; s < target; ++s) {
             int64_t nvs = (int64_t)n_video[s] * F;
-            rotate_segment(ks_[s], stride, h, nvs, nvs, t0, gh, gw, theta, tmp);
+            double *cs_s = segment_cs(nvs, t0, gh, gw, theta);
+            rotate_segment(ks_[s], stride, h, nvs, NULL, nvs, cs_s, tmp);
+            free(cs_s);
             plain_segment(vs[s], stride, h, nvs, tmp + nvs * ORC_D);
             for (int64_t n = 0; n < nvs; ++n) {
                 if (t0 + n / F < lo) continue;
@@ -491,9 +532,11 @@ int orc_full_seq_attn(int n_seg, const uint16_t *const *qs, const uint16_t *cons
             t0 += n_video[s];
         }
         int64_t nvt = (int64_t)n_video[target] * F;
-        rotate_segment(ks_[target], stride, h, nvt, nq, t0_target, gh, gw, theta, keys + j * ORC_D);
+        double *cs_t = segment_cs(nvt, t0_target, gh, gw, theta);
+        rotate_segment(ks_[target], stride, h, nvt, NULL, nq, cs_t, keys + j * ORC_D);
         plain_segment(vs[target], stride, h, nq, vals + j * ORC_D);
-        rotate_segment(qs[target], stride, h, nvt, nq, t0_target, gh, gw, theta, qr);
+        rotate_segment(qs[target], stride, h, nvt, NULL, nq, cs_t, qr);
+        free(cs_t);
         key_set kset = {nk, keys, vals};
         attend_rows_parallel(&kset, qr, nq, ob, lb, nthreads);
         for (int64_t r = 0; r < nq; ++r) {

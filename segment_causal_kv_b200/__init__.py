@@ -1,0 +1,239 @@
+"""Python binding of the sm_100a segment-causal attention library (``libnomas.so``).
+
+Argument marshalling only: every step of the hot path runs in the library's
+CUDA kernels, reached through the C ABI declared in ``include/nomas.h``. The
+functions keep the C names (``nomas_cache_reset``, ``nomas_kv_commit``,
+``nomas_seg_attn``, ...); ``KVCache`` is a convenience wrapper that owns the
+cache tensors (PyTorch is used for device memory and streams only).
+
+There is no fallback: if ``libnomas.so`` has not been built (``python
+segment_causal_kv_b200/build.py`` or ``__graft_entry__.build()``), importing
+the library raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libnomas.so")
+
+NOMAS_OK = 0
+NOMAS_ERR_ARG = -1
+NOMAS_ERR_ALIGN = -2
+NOMAS_ERR_STATE = -3
+NOMAS_ERR_CAPACITY = -4
+NOMAS_ERR_WORKSPACE = -5
+NOMAS_ERR_CUDA = -6
+NOMAS_ERR_DEVICE = -7
+NOMAS_ERR_DEVICE_TIMEOUT = -8
+
+NOMAS_CACHE_BF16 = 0
+NOMAS_CACHE_INT8 = 1
+HEAD_DIM = 128
+
+# exported symbols (checked against include/nomas.h by the tests)
+EXPORTS = ("nomas_cache_reset", "nomas_kv_commit", "nomas_seg_attn_workspace_bytes", "nomas_seg_attn",
+           "nomas_device_status", "nomas_status_string")
+
+
+class NomasCacheDesc(ctypes.Structure):
+    """Mirror of ``struct nomas_cache``."""
+
+    _fields_ = [
+        ("mode", ctypes.c_int32),
+        ("heads", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32),
+        ("grid_h", ctypes.c_int32),
+        ("grid_w", ctypes.c_int32),
+        ("window_frames", ctypes.c_int32),
+        ("capacity_frames", ctypes.c_int32),
+        ("rope_theta", ctypes.c_float),
+        ("k", ctypes.c_void_p),
+        ("v", ctypes.c_void_p),
+        ("k_scale", ctypes.c_void_p),
+        ("v_scale", ctypes.c_void_p),
+        ("frames_committed", ctypes.c_int64),
+        ("valid_frames", ctypes.c_int32),
+        ("head_slot", ctypes.c_int32),
+        ("check", ctypes.c_uint64),
+    ]
+
+
+class NomasError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        super().__init__(f"{what}: {nomas_status_string(status)} ({status})" if what else nomas_status_string(status))
+
+
+_lib = None
+
+
+def lib():
+    """Load ``libnomas.so`` (raises ImportError when it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with `python {os.path.join(HERE, 'build.py')}`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I32, I64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
+        D = ctypes.POINTER(NomasCacheDesc)
+        L.nomas_cache_reset.argtypes = [D]
+        L.nomas_cache_reset.restype = ctypes.c_int
+        L.nomas_kv_commit.argtypes = [D, P, P, I64, I32, P]
+        L.nomas_kv_commit.restype = ctypes.c_int
+        L.nomas_seg_attn_workspace_bytes.argtypes = [D, I32, I32]
+        L.nomas_seg_attn_workspace_bytes.restype = ctypes.c_size_t
+        L.nomas_seg_attn.argtypes = [D, P, P, P, I64, I32, I32, P, P, P, ctypes.c_size_t, P]
+        L.nomas_seg_attn.restype = ctypes.c_int
+        L.nomas_device_status.argtypes = [P, P]
+        L.nomas_device_status.restype = ctypes.c_int
+        L.nomas_status_string.argtypes = [ctypes.c_int]
+        L.nomas_status_string.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+# ---------------------------------------------------------------- raw C ABI
+
+def nomas_status_string(status: int) -> str:
+    return lib().nomas_status_string(int(status)).decode()
+
+
+def nomas_cache_reset(desc: NomasCacheDesc) -> int:
+    return lib().nomas_cache_reset(ctypes.byref(desc))
+
+
+def nomas_kv_commit(desc: NomasCacheDesc, k_ptr: int, v_ptr: int, token_stride: int, n_frames: int,
+                    stream: int | None) -> int:
+    return lib().nomas_kv_commit(ctypes.byref(desc), k_ptr, v_ptr, token_stride, n_frames, stream)
+
+
+def nomas_seg_attn_workspace_bytes(desc: NomasCacheDesc, n_video_frames: int, n_text: int) -> int:
+    return int(lib().nomas_seg_attn_workspace_bytes(ctypes.byref(desc), n_video_frames, n_text))
+
+
+def nomas_seg_attn(desc: NomasCacheDesc, q_ptr: int, k_ptr: int, v_ptr: int, token_stride: int,
+                   n_video_frames: int, n_text: int, out_ptr: int, lse_ptr: int | None, ws_ptr: int | None,
+                   ws_bytes: int, stream: int | None) -> int:
+    return lib().nomas_seg_attn(ctypes.byref(desc), q_ptr, k_ptr, v_ptr, token_stride, n_video_frames, n_text,
+                                out_ptr, lse_ptr, ws_ptr, ws_bytes, stream)
+
+
+def nomas_device_status(ws_ptr: int, stream: int | None) -> int:
+    return lib().nomas_device_status(ws_ptr, stream)
+
+
+def _check(rc: int, what: str) -> None:
+    if rc != NOMAS_OK:
+        raise NomasError(rc, what)
+
+
+# ---------------------------------------------------------------- convenience
+
+def _torch():
+    import torch
+    return torch
+
+
+def _stream_handle(stream) -> int | None:
+    torch = _torch()
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else stream
+
+
+class KVCache:
+    """One layer's lifelong K/V cache in device memory, driven through the C ABI.
+
+    mode: "int8" (codes + fp32 per-(token, head) scales) or "bf16".
+    window: history budget in latent frames (0 = full history).
+    """
+
+    def __init__(self, mode: str, heads: int, grid_h: int, grid_w: int, window: int, capacity: int,
+                 theta: float = 256.0, device=None):
+        torch = _torch()
+        self.device = torch.device(device if device is not None else "cuda")
+        self.mode = mode
+        self.heads, self.grid_h, self.grid_w = heads, grid_h, grid_w
+        self.window, self.capacity = window, capacity
+        F = grid_h * grid_w
+        if mode == "int8":
+            self.k = torch.zeros((heads, capacity * F, HEAD_DIM), dtype=torch.int8, device=self.device)
+            self.v = torch.zeros_like(self.k)
+            self.k_scale = torch.zeros((heads, capacity * F), dtype=torch.float32, device=self.device)
+            self.v_scale = torch.zeros_like(self.k_scale)
+            m = NOMAS_CACHE_INT8
+        elif mode == "bf16":
+            self.k = torch.zeros((heads, capacity * F, HEAD_DIM), dtype=torch.bfloat16, device=self.device)
+            self.v = torch.zeros_like(self.k)
+            self.k_scale = self.v_scale = None
+            m = NOMAS_CACHE_BF16
+        else:
+            raise ValueError(mode)
+        self.desc = NomasCacheDesc(m, heads, HEAD_DIM, grid_h, grid_w, window, capacity, theta,
+                                   self.k.data_ptr(), self.v.data_ptr(),
+                                   self.k_scale.data_ptr() if self.k_scale is not None else None,
+                                   self.v_scale.data_ptr() if self.v_scale is not None else None, 0, 0, 0, 0)
+        self._ws = None
+        self.reset()
+
+    @property
+    def tokens_per_frame(self) -> int:
+        return self.grid_h * self.grid_w
+
+    @property
+    def frames_committed(self) -> int:
+        return int(self.desc.frames_committed)
+
+    @property
+    def valid_frames(self) -> int:
+        return int(self.desc.valid_frames)
+
+    @property
+    def head_slot(self) -> int:
+        return int(self.desc.head_slot)
+
+    def reset(self) -> None:
+        _check(nomas_cache_reset(self.desc), "nomas_cache_reset")
+
+    def commit(self, k, v, n_frames: int, stream=None) -> None:
+        """k, v: BF16 [n_frames * F][heads][128] (token stride taken from the tensor)."""
+        assert k.dtype == _torch().bfloat16 and v.dtype == k.dtype and k.stride() == v.stride()
+        assert k.shape[0] >= n_frames * self.tokens_per_frame and k.stride(2) == 1 and k.stride(1) == HEAD_DIM
+        _check(nomas_kv_commit(self.desc, k.data_ptr(), v.data_ptr(), k.stride(0), n_frames,
+                               _stream_handle(stream)), "nomas_kv_commit")
+
+    def workspace_bytes(self, n_video_frames: int, n_text: int) -> int:
+        return nomas_seg_attn_workspace_bytes(self.desc, n_video_frames, n_text)
+
+    def workspace(self, n_video_frames: int, n_text: int):
+        """A cached device workspace large enough for this call (status header zeroed)."""
+        torch = _torch()
+        need = self.workspace_bytes(n_video_frames, n_text)
+        if self._ws is None or self._ws.numel() < need:
+            self._ws = torch.zeros(max(need, 256), dtype=torch.uint8, device=self.device)
+        return self._ws
+
+    def seg_attn(self, q, k, v, n_video_frames: int, n_text: int, out=None, lse=None, workspace=None,
+                 stream=None):
+        """Segment attention; q, k, v BF16 [Nq][heads][128] sharing one token stride. Returns out."""
+        torch = _torch()
+        nq = n_video_frames * self.tokens_per_frame + n_text
+        for t in (q, k, v):
+            assert t.dtype == torch.bfloat16 and t.shape[0] == nq and t.stride() == q.stride()
+        assert q.stride(2) == 1 and q.stride(1) == HEAD_DIM
+        if out is None:
+            out = torch.empty((nq, self.heads, HEAD_DIM), dtype=torch.bfloat16, device=q.device)
+        ws = workspace if workspace is not None else self.workspace(n_video_frames, n_text)
+        _check(nomas_seg_attn(self.desc, q.data_ptr(), k.data_ptr(), v.data_ptr(), q.stride(0), n_video_frames,
+                              n_text, out.data_ptr(), lse.data_ptr() if lse is not None else None, ws.data_ptr(),
+                              ws.numel() * ws.element_size(), _stream_handle(stream)), "nomas_seg_attn")
+        return out
+
+    def device_status(self, stream=None) -> int:
+        """Synchronise and read/clear the workspace status header (NOMAS_OK or NOMAS_ERR_DEVICE_TIMEOUT)."""
+        if self._ws is None:
+            return NOMAS_OK
+        return nomas_device_status(self._ws.data_ptr(), _stream_handle(stream))

@@ -1,0 +1,403 @@
+// C ABI of the library (declared in include/nomas.h): argument and state
+// validation, RoPE tables, TMA descriptors, split selection and launches.
+// Every check runs before the first launch, so an error return leaves the
+// stream and the cache untouched.
+#include "nomas_internal.h"
+
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+using namespace nomas;
+
+namespace {
+
+constexpr int kBM = 128;
+constexpr int kAssumedSms = 148;       // split choice is a pure function of the shape
+constexpr size_t kWsHeader = 256;
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+uint64_t fnv(uint64_t h, const void* p, size_t n) {
+    const auto* b = static_cast<const uint8_t*>(p);
+    for (size_t i = 0; i < n; ++i) {
+        h ^= b[i];
+        h *= 0x100000001B3ull;
+    }
+    return h;
+}
+
+uint64_t config_stamp(const nomas_cache* c) {
+    uint64_t h = 0xCBF29CE484222325ull;
+    h = fnv(h, &c->mode, sizeof(int32_t) * 7);
+    h = fnv(h, &c->rope_theta, sizeof(float));
+    h = fnv(h, &c->k, sizeof(void*) * 2);
+    h = fnv(h, &c->k_scale, sizeof(float*) * 2);
+    return h | 1ull; // never 0, so a zeroed descriptor never validates
+}
+
+int validate_config(const nomas_cache* c) {
+    if (!c) return NOMAS_ERR_ARG;
+    if (c->mode != NOMAS_CACHE_BF16 && c->mode != NOMAS_CACHE_INT8) return NOMAS_ERR_ARG;
+    if (c->heads <= 0 || c->head_dim != NOMAS_HEAD_DIM) return NOMAS_ERR_ARG;
+    if (c->grid_h <= 0 || c->grid_w <= 0 || c->grid_h + c->grid_w > NOMAS_MAX_GRID_HW) return NOMAS_ERR_ARG;
+    if (c->capacity_frames <= 0 || c->window_frames < 0) return NOMAS_ERR_ARG;
+    if (c->window_frames > 0 && c->capacity_frames != c->window_frames) return NOMAS_ERR_ARG;
+    if (!(c->rope_theta > 0.0f) || !std::isfinite(c->rope_theta)) return NOMAS_ERR_ARG;
+    const int64_t tpf = static_cast<int64_t>(c->grid_h) * c->grid_w;
+    if (static_cast<int64_t>(c->capacity_frames) * tpf > (int64_t(1) << 31) - 1) return NOMAS_ERR_ARG;
+    if (!c->k || !c->v) return NOMAS_ERR_ARG;
+    if (c->mode == NOMAS_CACHE_INT8 && (!c->k_scale || !c->v_scale)) return NOMAS_ERR_ARG;
+    if (c->mode == NOMAS_CACHE_BF16 && (c->k_scale || c->v_scale)) return NOMAS_ERR_ARG;
+    if (!aligned(c->k, 16) || !aligned(c->v, 16)) return NOMAS_ERR_ALIGN;
+    if (c->mode == NOMAS_CACHE_INT8 && (!aligned(c->k_scale, 16) || !aligned(c->v_scale, 16))) return NOMAS_ERR_ALIGN;
+    return NOMAS_OK;
+}
+
+int validate_state(const nomas_cache* c) {
+    int rc = validate_config(c);
+    if (rc != NOMAS_OK) return rc;
+    if (c->check != config_stamp(c)) return NOMAS_ERR_STATE;
+    if (c->frames_committed < 0 || c->valid_frames < 0 || c->valid_frames > c->capacity_frames)
+        return NOMAS_ERR_STATE;
+    return NOMAS_OK;
+}
+
+// ---------------------------------------------------------------- RoPE tables
+// c, s = fp32 roundings of the double-precision cos/sin of pos * theta^(-2j/d).
+double inv_freq(double theta, int j, int d) { return pow(theta, -2.0 * static_cast<double>(j) / static_cast<double>(d)); }
+
+float2 rope_cs(double pos, double theta, int j, int d) {
+    const double ang = pos * inv_freq(theta, j, d);
+    return make_float2(static_cast<float>(cos(ang)), static_cast<float>(sin(ang)));
+}
+
+// Spatial rows are fixed per (theta, grid); cache the last one per thread.
+struct HwCache {
+    float theta = -1.0f;
+    int gh = -1, gw = -1;
+    float2 hw[NOMAS_MAX_GRID_HW][kHWPairs];
+};
+
+void fill_hw(RopeTab& tab, float theta, int gh, int gw) {
+    thread_local HwCache hc;
+    if (hc.theta != theta || hc.gh != gh || hc.gw != gw) {
+        for (int r = 0; r < gh; ++r)
+            for (int j = 0; j < kHWPairs; ++j) hc.hw[r][j] = rope_cs(static_cast<double>(r), theta, j, 56);
+        for (int col = 0; col < gw; ++col)
+            for (int j = 0; j < kHWPairs; ++j) hc.hw[gh + col][j] = rope_cs(static_cast<double>(col), theta, j, 56);
+        hc.theta = theta;
+        hc.gh = gh;
+        hc.gw = gw;
+    }
+    std::memcpy(tab.hw, hc.hw, sizeof(float2) * kHWPairs * (gh + gw));
+}
+
+void fill_t(RopeTab& tab, float theta, int64_t abs_frame0, int n_frames) {
+    for (int i = 0; i < n_frames; ++i)
+        for (int j = 0; j < kTPairs; ++j) tab.t[i][j] = rope_cs(static_cast<double>(abs_frame0 + i), theta, j, 16);
+}
+
+// ---------------------------------------------------------------- device checks
+int check_device() {
+    static std::mutex mu;
+    static int ok_dev[64] = {0}; // 0 unknown, 1 ok, -1 bad
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return NOMAS_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(mu);
+    if (ok_dev[dev] == 0) {
+        int major = 0, minor = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+            return NOMAS_ERR_CUDA;
+        ok_dev[dev] = (major == 10 && minor == 0) ? 1 : -1;
+    }
+    return ok_dev[dev] == 1 ? NOMAS_OK : NOMAS_ERR_DEVICE;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// 3D BF16 tensor map, 128B swizzle, box {64, b1, b2}; out-of-range rows read as zero.
+bool make_tmap(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t stride1_bytes,
+               uint64_t stride2_bytes, uint32_t b1, uint32_t b2) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {d0, d1, d2};
+    const cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
+    const cuuint32_t box[3] = {64, b1, b2};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------- attention plan
+struct Plan {
+    int64_t tpf, nv, nq, nc;
+    int tiles_c, tiles_q, pairs, splits, tiles_per_split;
+    size_t off_qt, off_kt, off_po, off_pml, total;
+};
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Split count minimising a makespan model: waves x (tiles per split + fixed
+// per-CTA cost), for a 148-SM part with one CTA per SM.
+void choose_splits(int units, int tiles, int& splits, int& tps) {
+    double best = 1e300;
+    splits = 1;
+    tps = tiles > 0 ? tiles : 1;
+    if (tiles <= 0) return;
+    for (int s = 1; s <= 32; ++s) {
+        const int t = (tiles + s - 1) / s;
+        const int s_eff = (tiles + t - 1) / t;
+        if (s > 1 && t < 4) break;
+        const int64_t ctas = static_cast<int64_t>(units) * s_eff;
+        const int64_t waves = (ctas + kAssumedSms - 1) / kAssumedSms;
+        const double cost = static_cast<double>(waves) * (t + 3.0) + (s_eff > 1 ? 2.0 : 0.0);
+        if (cost < best - 1e-9) {
+            best = cost;
+            splits = s_eff;
+            tps = t;
+        }
+    }
+}
+
+Plan make_plan(const nomas_cache* c, int32_t n_video_frames, int32_t n_text) {
+    Plan p{};
+    p.tpf = static_cast<int64_t>(c->grid_h) * c->grid_w;
+    p.nv = static_cast<int64_t>(n_video_frames) * p.tpf;
+    p.nq = p.nv + n_text;
+    p.nc = static_cast<int64_t>(c->valid_frames) * p.tpf;
+    p.tiles_c = static_cast<int>((p.nc + kBM - 1) / kBM);
+    p.tiles_q = static_cast<int>((p.nq + kBM - 1) / kBM);
+    p.pairs = (p.tiles_q + 1) / 2;
+    choose_splits(c->heads * p.pairs, p.tiles_c + p.tiles_q, p.splits, p.tiles_per_split);
+    const size_t qk_bytes = static_cast<size_t>(c->heads) * p.nq * kD * 2;
+    const size_t prow = static_cast<size_t>(p.splits) * c->heads * p.pairs * 2 * kBM;
+    p.off_qt = kWsHeader;
+    p.off_kt = round_up(p.off_qt + qk_bytes, 256);
+    p.off_po = round_up(p.off_kt + qk_bytes, 256);
+    p.off_pml = p.off_po + (p.splits > 1 ? prow * kD * sizeof(float) : 0);
+    p.total = round_up(p.off_pml + (p.splits > 1 ? prow * sizeof(float2) : 0), 256);
+    return p;
+}
+
+} // namespace
+
+extern "C" {
+
+int nomas_cache_reset(nomas_cache* c) {
+    const int rc = validate_config(c);
+    if (rc != NOMAS_OK) return rc;
+    c->frames_committed = 0;
+    c->valid_frames = 0;
+    c->head_slot = 0;
+    c->check = config_stamp(c);
+    return NOMAS_OK;
+}
+
+int nomas_kv_commit(nomas_cache* c, const void* k, const void* v, int64_t token_stride, int32_t n_frames,
+                    void* stream) {
+    int rc = validate_state(c);
+    if (rc != NOMAS_OK) return rc;
+    if (n_frames < 0) return NOMAS_ERR_ARG;
+    if (n_frames == 0) return NOMAS_OK;
+    if (!k || !v) return NOMAS_ERR_ARG;
+    if (token_stride < static_cast<int64_t>(c->heads) * kD || token_stride % 8 != 0) return NOMAS_ERR_ARG;
+    if (!aligned(k, 16) || !aligned(v, 16)) return NOMAS_ERR_ALIGN;
+    const int W = c->window_frames;
+    if (W == 0 && c->frames_committed + n_frames > c->capacity_frames) return NOMAS_ERR_CAPACITY;
+    if ((rc = check_device()) != NOMAS_OK) return rc;
+
+    const int tpf = c->grid_h * c->grid_w;
+    const int first = (W > 0 && n_frames > W) ? n_frames - W : 0;
+    RopeTab tab;
+    fill_hw(tab, c->rope_theta, c->grid_h, c->grid_w);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    for (int f0 = first; f0 < n_frames; f0 += kMaxFramesPerLaunch) {
+        const int nf = (n_frames - f0) < kMaxFramesPerLaunch ? (n_frames - f0) : kMaxFramesPerLaunch;
+        CommitArgs a{};
+        a.k = static_cast<const uint16_t*>(k);
+        a.v = static_cast<const uint16_t*>(v);
+        a.token_stride = token_stride;
+        a.ck = c->k;
+        a.cv = c->v;
+        a.cks = c->k_scale;
+        a.cvs = c->v_scale;
+        a.cap_tok = static_cast<int64_t>(c->capacity_frames) * tpf;
+        a.heads = c->heads;
+        a.tpf = tpf;
+        a.grid_h = c->grid_h;
+        a.grid_w = c->grid_w;
+        a.n_frames = nf;
+        a.in_frame0 = f0;
+        a.abs_frame0 = c->frames_committed + f0;
+        a.window = W;
+        a.int8_mode = c->mode == NOMAS_CACHE_INT8;
+        fill_t(tab, c->rope_theta, a.abs_frame0, nf);
+        if (launch_commit(a, tab, s) != cudaSuccess) return NOMAS_ERR_CUDA;
+    }
+    c->frames_committed += n_frames;
+    if (W > 0) {
+        c->valid_frames = static_cast<int32_t>(c->frames_committed < W ? c->frames_committed : W);
+        c->head_slot = static_cast<int32_t>(c->frames_committed % W);
+    } else {
+        c->valid_frames = static_cast<int32_t>(c->frames_committed);
+        c->head_slot = static_cast<int32_t>(c->frames_committed);
+    }
+    return NOMAS_OK;
+}
+
+size_t nomas_seg_attn_workspace_bytes(const nomas_cache* c, int32_t n_video_frames, int32_t n_text) {
+    if (validate_state(c) != NOMAS_OK || n_video_frames < 0 || n_text < 0) return 0;
+    return make_plan(c, n_video_frames, n_text).total;
+}
+
+int nomas_seg_attn(const nomas_cache* c, const void* q, const void* k, const void* v, int64_t token_stride,
+                   int32_t n_video_frames, int32_t n_text, void* out, float* lse, void* workspace,
+                   size_t workspace_bytes, void* stream) {
+    int rc = validate_state(c);
+    if (rc != NOMAS_OK) return rc;
+    if (n_video_frames < 0 || n_text < 0) return NOMAS_ERR_ARG;
+    const Plan p = make_plan(c, n_video_frames, n_text);
+    if (p.nq == 0) return NOMAS_OK;
+    if (p.nq > (int64_t(1) << 30)) return NOMAS_ERR_ARG;
+    if (!q || !k || !v || !out) return NOMAS_ERR_ARG;
+    if (token_stride < static_cast<int64_t>(c->heads) * kD || token_stride % 8 != 0) return NOMAS_ERR_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16)) return NOMAS_ERR_ALIGN;
+    if (lse && !aligned(lse, 4)) return NOMAS_ERR_ALIGN;
+    if (!workspace || workspace_bytes < p.total) return NOMAS_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return NOMAS_ERR_ALIGN;
+    if ((rc = check_device()) != NOMAS_OK) return rc;
+
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    uint16_t* qt = reinterpret_cast<uint16_t*>(ws + p.off_qt);
+    uint16_t* kt = reinterpret_cast<uint16_t*>(ws + p.off_kt);
+
+    // 1) RoPE + relayout of the current Q and K (video frames in chunks)
+    RopeTab tab;
+    fill_hw(tab, c->rope_theta, c->grid_h, c->grid_w);
+    {
+        int f0 = 0;
+        do {
+            const int nf = (n_video_frames - f0) < kMaxFramesPerLaunch ? (n_video_frames - f0) : kMaxFramesPerLaunch;
+            PrepArgs a{};
+            a.q = static_cast<const uint16_t*>(q);
+            a.k = static_cast<const uint16_t*>(k);
+            a.token_stride = token_stride;
+            a.qt = qt;
+            a.kt = kt;
+            a.heads = c->heads;
+            a.tpf = static_cast<int32_t>(p.tpf);
+            a.grid_h = c->grid_h;
+            a.grid_w = c->grid_w;
+            a.nq = static_cast<int32_t>(p.nq);
+            a.nv = static_cast<int32_t>(p.nv);
+            a.tok0 = static_cast<int32_t>(f0 * p.tpf);
+            const bool last = f0 + nf >= n_video_frames;
+            a.tok1 = last ? static_cast<int32_t>(p.nq) : static_cast<int32_t>((f0 + nf) * p.tpf);
+            a.frame0 = f0;
+            if (nf > 0) fill_t(tab, c->rope_theta, c->frames_committed + f0, nf);
+            if (a.tok1 > a.tok0 && launch_prep(a, tab, s) != cudaSuccess) return NOMAS_ERR_CUDA;
+            f0 += nf;
+            if (last) break;
+        } while (true);
+    }
+
+    // 2) tensor maps
+    CUtensorMap tm_q, tm_kcur, tm_vcur, tm_kc, tm_vc;
+    const uint64_t row_bytes = kD * 2;
+    bool ok = make_tmap(&tm_q, qt, kD, p.nq, c->heads, row_bytes, p.nq * row_bytes, kBM, 1) &&
+              make_tmap(&tm_kcur, kt, kD, p.nq, c->heads, row_bytes, p.nq * row_bytes, kBM, 1) &&
+              make_tmap(&tm_vcur, v, kD, c->heads, p.nq, row_bytes, token_stride * 2, 1, kBM);
+    const int64_t cap_tok = static_cast<int64_t>(c->capacity_frames) * p.tpf;
+    if (c->mode == NOMAS_CACHE_BF16) {
+        const uint64_t nc_ext = p.nc > 0 ? p.nc : 1;
+        ok = ok && make_tmap(&tm_kc, c->k, kD, nc_ext, c->heads, row_bytes, cap_tok * row_bytes, kBM, 1) &&
+             make_tmap(&tm_vc, c->v, kD, nc_ext, c->heads, row_bytes, cap_tok * row_bytes, kBM, 1);
+    } else {
+        tm_kc = tm_q;
+        tm_vc = tm_q;
+    }
+    if (!ok) return NOMAS_ERR_CUDA;
+
+    // 3) attention (+ combine of KV splits)
+    AttnArgs a{};
+    a.heads = c->heads;
+    a.nq = static_cast<int32_t>(p.nq);
+    a.nc = static_cast<int32_t>(p.nc);
+    a.tiles_c = p.tiles_c;
+    a.tiles_q = p.tiles_q;
+    a.pairs = p.pairs;
+    a.splits = p.splits;
+    a.tiles_per_split = p.tiles_per_split;
+    a.cap_tok = cap_tok;
+    a.kc8 = static_cast<const int8_t*>(c->k);
+    a.vc8 = static_cast<const int8_t*>(c->v);
+    a.ksc = c->k_scale;
+    a.vsc = c->v_scale;
+    a.out = static_cast<uint16_t*>(out);
+    a.lse = lse;
+    a.part_o = reinterpret_cast<float*>(ws + p.off_po);
+    a.part_ml = reinterpret_cast<float2*>(ws + p.off_pml);
+    a.err = reinterpret_cast<unsigned*>(ws);
+    a.scale_log2 = static_cast<float>(1.4426950408889634 / sqrt(static_cast<double>(kD)));
+    if (launch_attn(a, c->mode == NOMAS_CACHE_INT8, tm_q, tm_kcur, tm_vcur, tm_kc, tm_vc, s) != cudaSuccess)
+        return NOMAS_ERR_CUDA;
+    if (p.splits > 1) {
+        CombineArgs cb{};
+        cb.heads = c->heads;
+        cb.nq = static_cast<int32_t>(p.nq);
+        cb.pairs = p.pairs;
+        cb.splits = p.splits;
+        cb.part_o = a.part_o;
+        cb.part_ml = a.part_ml;
+        cb.out = a.out;
+        cb.lse = lse;
+        if (launch_combine(cb, s) != cudaSuccess) return NOMAS_ERR_CUDA;
+    }
+    return NOMAS_OK;
+}
+
+int nomas_device_status(void* workspace, void* stream) {
+    if (!workspace) return NOMAS_ERR_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return NOMAS_ERR_CUDA;
+    unsigned word = 0;
+    if (cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) return NOMAS_ERR_CUDA;
+    if (word == 0) return NOMAS_OK;
+    if (cudaMemset(workspace, 0, sizeof(word)) != cudaSuccess) return NOMAS_ERR_CUDA;
+    return NOMAS_ERR_DEVICE_TIMEOUT;
+}
+
+const char* nomas_status_string(int status) {
+    switch (status) {
+    case NOMAS_OK: return "NOMAS_OK";
+    case NOMAS_ERR_ARG: return "NOMAS_ERR_ARG: invalid argument";
+    case NOMAS_ERR_ALIGN: return "NOMAS_ERR_ALIGN: pointer or stride not aligned";
+    case NOMAS_ERR_STATE: return "NOMAS_ERR_STATE: cache descriptor not reset or changed";
+    case NOMAS_ERR_CAPACITY: return "NOMAS_ERR_CAPACITY: full-history cache is full";
+    case NOMAS_ERR_WORKSPACE: return "NOMAS_ERR_WORKSPACE: workspace missing or too small";
+    case NOMAS_ERR_CUDA: return "NOMAS_ERR_CUDA: CUDA call failed";
+    case NOMAS_ERR_DEVICE: return "NOMAS_ERR_DEVICE: current device is not sm_100";
+    case NOMAS_ERR_DEVICE_TIMEOUT: return "NOMAS_ERR_DEVICE_TIMEOUT: a kernel abandoned a bounded wait";
+    default: return "unknown nomas status";
+    }
+}
+
+} // extern "C"

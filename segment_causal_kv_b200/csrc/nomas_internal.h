@@ -1,0 +1,95 @@
+// Internal interface between the C-ABI host code (nomas_host.cu) and the
+// kernel translation units. Not installed; not part of the ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+#include "../../include/nomas.h"
+
+namespace nomas {
+
+constexpr int kD = 128;             // head dimension
+constexpr int kPairs = kD / 2;      // RoPE pairs per head
+constexpr int kTPairs = 8;          // pairs of the t block (dims [0,16))
+constexpr int kHWPairs = 28;        // pairs of the h and w blocks (dims [16,72), [72,128))
+constexpr int kMaxFramesPerLaunch = 128;
+
+// RoPE cos/sin tables handed to kernels as launch arguments (read through the
+// constant bank). t rows are the latent frames one launch touches; hw rows
+// are grid rows [0, grid_h) followed by grid columns [grid_h, grid_h+grid_w).
+struct RopeTab {
+    float2 t[kMaxFramesPerLaunch][kTPairs];
+    float2 hw[NOMAS_MAX_GRID_HW][kHWPairs];
+};
+static_assert(sizeof(RopeTab) <= 30 * 1024, "RoPE table must fit the launch-argument limit");
+
+struct CommitArgs {
+    const uint16_t* k;      // segment K, BF16 bits, token-major
+    const uint16_t* v;      // segment V
+    int64_t token_stride;   // elements between tokens
+    void* ck;               // cache K (int8 codes or BF16 bits), head-major
+    void* cv;
+    float* cks;             // cache K scales (INT8 mode)
+    float* cvs;
+    int64_t cap_tok;        // capacity_frames * tokens_per_frame
+    int32_t heads, tpf, grid_h, grid_w;
+    int32_t n_frames;       // frames written by this launch
+    int32_t in_frame0;      // segment-local index of the first of them
+    int64_t abs_frame0;     // absolute frame index of the first of them
+    int32_t window;         // ring modulus (0: slot = absolute frame)
+    int32_t int8_mode;
+};
+
+struct PrepArgs {
+    const uint16_t* q;      // segment Q, BF16 bits, token-major
+    const uint16_t* k;
+    int64_t token_stride;
+    uint16_t* qt;           // rotated Q, head-major [heads][nq][128]
+    uint16_t* kt;           // rotated K, head-major
+    int32_t heads, tpf, grid_h, grid_w;
+    int32_t nq, nv;         // tokens in the segment, video tokens
+    int32_t tok0, tok1;     // token range handled by this launch
+    int32_t frame0;         // segment-local frame of table row t[0]
+};
+
+struct AttnArgs {
+    int32_t heads;
+    int32_t nq;             // current-segment tokens
+    int32_t nc;             // visible cache tokens
+    int32_t tiles_c;        // ceil(nc / 128)
+    int32_t tiles_q;        // ceil(nq / 128)
+    int32_t pairs;          // Q-tile pairs per head: ceil(ceil(nq/128) / 2)
+    int32_t splits;         // KV splits per (head, pair)
+    int32_t tiles_per_split;
+    int64_t cap_tok;        // cache row stride between heads (INT8 path)
+    const int8_t* kc8;      // INT8 cache codes (INT8 mode)
+    const int8_t* vc8;
+    const float* ksc;       // INT8 cache scales
+    const float* vsc;
+    uint16_t* out;          // [nq][heads][128] BF16
+    float* lse;             // [heads][nq] or null
+    float* part_o;          // [splits][heads][pairs*256][128] fp32 (splits > 1)
+    float2* part_ml;        // [splits][heads][pairs*256] (running max in log2 units, sum)
+    unsigned* err;          // workspace status word
+    float scale_log2;       // log2(e) / sqrt(128)
+};
+
+struct CombineArgs {
+    int32_t heads, nq, pairs, splits;
+    const float* part_o;
+    const float2* part_ml;
+    uint16_t* out;
+    float* lse;
+};
+
+// Kernel launchers (return cudaError_t of the launch).
+cudaError_t launch_commit(const CommitArgs& a, const RopeTab& tab, cudaStream_t s);
+cudaError_t launch_prep(const PrepArgs& a, const RopeTab& tab, cudaStream_t s);
+cudaError_t launch_attn(const AttnArgs& a, bool int8_cache, const CUtensorMap& tm_q, const CUtensorMap& tm_kcur,
+                        const CUtensorMap& tm_vcur, const CUtensorMap& tm_kc, const CUtensorMap& tm_vc,
+                        cudaStream_t s);
+cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s);
+
+} // namespace nomas

@@ -1,0 +1,245 @@
+// HBM-bound kernels of the cache path:
+//  * commit_kernel: RoPE(K) -> per-(token, head) INT8 quantisation (or BF16
+//    rounding) -> write into the ring-buffer cache; V is quantised unrotated.
+//    (Hy-Nomas model card, "Single-GPU Low-Memory Inference": INT8 KV storage
+//    and an 18-latent-frame history budget; "Segment-Autoregressive Diffusion
+//    Transformer": cached keys/values of earlier segments, 3D RoPE.)
+//  * prep_kernel: RoPE of the current segment's Q and K, BF16 out, relayout
+//    token-major -> head-major for the attention kernel's TMA loads.
+//
+// Work split: a half-warp owns one (token, head) row of 128 elements; each
+// lane moves 16 bytes (8 BF16 = 4 RoPE pairs) with one 128-bit load per
+// tensor. The 16 lanes of a row fall into exactly one RoPE axis block each
+// (lanes 0-1: t, 2-8: h, 9-15: w). Rows are visited in token-major order so
+// reads are contiguous; every row write is one full 128-byte (codes) or
+// 256-byte (BF16) run. The RoPE tables arrive as launch arguments and are
+// staged once per block into shared memory.
+//
+// Commit arithmetic is fixed bit for bit: products and fused multiply-adds
+// use the _rn intrinsics (no contraction freedom), the scale is an IEEE
+// division absmax / 127, codes are round-half-even of an IEEE division.
+#include "nomas_internal.h"
+
+#include <cuda_bf16.h>
+
+namespace nomas {
+
+namespace {
+
+constexpr int kThreads = 256;
+
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+__device__ __forceinline__ uint32_t rne_bf16x2(float lo, float hi) {
+    // round-half-even to BF16 of two finite fp32 values, packed (lo in bits 0-15)
+    uint32_t a = __float_as_uint(lo), b = __float_as_uint(hi);
+    a = (a + 0x7FFFu + ((a >> 16) & 1u)) >> 16;
+    b = (b + 0x7FFFu + ((b >> 16) & 1u)) >> 16;
+    return a | (b << 16);
+}
+
+// Stage the RoPE rows a block needs into shared memory.
+__device__ __forceinline__ void stage_tables(const RopeTab& tab, int n_t, int n_hw, float2* s_t, float2* s_hw) {
+    for (int i = threadIdx.x; i < n_t * kTPairs; i += blockDim.x) s_t[i] = tab.t[i / kTPairs][i % kTPairs];
+    for (int i = threadIdx.x; i < n_hw * kHWPairs; i += blockDim.x) s_hw[i] = tab.hw[i / kHWPairs][i % kHWPairs];
+    __syncthreads();
+}
+
+// cos/sin of the 4 pairs a lane owns (pairs 4*l .. 4*l+3 of the head).
+__device__ __forceinline__ void lane_coeffs(int l, int frame, int hh, int ww, int grid_h, const float2* s_t,
+                                            const float2* s_hw, float2 (&cs)[4]) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int p = 4 * l + i;
+        if (l < 2)
+            cs[i] = s_t[frame * kTPairs + p];
+        else if (l < 9)
+            cs[i] = s_hw[hh * kHWPairs + (p - kTPairs)];
+        else
+            cs[i] = s_hw[(grid_h + ww) * kHWPairs + (p - kTPairs - kHWPairs)];
+    }
+}
+
+// y0 = fma(x0, c, -rn(x1*s)), y1 = fma(x0, s, rn(x1*c)) on 4 pairs.
+__device__ __forceinline__ void rotate8(const uint4 x, const float2 (&cs)[4], float (&y)[8]) {
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float x0 = bf16lo(w[i]), x1 = bf16hi(w[i]);
+        const float c = cs[i].x, s = cs[i].y;
+        y[2 * i] = __fmaf_rn(x0, c, -__fmul_rn(x1, s));
+        y[2 * i + 1] = __fmaf_rn(x0, s, __fmul_rn(x1, c));
+    }
+}
+
+__device__ __forceinline__ void unpack8(const uint4 x, float (&y)[8]) {
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        y[2 * i] = bf16lo(w[i]);
+        y[2 * i + 1] = bf16hi(w[i]);
+    }
+}
+
+// Half-warp INT8 quantisation of one row: returns 8 packed codes of this lane
+// and the row scale. Both half-warps of a warp must call it together.
+__device__ __forceinline__ uint2 quantize8(const float (&y)[8], float& scale_out) {
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(y[i]));
+#pragma unroll
+    for (int off = 8; off >= 1; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off, 16));
+    uint32_t b[8];
+    if (amax == 0.0f) {
+        scale_out = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) b[i] = 0;
+    } else {
+        const float scale = __fdiv_rn(amax, 127.0f);
+        scale_out = scale;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            int q = __float2int_rn(__fdiv_rn(y[i], scale));
+            q = max(-127, min(127, q));
+            b[i] = static_cast<uint32_t>(q) & 0xFFu;
+        }
+    }
+    uint2 r;
+    r.x = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
+    r.y = b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24);
+    return r;
+}
+
+__global__ void __launch_bounds__(kThreads) commit_kernel(const __grid_constant__ CommitArgs a,
+                                                          const __grid_constant__ RopeTab tab) {
+    __shared__ float2 s_t[kMaxFramesPerLaunch * kTPairs];
+    __shared__ float2 s_hw[NOMAS_MAX_GRID_HW * kHWPairs];
+    stage_tables(tab, a.n_frames, a.grid_h + a.grid_w, s_t, s_hw);
+
+    const int lane = threadIdx.x & 31;
+    const int half = lane >> 4;
+    const int l = lane & 15;
+    const int64_t rows = static_cast<int64_t>(a.n_frames) * a.tpf * a.heads;
+    const int64_t warps = static_cast<int64_t>(gridDim.x) * (kThreads / 32);
+    for (int64_t wp = static_cast<int64_t>(blockIdx.x) * (kThreads / 32) + (threadIdx.x >> 5); wp * 2 < rows;
+         wp += warps) {
+        const int64_t r = wp * 2 + half;
+        const bool valid = r < rows;
+        const int64_t rr = valid ? r : rows - 1;
+        const int64_t tok = rr / a.heads;
+        const int h = static_cast<int>(rr % a.heads);
+        const int fi = static_cast<int>(tok / a.tpf);
+        const int rif = static_cast<int>(tok % a.tpf);
+        const int64_t in_tok = static_cast<int64_t>(a.in_frame0 + fi) * a.tpf + rif;
+        const int64_t in_off = in_tok * a.token_stride + h * kD + l * 8;
+        const uint4 kx = __ldg(reinterpret_cast<const uint4*>(a.k + in_off));
+        const uint4 vx = __ldg(reinterpret_cast<const uint4*>(a.v + in_off));
+
+        float2 cs[4];
+        lane_coeffs(l, fi, rif / a.grid_w, rif % a.grid_w, a.grid_h, s_t, s_hw, cs);
+        float ky[8], vy[8];
+        rotate8(kx, cs, ky);
+        unpack8(vx, vy);
+
+        const int64_t absf = a.abs_frame0 + fi;
+        const int64_t slot = a.window > 0 ? absf % a.window : absf;
+        const int64_t row = static_cast<int64_t>(h) * a.cap_tok + slot * a.tpf + rif;
+        if (a.int8_mode) {
+            float ks, vs;
+            const uint2 kc = quantize8(ky, ks);
+            const uint2 vc = quantize8(vy, vs);
+            if (valid) {
+                *reinterpret_cast<uint2*>(static_cast<int8_t*>(a.ck) + row * kD + l * 8) = kc;
+                *reinterpret_cast<uint2*>(static_cast<int8_t*>(a.cv) + row * kD + l * 8) = vc;
+                if (l == 0) {
+                    a.cks[row] = ks;
+                    a.cvs[row] = vs;
+                }
+            }
+        } else if (valid) {
+            uint4 ko;
+            ko.x = rne_bf16x2(ky[0], ky[1]);
+            ko.y = rne_bf16x2(ky[2], ky[3]);
+            ko.z = rne_bf16x2(ky[4], ky[5]);
+            ko.w = rne_bf16x2(ky[6], ky[7]);
+            *reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.ck) + row * kD + l * 8) = ko;
+            *reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.cv) + row * kD + l * 8) = vx;
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kThreads) prep_kernel(const __grid_constant__ PrepArgs a,
+                                                        const __grid_constant__ RopeTab tab) {
+    __shared__ float2 s_t[kMaxFramesPerLaunch * kTPairs];
+    __shared__ float2 s_hw[NOMAS_MAX_GRID_HW * kHWPairs];
+    const int vid_lo = a.tok0 < a.nv ? a.tok0 : a.nv;
+    const int vid_hi = a.tok1 < a.nv ? a.tok1 : a.nv;
+    const int n_t = vid_hi > vid_lo ? (vid_hi - 1) / a.tpf - a.frame0 + 1 : 0;
+    stage_tables(tab, n_t, a.grid_h + a.grid_w, s_t, s_hw);
+
+    const int lane = threadIdx.x & 31;
+    const int l = lane & 15;
+    const int64_t rows = static_cast<int64_t>(a.tok1 - a.tok0) * a.heads;
+    const int64_t halves = static_cast<int64_t>(gridDim.x) * (kThreads / 16);
+    for (int64_t r = static_cast<int64_t>(blockIdx.x) * (kThreads / 16) + (threadIdx.x >> 4); r < rows;
+         r += halves) {
+        const int tok = a.tok0 + static_cast<int>(r / a.heads);
+        const int h = static_cast<int>(r % a.heads);
+        const int64_t in_off = static_cast<int64_t>(tok) * a.token_stride + h * kD + l * 8;
+        const uint4 qx = __ldg(reinterpret_cast<const uint4*>(a.q + in_off));
+        const uint4 kx = __ldg(reinterpret_cast<const uint4*>(a.k + in_off));
+        uint4 qo = qx, ko = kx;
+        if (tok < a.nv) {
+            const int fi = tok / a.tpf - a.frame0;
+            const int rif = tok % a.tpf;
+            float2 cs[4];
+            lane_coeffs(l, fi, rif / a.grid_w, rif % a.grid_w, a.grid_h, s_t, s_hw, cs);
+            float qy[8], ky[8];
+            rotate8(qx, cs, qy);
+            rotate8(kx, cs, ky);
+            qo.x = rne_bf16x2(qy[0], qy[1]);
+            qo.y = rne_bf16x2(qy[2], qy[3]);
+            qo.z = rne_bf16x2(qy[4], qy[5]);
+            qo.w = rne_bf16x2(qy[6], qy[7]);
+            ko.x = rne_bf16x2(ky[0], ky[1]);
+            ko.y = rne_bf16x2(ky[2], ky[3]);
+            ko.z = rne_bf16x2(ky[4], ky[5]);
+            ko.w = rne_bf16x2(ky[6], ky[7]);
+        }
+        const int64_t out_off = (static_cast<int64_t>(h) * a.nq + tok) * kD + l * 8;
+        *reinterpret_cast<uint4*>(a.qt + out_off) = qo;
+        *reinterpret_cast<uint4*>(a.kt + out_off) = ko;
+    }
+}
+
+int grid_for(int64_t work_items, int items_per_block) {
+    static int sms = 0;
+    if (sms == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (sms <= 0) sms = 148;
+    }
+    int64_t want = (work_items + items_per_block - 1) / items_per_block;
+    const int64_t cap = static_cast<int64_t>(sms) * 8;
+    if (want > cap) want = cap;
+    if (want < 1) want = 1;
+    return static_cast<int>(want);
+}
+
+} // namespace
+
+cudaError_t launch_commit(const CommitArgs& a, const RopeTab& tab, cudaStream_t s) {
+    const int64_t rows = static_cast<int64_t>(a.n_frames) * a.tpf * a.heads;
+    commit_kernel<<<grid_for(rows, kThreads / 16), kThreads, 0, s>>>(a, tab);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_prep(const PrepArgs& a, const RopeTab& tab, cudaStream_t s) {
+    const int64_t rows = static_cast<int64_t>(a.tok1 - a.tok0) * a.heads;
+    prep_kernel<<<grid_for(rows, kThreads / 16), kThreads, 0, s>>>(a, tab);
+    return cudaGetLastError();
+}
+
+} // namespace nomas

@@ -27,6 +27,10 @@ an 18-frame history budget (model card "Single-GPU Low-Memory Inference").
 
 from __future__ import annotations
 
+import ctypes
+import os
+import subprocess
+
 import numpy as np
 
 _GAMMA = np.uint64(0x9E3779B97F4A7C15)
@@ -83,11 +87,41 @@ def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
     return (np.asarray(b, dtype=np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32)
 
 
-def bf16_normal(seed: int, tensor_id: int, shape, std: float = 1.0, segment: int = 0) -> np.ndarray:
-    """BF16 bits (uint16 array of ``shape``) of N(0, std^2) draws."""
+def bf16_normal_numpy(seed: int, tensor_id: int, shape, std: float = 1.0, segment: int = 0) -> np.ndarray:
+    """Pure-numpy statement of the generator (slow; the C version below is used)."""
     n = int(np.prod(shape))
     z = normal_f64(stream_key(seed, tensor_id, segment), n) * std
     return f32_to_bf16_bits(z.astype(np.float32)).reshape(shape)
+
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_CLIB = None
+
+
+def _clib():
+    """gen.c compiled with gcc (same generator, multi-threaded)."""
+    global _CLIB
+    if _CLIB is None:
+        src = os.path.join(_HERE, "gen.c")
+        so = os.path.join(_HERE, "libsynth.so")
+        if not os.path.exists(so) or os.path.getmtime(so) < os.path.getmtime(src):
+            tmp = so + f".{os.getpid()}.tmp"
+            subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-o", tmp, src, "-lm", "-lpthread"])
+            os.replace(tmp, so)
+        lib = ctypes.CDLL(so)
+        lib.synth_bf16_normal.argtypes = [ctypes.c_uint64, ctypes.c_int64, ctypes.c_double, ctypes.c_void_p,
+                                          ctypes.c_int]
+        _CLIB = lib
+    return _CLIB
+
+
+def bf16_normal(seed: int, tensor_id: int, shape, std: float = 1.0, segment: int = 0) -> np.ndarray:
+    """BF16 bits (uint16 array of ``shape``) of N(0, std^2) draws."""
+    n = int(np.prod(shape))
+    out = np.empty(n, np.uint16)
+    key = int(stream_key(seed, tensor_id, segment))
+    _clib().synth_bf16_normal(key, n, float(std), out.ctypes.data_as(ctypes.c_void_p), os.cpu_count() or 1)
+    return out.reshape(shape)
 
 
 class Geometry:

@@ -1,0 +1,158 @@
+"""Parity of nomas_seg_attn (tcgen05 kernels, through the C ABI) with the fp64
+oracle: max-abs error <= 2e-2 and relative L2 error <= 5e-3 on every case,
+from tiny shapes to the full single-GPU configuration (sampled rows)."""
+
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from harness import MAX_ABS, REL_L2, current_segment, errors, make_caches, sample_rows, to_dev, to_f64
+
+pytestmark = pytest.mark.gpu
+
+
+def run_case(w, rows=None, check_lse=True, rel_l2=REL_L2):
+    torch = __import__("torch")
+    gpu, orc = make_caches(w)
+    q, k, v = current_segment(w)
+    nq = q.shape[0]
+    lse = torch.full((w["heads"], nq), float("nan"), dtype=torch.float32, device="cuda")
+    out = torch.full((nq, w["heads"], 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+    gpu.seg_attn(to_dev(q), to_dev(k), to_dev(v), w["cur_frames"], w["n_text"], out=out, lse=lse)
+    torch.cuda.synchronize()
+    assert gpu.device_status() == 0
+    ref, ref_lse = orc.seg_attn(q, k, v, w["cur_frames"], w["n_text"], rows=rows)
+    got = to_f64(out)
+    got_lse = lse.cpu().numpy().astype(np.float64)
+    if rows is not None:
+        got = got[rows]
+        got_lse = got_lse[:, rows]
+    assert np.isfinite(got).all()
+    mx, rel = errors(got, ref)
+    assert mx <= MAX_ABS and rel <= rel_l2, (mx, rel)
+    if check_lse:
+        np.testing.assert_allclose(got_lse, ref_lse, rtol=0, atol=5e-3)
+    return mx, rel
+
+
+def wl(**kw):
+    base = dict(heads=2, grid_h=4, grid_w=8, mode="bf16", window=0, capacity=8, hist_commits=[2], cur_frames=2,
+                n_text=16, seed=0, q_std=1.0, kv_std=1.0)
+    base.update(kw)
+    return base
+
+
+def test_tiny_workload():
+    run_case(synth.WORKLOADS["tiny"])
+
+
+def test_tiny_int8():
+    run_case(wl(mode="int8", window=4, capacity=4, hist_commits=[1, 2]))
+
+
+@pytest.mark.parametrize("mode", ["bf16", "int8"])
+def test_ragged_tiles_and_tails(mode):
+    # 35 tokens/frame, 4 history frames = 140 keys (128 + 12); 5 frames + 37 text = 212 queries (128 + 84)
+    run_case(wl(heads=3, grid_h=5, grid_w=7, mode=mode, window=4 if mode == "int8" else 0,
+                capacity=4 if mode == "int8" else 12, hist_commits=[3, 1], cur_frames=5, n_text=37, seed=5))
+
+
+@pytest.mark.parametrize("mode", ["bf16", "int8"])
+def test_multi_tile_with_kv_splits(mode):
+    # 256 tokens/frame: 1536 cached keys (12 tiles), 868 queries (7 tiles): the split-KV + combine path
+    run_case(wl(heads=4, grid_h=16, grid_w=16, mode=mode, window=6 if mode == "int8" else 0,
+                capacity=6 if mode == "int8" else 10, hist_commits=[2, 2, 2], cur_frames=3, n_text=100, seed=6))
+
+
+def test_no_history():
+    run_case(wl(hist_commits=[], cur_frames=3, n_text=20, seed=7))
+
+
+def test_text_only_segment():
+    run_case(wl(cur_frames=0, n_text=45, seed=8))
+
+
+def test_single_query_token():
+    run_case(wl(hist_commits=[], cur_frames=0, n_text=1, seed=9))
+
+
+def test_video_only_segment_one_token_frames():
+    run_case(wl(heads=2, grid_h=1, grid_w=1, hist_commits=[3], cur_frames=5, n_text=0, seed=10))
+
+
+def test_wrapped_int8_ring():
+    # 7 frames committed through a 3-frame window; the visible history is the last 3
+    run_case(wl(heads=2, grid_h=6, grid_w=8, mode="int8", window=3, capacity=3, hist_commits=[2, 4, 1],
+                cur_frames=2, n_text=10, seed=11))
+
+
+def test_peaky_softmax():
+    """Scores three times larger exercise the running-max rescaling of O.
+
+    The kernel's operands are BF16 (rotated Q and K, dequantised cache, P),
+    each rounded with relative error up to 2^-9. A score error grows with the
+    score's size, and a peaked softmax passes it on to the output almost
+    undamped: with q_std = 3 the expected relative L2 error is about three
+    times the N(0,1) figure (~2e-3 measured), so this stress case is held to
+    rel-L2 <= 1e-2 while keeping the max-abs bound of 2e-2.
+    """
+    run_case(wl(heads=2, grid_h=8, grid_w=16, mode="int8", window=4, capacity=4, hist_commits=[2, 2],
+                cur_frames=2, n_text=30, seed=12, q_std=3.0), rel_l2=1e-2)
+
+
+def test_int8_split_mixing_cache_and_current_tiles():
+    """160 Q-tile pairs x 38 KV tiles: three KV splits, the middle one runs five
+    dequantised cache tiles and then TMA-loaded current-segment tiles."""
+    w = wl(heads=16, grid_h=8, grid_w=16, mode="int8", window=18, capacity=18, hist_commits=[6, 6, 6],
+           cur_frames=19, n_text=64, seed=15)
+    F = 128
+    nq = 19 * F + 64
+    run_case(w, rows=sample_rows(nq, F, 19, per_head=24))
+
+
+def test_repeated_calls_are_deterministic():
+    torch = __import__("torch")
+    w = wl(heads=4, grid_h=16, grid_w=16, mode="int8", window=6, capacity=6, hist_commits=[3, 3], cur_frames=3,
+           n_text=100, seed=13)
+    gpu, _ = make_caches(w, with_oracle=False)
+    q, k, v = [to_dev(x) for x in current_segment(w)]
+    a = gpu.seg_attn(q, k, v, 3, 100).clone()
+    b = gpu.seg_attn(q, k, v, 3, 100)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+
+
+def test_cache_is_read_only():
+    torch = __import__("torch")
+    w = wl(heads=2, grid_h=6, grid_w=8, mode="int8", window=8, capacity=8, hist_commits=[2], cur_frames=2,
+           n_text=8, seed=14)
+    gpu, _ = make_caches(w, with_oracle=False)
+    before = (gpu.k.clone(), gpu.v.clone(), gpu.k_scale.clone(), gpu.v_scale.clone())
+    q, k, v = [to_dev(x) for x in current_segment(w)]
+    gpu.seg_attn(q, k, v, 2, 8)
+    torch.cuda.synchronize()
+    for a, b in zip(before, (gpu.k, gpu.v, gpu.k_scale, gpu.v_scale)):
+        assert torch.equal(a, b)
+    assert gpu.frames_committed == 2
+
+
+def test_single_gpu_configuration_sampled_rows():
+    w = synth.WORKLOADS["single_gpu_int8_18f"]
+    F = w["grid_h"] * w["grid_w"]
+    nq = w["cur_frames"] * F + w["n_text"]
+    rows = sample_rows(nq, F, w["cur_frames"], per_head=48)
+    mx, rel = run_case(w, rows=rows)
+    print(f"single-GPU cfg: max-abs {mx:.3e} rel-L2 {rel:.3e}")
+
+
+@pytest.mark.slow
+def test_full_history_bf16_sampled_rows():
+    w = synth.WORKLOADS["full_history_bf16"]
+    F = w["grid_h"] * w["grid_w"]
+    nq = w["cur_frames"] * F + w["n_text"]
+    rows = sample_rows(nq, F, w["cur_frames"], per_head=12)
+    mx, rel = run_case(w, rows=rows)
+    print(f"full-history BF16: max-abs {mx:.3e} rel-L2 {rel:.3e}")

@@ -1,0 +1,105 @@
+"""Bit-exact parity of nomas_kv_commit (CUDA, through the C ABI) with the
+oracle's commit: INT8 codes, fp32 scales (as bit patterns), BF16 cache
+values, slot placement and the host counters."""
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from harness import make_caches, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def assert_cache_equal(gpu, orc):
+    torch = __import__("torch")
+    torch.cuda.synchronize()
+    if gpu.mode == "int8":
+        assert np.array_equal(gpu.k.cpu().numpy(), orc.k_code)
+        assert np.array_equal(gpu.v.cpu().numpy(), orc.v_code)
+        assert np.array_equal(gpu.k_scale.cpu().numpy().view(np.uint32), orc.k_scale.view(np.uint32))
+        assert np.array_equal(gpu.v_scale.cpu().numpy().view(np.uint32), orc.v_scale.view(np.uint32))
+    else:
+        assert np.array_equal(gpu.k.cpu().view(torch.int16).numpy().view(np.uint16), orc.k_bf16)
+        assert np.array_equal(gpu.v.cpu().view(torch.int16).numpy().view(np.uint16), orc.v_bf16)
+    assert gpu.frames_committed == orc.frames_committed
+    assert gpu.valid_frames == orc.valid_frames
+
+
+def test_commit_int8_eighteen_frame_history_bit_exact():
+    w = synth.WORKLOADS["single_gpu_int8_18f"]
+    gpu, orc = make_caches(w)
+    assert_cache_equal(gpu, orc)
+    assert gpu.valid_frames == 18 and gpu.head_slot == 0
+
+
+@pytest.mark.parametrize("mode", ["int8", "bf16"])
+def test_commit_ring_wraps_and_long_commits(mode):
+    W = 4
+    geo = synth.Geometry(3, 5, 7)
+    import segment_causal_kv_b200 as nm
+    gpu = nm.KVCache(mode, 3, 5, 7, W, W)
+    orc = oracle.OracleCache(oracle.MODE_INT8 if mode == "int8" else oracle.MODE_BF16, 3, 5, 7, W, W)
+    for s, nf in enumerate([3, 2, 5, 1, 9, 4]):
+        k, v = synth.history_kv(geo, nf, 90, s)
+        gpu.commit(to_dev(k), to_dev(v), nf)
+        orc.commit(k, v, nf)
+        assert_cache_equal(gpu, orc)
+        assert gpu.head_slot == gpu.frames_committed % W
+
+
+def test_commit_bf16_full_history_and_capacity():
+    geo = synth.Geometry(2, 4, 8)
+    import segment_causal_kv_b200 as nm
+    gpu = nm.KVCache("bf16", 2, 4, 8, 0, 6)
+    orc = oracle.OracleCache(oracle.MODE_BF16, 2, 4, 8, 0, 6)
+    for s, nf in enumerate([2, 3, 1]):
+        k, v = synth.history_kv(geo, nf, 91, s)
+        gpu.commit(to_dev(k), to_dev(v), nf)
+        orc.commit(k, v, nf)
+    assert_cache_equal(gpu, orc)
+    k, v = synth.history_kv(geo, 1, 91, 9)
+    with pytest.raises(nm.NomasError) as e:
+        gpu.commit(to_dev(k), to_dev(v), 1)
+    assert e.value.status == nm.NOMAS_ERR_CAPACITY
+
+
+def test_commit_with_padded_token_stride_and_zero_rows():
+    torch = __import__("torch")
+    import segment_causal_kv_b200 as nm
+    H, gh, gw = 4, 3, 6
+    geo = synth.Geometry(H, gh, gw)
+    k, v = synth.history_kv(geo, 2, 92, 0)
+    k[5, 1, :] = 0          # an all-zero (token, head) row: scale 0, codes 0
+    v[7, :, :] = 0
+    k[9, 2, 3] = 0x8000     # negative zero
+    n = k.shape[0]
+    pad = 64
+    kb = torch.zeros((n, H * 128 + pad), dtype=torch.bfloat16, device="cuda")
+    vb = torch.zeros_like(kb)
+    kb[:, :H * 128] = to_dev(k).reshape(n, H * 128)
+    vb[:, :H * 128] = to_dev(v).reshape(n, H * 128)
+    kv = kb[:, :H * 128].view(n, H, 128)
+    vv = vb[:, :H * 128].view(n, H, 128)
+    assert kv.stride(0) == H * 128 + pad
+    gpu = nm.KVCache("int8", H, gh, gw, 3, 3)
+    gpu.commit(kv, vv, 2)
+    orc = oracle.OracleCache(oracle.MODE_INT8, H, gh, gw, 3, 3)
+    orc.commit(k, v, 2)
+    assert_cache_equal(gpu, orc)
+    F = gh * gw
+    assert gpu.k_scale[1, 5].item() == 0.0 and not gpu.k[1, 5].any()
+
+
+def test_commit_large_segment_spans_several_launches():
+    # 130 frames of a 2x2 grid: more frames than one launch's RoPE table holds
+    import segment_causal_kv_b200 as nm
+    geo = synth.Geometry(2, 2, 2)
+    gpu = nm.KVCache("int8", 2, 2, 2, 0, 140)
+    orc = oracle.OracleCache(oracle.MODE_INT8, 2, 2, 2, 0, 140)
+    for s, nf in enumerate([5, 130]):
+        k, v = synth.history_kv(geo, nf, 93, s)
+        gpu.commit(to_dev(k), to_dev(v), nf)
+        orc.commit(k, v, nf)
+    assert_cache_equal(gpu, orc)
