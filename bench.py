@@ -174,11 +174,14 @@ def cpu_baseline(w):
     orc, q, k, v = oracle_setup(w)
     _, nq, _, _, _ = workload_shape(w)
     rng = np.random.default_rng(0)
-    probe = np.sort(rng.choice(nq, 8, replace=False))
-    _, dt, _ = oracle_rate(orc, q, k, v, w, probe, nthreads)
-    n = int(np.clip(8 * 12.0 / max(dt, 1e-3), 8, nq))
-    rows = np.sort(rng.choice(nq, n, replace=False))
-    rate, dt, flop = oracle_rate(orc, q, k, v, w, rows, nthreads)
+    # grow the row sample until one timed call takes >= 10 s of host time
+    n = 16
+    while True:
+        rows = np.sort(rng.choice(nq, n, replace=False))
+        rate, dt, flop = oracle_rate(orc, q, k, v, w, rows, nthreads)
+        if dt >= 10.0 or n >= nq:
+            break
+        n = int(min(nq, max(2 * n, n * 12.0 / max(dt, 1e-3))))
     return {"value": rate, "unit": "TFLOP/s", "cores": nthreads, "kind": "oracle",
             "sample": f"{n} query rows x {w['heads']} heads of the {WORKLOAD} workload (fp64 two-pass softmax over "
                       f"all {workload_shape(w)[3]} keys), {dt:.1f} s, {flop / 1e9:.1f} GFLOP"}

@@ -34,7 +34,8 @@ def run_case(w, rows=None, check_lse=True, rel_l2=REL_L2):
     mx, rel = errors(got, ref)
     assert mx <= MAX_ABS and rel <= rel_l2, (mx, rel)
     if check_lse:
-        np.testing.assert_allclose(got_lse, ref_lse, rtol=0, atol=5e-3)
+        # the log-sum-exp carries the score error of BF16 operands, which grows with |score|
+        np.testing.assert_allclose(got_lse, ref_lse, rtol=2.0 ** -8, atol=5e-3)
     return mx, rel
 
 
