@@ -13,7 +13,8 @@
 // (lanes 0-1: t, 2-8: h, 9-15: w). Rows are visited in token-major order so
 // reads are contiguous; every row write is one full 128-byte (codes) or
 // 256-byte (BF16) run. The RoPE tables arrive as launch arguments and are
-// staged once per block into shared memory.
+// staged once per block into shared memory; the grid is persistent (two
+// blocks per SM) so the staging is paid a few hundred times, not per row.
 //
 // Commit arithmetic is fixed bit for bit: products and fused multiply-adds
 // use the _rn intrinsics (no contraction freedom), the scale is an IEEE
@@ -26,7 +27,7 @@ namespace nomas {
 
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;
 
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
@@ -221,8 +222,9 @@ int grid_for(int64_t work_items, int items_per_block) {
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         if (sms <= 0) sms = 148;
     }
+    // a persistent grid: every block stages the RoPE rows once and then loops
     int64_t want = (work_items + items_per_block - 1) / items_per_block;
-    const int64_t cap = static_cast<int64_t>(sms) * 8;
+    const int64_t cap = static_cast<int64_t>(sms) * 2;
     if (want > cap) want = cap;
     if (want < 1) want = 1;
     return static_cast<int>(want);

@@ -44,7 +44,7 @@ constexpr int BN = 128;
 constexpr int kStages = 2;
 constexpr uint32_t kTileBytes = BM * kD * 2; // one BF16 128x128 tile
 constexpr uint32_t kHalfBytes = kTileBytes / 2;
-constexpr float kRescaleThreshold = 8.0f;
+constexpr float kRescaleThreshold = 8.0f; // P <= 2^8 between rescales
 
 // shared memory map (offsets from a 1024-byte aligned base)
 constexpr uint32_t kOffQ = 0;                                // 2 tiles
@@ -84,10 +84,95 @@ __device__ __forceinline__ uint64_t desc_mnmajor(uint32_t tile, int kk) {
     return smem_desc(tile + kk * 2048, kHalfBytes, 1024, kSwizzle128B);
 }
 
-__device__ __forceinline__ float dq(uint32_t biased_word, int byte, float scale) {
-    // byte of an offset-binary word -> exact float code -> times scale
-    const float f = __uint_as_float(__byte_perm(biased_word, 0x4B000000u, 0x7540u + byte)) - 8388736.0f;
-    return f * scale;
+// 8 INT8 codes -> 8 BF16 values code * scale. A code c is read exactly as the
+// float 2^23 + (c + 128) (the byte of c ^ 0x80 placed under the exponent of 2^23),
+// minus 2^23 + 128, then scaled in fp32 and rounded once to BF16.
+__device__ __forceinline__ uint4 dequant8(uint2 w, float scale) {
+    const uint32_t w0 = w.x ^ 0x80808080u, w1 = w.y ^ 0x80808080u;
+    const float2 bias = make_float2(-8388736.0f, -8388736.0f);
+    const float2 sc = make_float2(scale, scale);
+    uint32_t out[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const uint32_t src = q < 2 ? w0 : w1;
+        const uint32_t b = (q & 1) * 2;
+        float2 f = make_float2(__uint_as_float(__byte_perm(src, 0x4B000000u, 0x7540u + b)),
+                               __uint_as_float(__byte_perm(src, 0x4B000000u, 0x7541u + b)));
+        f = __fmul2_rn(__fadd2_rn(f, bias), sc);
+        out[q] = pack_bf16x2(f.x, f.y);
+    }
+    return make_uint4(out[0], out[1], out[2], out[3]);
+}
+
+// 64 columns of packed P from registers into TMEM (one row per thread).
+__device__ __forceinline__ void tmem_st_p64(uint32_t taddr, const uint32_t (&r)[64]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x64.b32 [%0], "
+        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+        "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, "
+        "%33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, "
+        "%49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63, %64};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+        "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+        "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31]), "r"(r[32]),
+        "r"(r[33]), "r"(r[34]), "r"(r[35]), "r"(r[36]), "r"(r[37]), "r"(r[38]), "r"(r[39]), "r"(r[40]),
+        "r"(r[41]), "r"(r[42]), "r"(r[43]), "r"(r[44]), "r"(r[45]), "r"(r[46]), "r"(r[47]), "r"(r[48]),
+        "r"(r[49]), "r"(r[50]), "r"(r[51]), "r"(r[52]), "r"(r[53]), "r"(r[54]), "r"(r[55]), "r"(r[56]),
+        "r"(r[57]), "r"(r[58]), "r"(r[59]), "r"(r[60]), "r"(r[61]), "r"(r[62]), "r"(r[63])
+        : "memory");
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+// Maximum of one 128-key S row over its valid columns (kMask: columns >= vc ignored).
+template <bool kMask>
+__device__ __forceinline__ float row_max(uint32_t t_s, int vc) {
+    float mx = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+        uint32_t s[64];
+        tmem_ld64(t_s + c * 64, s);
+#pragma unroll
+        for (int e = 0; e < 64; ++e) {
+            const float x = __uint_as_float(s[e]);
+            mx = (!kMask || c * 64 + e < vc) ? fmaxf(mx, x) : mx;
+        }
+    }
+    return mx;
+}
+
+// P = 2^(s * scale_log2 - m) of one 128-key S row, written as packed BF16 pairs
+// over the first 64 columns of the row's S block (a 64-column chunk of S is in
+// registers before the P columns over it are written). Returns the fp32 sum.
+template <bool kMask>
+__device__ __forceinline__ float row_exp_store(uint32_t t_s, float sl2, float m, int vc) {
+    const float2 sl2x2 = make_float2(sl2, sl2);
+    const float2 negm = make_float2(-m, -m);
+    float2 sum2 = make_float2(0.0f, 0.0f);
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+        uint32_t s[64];
+        tmem_ld64(t_s + c * 64, s);
+        uint32_t p[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+            float2 x = __ffma2_rn(make_float2(__uint_as_float(s[2 * e]), __uint_as_float(s[2 * e + 1])), sl2x2, negm);
+            if (kMask) {
+                const int col = c * 64 + 2 * e;
+                x.x = col < vc ? x.x : -INFINITY;
+                x.y = col + 1 < vc ? x.y : -INFINITY;
+            }
+            const float p0 = ex2_approx(x.x), p1 = ex2_approx(x.y);
+            sum2 = __fadd2_rn(sum2, make_float2(p0, p1));
+            p[e] = pack_bf16x2(p0, p1);
+        }
+        tmem_st32(t_s + c * 32, p);
+    }
+    return sum2.x + sum2.y;
 }
 
 // Arm stage `st` for tile t and issue its K and V loads (4 TMA boxes).
@@ -289,19 +374,10 @@ __global__ void __launch_bounds__(kInt8 ? 512 : 384, 1)
                 if (!(ok = mbar_wait(bar(B_SFULL + w), i & 1, ctl))) break;
                 tc_fence_after();
                 const int vc = tile_valid(a, t_begin + i);
-                // pass 1: row max of the raw scores
-                float mx = -INFINITY;
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t s[32];
-                    tmem_ld32(t_s + c * 32, s);
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const float x = __uint_as_float(s[e]);
-                        mx = (c * 32 + e < vc) ? fmaxf(mx, x) : mx;
-                    }
-                }
-                const float mxl = mx * sl2;
+                const bool full = (vc == BN);
+                // pass 1: tile max; the reference max moves only when it is exceeded
+                // by more than the threshold (then O is rescaled in TMEM)
+                const float mxl = (full ? row_max<false>(t_s, vc) : row_max<true>(t_s, vc)) * sl2;
                 const bool resc = mxl > m_ref + kRescaleThreshold;
                 const float m_new = resc ? mxl : m_ref;
                 const float alpha = resc ? ex2_approx(m_ref - m_new) : 1.0f; // 0 on the first tile
@@ -310,7 +386,7 @@ __global__ void __launch_bounds__(kInt8 ? 512 : 384, 1)
                     for (int c = 0; c < 4; ++c) {
                         uint32_t o[32];
                         tmem_ld32(t_o + c * 32, o);
-    #pragma unroll
+#pragma unroll
                         for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
                         tmem_st32(t_o + c * 32, o);
                     }
@@ -318,32 +394,8 @@ __global__ void __launch_bounds__(kInt8 ? 512 : 384, 1)
                 }
                 l *= alpha;
                 m_ref = m_new;
-                // pass 2: P = 2^(s*scale - m), BF16, into the first 64 columns of S
-                const float neg_m = -m_ref;
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t s[32];
-                    tmem_ld32(t_s + c * 32, s);
-                    uint32_t p[16];
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const int col = c * 32 + 2 * e;
-                        float p0 = ex2_approx(fmaf(__uint_as_float(s[2 * e]), sl2, neg_m));
-                        float p1 = ex2_approx(fmaf(__uint_as_float(s[2 * e + 1]), sl2, neg_m));
-                        p0 = col < vc ? p0 : 0.0f;
-                        p1 = col + 1 < vc ? p1 : 0.0f;
-                        l += p0 + p1;
-                        p[e] = pack_bf16x2(p0, p1);
-                    }
-                    // P columns [16c, 16c+16): S columns below 32(c+1) are already in registers
-                    asm volatile(
-                        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
-                        "%11, %12, %13, %14, %15, %16};" ::"r"(t_s + c * 16),
-                        "r"(p[0]), "r"(p[1]), "r"(p[2]), "r"(p[3]), "r"(p[4]), "r"(p[5]), "r"(p[6]), "r"(p[7]),
-                        "r"(p[8]), "r"(p[9]), "r"(p[10]), "r"(p[11]), "r"(p[12]), "r"(p[13]), "r"(p[14]),
-                        "r"(p[15])
-                        : "memory");
-                }
+                // pass 2: P into TMEM, row sum in fp32
+                l += full ? row_exp_store<false>(t_s, sl2, m_ref, vc) : row_exp_store<true>(t_s, sl2, m_ref, vc);
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
@@ -362,7 +414,7 @@ __global__ void __launch_bounds__(kInt8 ? 512 : 384, 1)
                     for (int c = 0; c < 4; ++c) {
                         uint32_t o[32];
                         tmem_ld32(t_o + c * 32, o);
-                            uint32_t b[16];
+                        uint32_t b[16];
 #pragma unroll
                         for (int e = 0; e < 16; ++e)
                             b[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
@@ -374,7 +426,8 @@ __global__ void __launch_bounds__(kInt8 ? 512 : 384, 1)
                             d4[3] = make_uint4(b[12], b[13], b[14], b[15]);
                         }
                     }
-                    if (row_ok && a.lse) a.lse[static_cast<int64_t>(head) * a.nq + qrow] = (m_ref + log2f(l)) * 0.69314718055994531f;
+                    if (row_ok && a.lse)
+                        a.lse[static_cast<int64_t>(head) * a.nq + qrow] = (m_ref + log2f(l)) * 0.69314718055994531f;
                 } else {
                     const int64_t prow = (static_cast<int64_t>(split) * a.heads + head) * (a.pairs * 2 * BM) +
                                          static_cast<int64_t>(pair) * 2 * BM + w * BM + r;
@@ -383,7 +436,7 @@ __global__ void __launch_bounds__(kInt8 ? 512 : 384, 1)
                     for (int c = 0; c < 4; ++c) {
                         uint32_t o[32];
                         tmem_ld32(t_o + c * 32, o);
-                            if (row_ok) {
+                        if (row_ok) {
                             uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
 #pragma unroll
                             for (int e = 0; e < 8; ++e) d4[e] = make_uint4(o[4 * e], o[4 * e + 1], o[4 * e + 2], o[4 * e + 3]);
@@ -394,12 +447,42 @@ __global__ void __launch_bounds__(kInt8 ? 512 : 384, 1)
             }
         }
     } else if (kInt8 && warp >= 12) {
-        // ================================================================ INT8 dequantiser
+        // ================================================================ INT8 filler
+        // Warp wq converts rows [32 wq, 32 wq + 32) of a cache tile; in step j a
+        // warp covers rows 2j and 2j+1, 16 lanes per row, 8 codes per lane, so a
+        // lane writes exactly one 16-byte BF16 chunk and each quarter-warp hits 8
+        // distinct chunk slots of the swizzled row (no bank conflicts). The next
+        // cache tile's codes are loaded into registers as soon as the current
+        // tile has been converted, so global latency overlaps the MMA pipeline.
         const int wq = warp - 12;
-        const int sub = lane >> 3;   // row inside a group of 4
-        const int chunk = lane & 7;  // 16-code chunk of the row
+        const int half = lane >> 4;
+        const int l16 = lane & 15;
         const bool elected = (wq == 0 && lane == 0);
+        const uint32_t chunk_off = (l16 >> 3) * kHalfBytes;
+        uint2 kb[16], vb[16];
+        float ks_own = 0.0f, vs_own = 0.0f; // scales of row 2*l16 + half of this warp's block
+        // row (32 wq + 2j + half) of a tile: (row & 7) = (2j & 7) ^ half, so the swizzled
+        // chunk slot is slot0 ^ (2j & 7) and the byte offset is a constant per j
+        const uint32_t slot0 = static_cast<uint32_t>((l16 & 7) ^ half);
+        const uint32_t row_off0 = chunk_off + static_cast<uint32_t>(wq * 32 + half) * 128u;
+        auto load_tile = [&](int t) {
+            const int key0 = t * BN + wq * 32 + half;
+            const int64_t grow0 = static_cast<int64_t>(head) * a.cap_tok + key0;
+            const uint2* kp = reinterpret_cast<const uint2*>(a.kc8 + grow0 * kD) + l16;
+            const uint2* vp = reinterpret_cast<const uint2*>(a.vc8 + grow0 * kD) + l16;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const bool in = key0 + 2 * j < a.nc;
+                kb[j] = in ? __ldg(kp + j * 32) : make_uint2(0u, 0u); // 2 rows = 256 B = 32 uint2
+                vb[j] = in ? __ldg(vp + j * 32) : make_uint2(0u, 0u);
+            }
+            const int skey = t * BN + wq * 32 + 2 * l16 + half;
+            const bool sin_ = skey < a.nc;
+            ks_own = sin_ ? __ldg(a.ksc + static_cast<int64_t>(head) * a.cap_tok + skey) : 0.0f;
+            vs_own = sin_ ? __ldg(a.vsc + static_cast<int64_t>(head) * a.cap_tok + skey) : 0.0f;
+        };
         int armed_phase[kStages] = {-1, -1};
+        if (t_begin < a.tiles_c) load_tile(t_begin);
         for (int i = 0; i < n; ++i) {
             const int t = t_begin + i;
             const int st = i % kStages;
@@ -421,42 +504,15 @@ __global__ void __launch_bounds__(kInt8 ? 512 : 384, 1)
                 }
                 continue;
             }
-#pragma unroll 2
-            for (int it = 0; it < 8; ++it) {
-                const int row = wq * 32 + it * 4 + sub;
-                const int key = t * BN + row;
-                uint4 kc = make_uint4(0, 0, 0, 0), vcw = make_uint4(0, 0, 0, 0);
-                float ks = 0.0f, vs = 0.0f;
-                if (key < a.nc) {
-                    const int64_t grow = static_cast<int64_t>(head) * a.cap_tok + key;
-                    kc = __ldg(reinterpret_cast<const uint4*>(a.kc8 + grow * kD) + chunk);
-                    vcw = __ldg(reinterpret_cast<const uint4*>(a.vc8 + grow * kD) + chunk);
-                    ks = __ldg(a.ksc + grow);
-                    vs = __ldg(a.vsc + grow);
-                }
-                const uint32_t kw[4] = {kc.x ^ 0x80808080u, kc.y ^ 0x80808080u, kc.z ^ 0x80808080u, kc.w ^ 0x80808080u};
-                const uint32_t vw[4] = {vcw.x ^ 0x80808080u, vcw.y ^ 0x80808080u, vcw.z ^ 0x80808080u,
-                                        vcw.w ^ 0x80808080u};
-                uint32_t kb[8], vb[8];
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    kb[2 * q] = pack_bf16x2(dq(kw[q], 0, ks), dq(kw[q], 1, ks));
-                    kb[2 * q + 1] = pack_bf16x2(dq(kw[q], 2, ks), dq(kw[q], 3, ks));
-                    vb[2 * q] = pack_bf16x2(dq(vw[q], 0, vs), dq(vw[q], 1, vs));
-                    vb[2 * q + 1] = pack_bf16x2(dq(vw[q], 2, vs), dq(vw[q], 3, vs));
-                }
-#pragma unroll
-                for (int hc = 0; hc < 2; ++hc) {
-                    const int c8 = 2 * chunk + hc; // 8-dim chunk, 0..15
-                    const uint32_t off = (c8 >> 3) * kHalfBytes + row * 128 + (((c8 & 7) ^ (row & 7)) << 4);
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(ktile + off), "r"(kb[4 * hc]),
-                                 "r"(kb[4 * hc + 1]), "r"(kb[4 * hc + 2]), "r"(kb[4 * hc + 3])
-                                 : "memory");
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(vtile + off), "r"(vb[4 * hc]),
-                                 "r"(vb[4 * hc + 1]), "r"(vb[4 * hc + 2]), "r"(vb[4 * hc + 3])
-                                 : "memory");
-                }
+            for (int j = 0; j < 16; ++j) {
+                const float ks = __shfl_sync(0xFFFFFFFFu, ks_own, half * 16 + j);
+                const float vs = __shfl_sync(0xFFFFFFFFu, vs_own, half * 16 + j);
+                const uint32_t off = row_off0 + j * 256u + ((slot0 ^ static_cast<uint32_t>((2 * j) & 7)) << 4);
+                st_shared_v4(ktile + off, dequant8(kb[j], ks));
+                st_shared_v4(vtile + off, dequant8(vb[j], vs));
             }
+            if (t + 1 < a.tiles_c && i + 1 < n) load_tile(t + 1);
             fence_proxy_async_smem();
             named_bar_sync(1, 128);
             if (elected) {
