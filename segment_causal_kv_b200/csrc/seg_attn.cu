@@ -104,31 +104,25 @@ __device__ __forceinline__ uint4 dequant8(uint2 w, float scale) {
     return make_uint4(out[0], out[1], out[2], out[3]);
 }
 
-// 64 columns of packed P from registers into TMEM (one row per thread).
-__device__ __forceinline__ void tmem_st_p64(uint32_t taddr, const uint32_t (&r)[64]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x64.b32 [%0], "
-        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
-        "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, "
-        "%33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, "
-        "%49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63, %64};" ::"r"(taddr),
-        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
-        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
-        "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
-        "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31]), "r"(r[32]),
-        "r"(r[33]), "r"(r[34]), "r"(r[35]), "r"(r[36]), "r"(r[37]), "r"(r[38]), "r"(r[39]), "r"(r[40]),
-        "r"(r[41]), "r"(r[42]), "r"(r[43]), "r"(r[44]), "r"(r[45]), "r"(r[46]), "r"(r[47]), "r"(r[48]),
-        "r"(r[49]), "r"(r[50]), "r"(r[51]), "r"(r[52]), "r"(r[53]), "r"(r[54]), "r"(r[55]), "r"(r[56]),
-        "r"(r[57]), "r"(r[58]), "r"(r[59]), "r"(r[60]), "r"(r[61]), "r"(r[62]), "r"(r[63])
-        : "memory");
-}
-
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
                  : "memory");
 }
 
-// Maximum of one 128-key S row over its valid columns (kMask: columns >= vc ignored).
+// 16 columns of 32-bit values from registers into TMEM (one row per thread).
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]) : "memory");
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// Maximum of one 128-key S row over its valid columns (kMask: columns >= vc
+// ignored). Eight independent accumulators keep the reduction off a single
+// dependency chain.
 template <bool kMask>
 __device__ __forceinline__ float row_max(uint32_t t_s, int vc) {
     float mx = -INFINITY;
@@ -136,43 +130,112 @@ __device__ __forceinline__ float row_max(uint32_t t_s, int vc) {
     for (int c = 0; c < 2; ++c) {
         uint32_t s[64];
         tmem_ld64(t_s + c * 64, s);
+        float m[8];
 #pragma unroll
-        for (int e = 0; e < 64; ++e) {
-            const float x = __uint_as_float(s[e]);
-            mx = (!kMask || c * 64 + e < vc) ? fmaxf(mx, x) : mx;
+        for (int k = 0; k < 8; ++k) m[k] = mx;
+#pragma unroll
+        for (int e = 0; e < 64; e += 2) {
+            float x0 = __uint_as_float(s[e]), x1 = __uint_as_float(s[e + 1]);
+            if (kMask) {
+                x0 = (c * 64 + e < vc) ? x0 : -INFINITY;
+                x1 = (c * 64 + e + 1 < vc) ? x1 : -INFINITY;
+            }
+            m[(e >> 1) & 7] = max3(m[(e >> 1) & 7], x0, x1);
         }
+        mx = max3(max3(m[0], m[1], m[2]), max3(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
+        // keep this chunk's reduction ahead of the next TMEM load, so its 64
+        // registers are dead before the next 64 arrive
+        asm volatile("" : "+f"(mx));
     }
     return mx;
 }
 
 // P = 2^(s * scale_log2 - m) of one 128-key S row, written as packed BF16 pairs
-// over the first 64 columns of the row's S block (a 64-column chunk of S is in
-// registers before the P columns over it are written). Returns the fp32 sum.
+// over the first 64 columns of the row's S block (a 32-column chunk of S is in
+// registers before the 16 P columns over it are written). Returns the fp32
+// sum, accumulated in four independent packed pairs.
 template <bool kMask>
 __device__ __forceinline__ float row_exp_store(uint32_t t_s, float sl2, float m, int vc) {
     const float2 sl2x2 = make_float2(sl2, sl2);
     const float2 negm = make_float2(-m, -m);
-    float2 sum2 = make_float2(0.0f, 0.0f);
+    float2 acc[4];
 #pragma unroll
-    for (int c = 0; c < 2; ++c) {
-        uint32_t s[64];
-        tmem_ld64(t_s + c * 64, s);
-        uint32_t p[32];
+    for (int k = 0; k < 4; ++k) acc[k] = make_float2(0.0f, 0.0f);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
+    for (int c = 0; c < 4; ++c) {
+        uint32_t s[32];
+        tmem_ld32(t_s + c * 32, s);
+        uint32_t p[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
             float2 x = __ffma2_rn(make_float2(__uint_as_float(s[2 * e]), __uint_as_float(s[2 * e + 1])), sl2x2, negm);
             if (kMask) {
-                const int col = c * 64 + 2 * e;
+                const int col = c * 32 + 2 * e;
                 x.x = col < vc ? x.x : -INFINITY;
                 x.y = col + 1 < vc ? x.y : -INFINITY;
             }
             const float p0 = ex2_approx(x.x), p1 = ex2_approx(x.y);
-            sum2 = __fadd2_rn(sum2, make_float2(p0, p1));
+            acc[e & 3] = __fadd2_rn(acc[e & 3], make_float2(p0, p1));
             p[e] = pack_bf16x2(p0, p1);
         }
-        tmem_st32(t_s + c * 32, p);
+        tmem_st16(t_s + c * 16, p);
     }
-    return sum2.x + sum2.y;
+    const float2 t = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+    return t.x + t.y;
+}
+
+// Cold paths kept out of line, so they do not add to the register pressure of
+// the per-tile loop: tail tiles (masked), O rescaling, the epilogues.
+__device__ __noinline__ float row_max_masked(uint32_t t_s, int vc) { return row_max<true>(t_s, vc); }
+__device__ __noinline__ float row_exp_store_masked(uint32_t t_s, float sl2, float m, int vc) {
+    return row_exp_store<true>(t_s, sl2, m, vc);
+}
+
+// O *= alpha for one row (one thread), in TMEM.
+__device__ __noinline__ void rescale_o(uint32_t t_o, float alpha) {
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+        uint32_t o[32];
+        tmem_ld32(t_o + c * 32, o);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+        tmem_st32(t_o + c * 32, o);
+        tmem_st_wait();
+    }
+}
+
+// Final output row: O / l -> BF16 (all lanes load from TMEM; only valid rows store).
+__device__ __noinline__ void store_out_row(uint32_t t_o, float inv_l, uint16_t* dst, bool row_ok) {
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+        uint32_t o[32];
+        tmem_ld32(t_o + c * 32, o);
+        uint32_t b[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+            b[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
+        if (row_ok) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+            d4[0] = make_uint4(b[0], b[1], b[2], b[3]);
+            d4[1] = make_uint4(b[4], b[5], b[6], b[7]);
+            d4[2] = make_uint4(b[8], b[9], b[10], b[11]);
+            d4[3] = make_uint4(b[12], b[13], b[14], b[15]);
+        }
+    }
+}
+
+// Partial row: unnormalised fp32 O.
+__device__ __noinline__ void store_partial_row(uint32_t t_o, float* dst, bool row_ok) {
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+        uint32_t o[32];
+        tmem_ld32(t_o + c * 32, o);
+        if (row_ok) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) d4[e] = make_uint4(o[4 * e], o[4 * e + 1], o[4 * e + 2], o[4 * e + 3]);
+        }
+    }
 }
 
 // Arm stage `st` for tile t and issue its K and V loads (4 TMA boxes).
@@ -377,25 +440,15 @@ __global__ void __launch_bounds__(kInt8 ? 512 : 384, 1)
                 const bool full = (vc == BN);
                 // pass 1: tile max; the reference max moves only when it is exceeded
                 // by more than the threshold (then O is rescaled in TMEM)
-                const float mxl = (full ? row_max<false>(t_s, vc) : row_max<true>(t_s, vc)) * sl2;
+                const float mxl = (full ? row_max<false>(t_s, vc) : row_max_masked(t_s, vc)) * sl2;
                 const bool resc = mxl > m_ref + kRescaleThreshold;
                 const float m_new = resc ? mxl : m_ref;
                 const float alpha = resc ? ex2_approx(m_ref - m_new) : 1.0f; // 0 on the first tile
-                if (i > 0 && __any_sync(0xFFFFFFFFu, resc)) {
-#pragma unroll 1
-                    for (int c = 0; c < 4; ++c) {
-                        uint32_t o[32];
-                        tmem_ld32(t_o + c * 32, o);
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                        tmem_st32(t_o + c * 32, o);
-                    }
-                    tmem_st_wait();
-                }
+                if (i > 0 && __any_sync(0xFFFFFFFFu, resc)) rescale_o(t_o, alpha);
                 l *= alpha;
                 m_ref = m_new;
                 // pass 2: P into TMEM, row sum in fp32
-                l += full ? row_exp_store<false>(t_s, sl2, m_ref, vc) : row_exp_store<true>(t_s, sl2, m_ref, vc);
+                l += full ? row_exp_store<false>(t_s, sl2, m_ref, vc) : row_exp_store_masked(t_s, sl2, m_ref, vc);
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
@@ -408,40 +461,13 @@ __global__ void __launch_bounds__(kInt8 ? 512 : 384, 1)
                 const int qrow = (qt0 + w) * BM + r;
                 const bool row_ok = qrow < a.nq;
                 if (a.splits == 1) {
-                    const float inv_l = 1.0f / l;
-                    uint16_t* dst = a.out + (static_cast<int64_t>(qrow) * a.heads + head) * kD;
-#pragma unroll 1
-                    for (int c = 0; c < 4; ++c) {
-                        uint32_t o[32];
-                        tmem_ld32(t_o + c * 32, o);
-                        uint32_t b[16];
-#pragma unroll
-                        for (int e = 0; e < 16; ++e)
-                            b[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
-                        if (row_ok) {
-                            uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
-                            d4[0] = make_uint4(b[0], b[1], b[2], b[3]);
-                            d4[1] = make_uint4(b[4], b[5], b[6], b[7]);
-                            d4[2] = make_uint4(b[8], b[9], b[10], b[11]);
-                            d4[3] = make_uint4(b[12], b[13], b[14], b[15]);
-                        }
-                    }
+                    store_out_row(t_o, 1.0f / l, a.out + (static_cast<int64_t>(qrow) * a.heads + head) * kD, row_ok);
                     if (row_ok && a.lse)
                         a.lse[static_cast<int64_t>(head) * a.nq + qrow] = (m_ref + log2f(l)) * 0.69314718055994531f;
                 } else {
                     const int64_t prow = (static_cast<int64_t>(split) * a.heads + head) * (a.pairs * 2 * BM) +
                                          static_cast<int64_t>(pair) * 2 * BM + w * BM + r;
-                    float* dst = a.part_o + prow * kD;
-#pragma unroll 1
-                    for (int c = 0; c < 4; ++c) {
-                        uint32_t o[32];
-                        tmem_ld32(t_o + c * 32, o);
-                        if (row_ok) {
-                            uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) d4[e] = make_uint4(o[4 * e], o[4 * e + 1], o[4 * e + 2], o[4 * e + 3]);
-                        }
-                    }
+                    store_partial_row(t_o, a.part_o + prow * kD, row_ok);
                     if (row_ok) a.part_ml[prow] = make_float2(m_ref, l);
                 }
             }
