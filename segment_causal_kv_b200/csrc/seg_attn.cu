@@ -58,8 +58,9 @@ enum {
     B_QFULL = 0,
     B_KFULL = 1,                // + stage
     B_VFULL = B_KFULL + kStages,
-    B_KVEMPTY = B_VFULL + kStages,
-    B_SFULL = B_KVEMPTY + kStages, // + softmax warpgroup
+    B_KEMPTY = B_VFULL + kStages,  // K and V stages are released separately: K as soon
+    B_VEMPTY = B_KEMPTY + kStages, // as the S MMAs that read it are done, V after P.V
+    B_SFULL = B_VEMPTY + kStages,  // + softmax warpgroup
     B_PFULL = B_SFULL + 2,
     B_OFULL = B_PFULL + 2,
     B_DRAIN = B_OFULL + 2,
@@ -238,34 +239,41 @@ __device__ __noinline__ void store_partial_row(uint32_t t_o, float* dst, bool ro
     }
 }
 
-// Arm stage `st` for tile t and issue its K and V loads (4 TMA boxes).
-__device__ __forceinline__ void load_kv_tile(const AttnArgs& a, int t, int head, uint32_t kdst, uint32_t vdst,
-                                             uint32_t kbar, uint32_t vbar, const CUtensorMap* tm_kc,
-                                             const CUtensorMap* tm_vc, const CUtensorMap* tm_kcur,
-                                             const CUtensorMap* tm_vcur) {
+// Arm a K (or V) stage for tile t and issue its two TMA boxes.
+__device__ __forceinline__ void load_k_tile(const AttnArgs& a, int t, int head, uint32_t kdst, uint32_t kbar,
+                                            const CUtensorMap* tm_kc, const CUtensorMap* tm_kcur) {
     mbar_arrive_expect_tx(kbar, kTileBytes);
-    mbar_arrive_expect_tx(vbar, kTileBytes);
     if (t < a.tiles_c) {
         tma_load_3d(kdst, tm_kc, 0, t * BN, head, kbar);
         tma_load_3d(kdst + kHalfBytes, tm_kc, 64, t * BN, head, kbar);
-        tma_load_3d(vdst, tm_vc, 0, t * BN, head, vbar);
-        tma_load_3d(vdst + kHalfBytes, tm_vc, 64, t * BN, head, vbar);
     } else {
         const int row = (t - a.tiles_c) * BN;
         tma_load_3d(kdst, tm_kcur, 0, row, head, kbar);
         tma_load_3d(kdst + kHalfBytes, tm_kcur, 64, row, head, kbar);
+    }
+}
+
+__device__ __forceinline__ void load_v_tile(const AttnArgs& a, int t, int head, uint32_t vdst, uint32_t vbar,
+                                            const CUtensorMap* tm_vc, const CUtensorMap* tm_vcur) {
+    mbar_arrive_expect_tx(vbar, kTileBytes);
+    if (t < a.tiles_c) {
+        tma_load_3d(vdst, tm_vc, 0, t * BN, head, vbar);
+        tma_load_3d(vdst + kHalfBytes, tm_vc, 64, t * BN, head, vbar);
+    } else {
+        const int row = (t - a.tiles_c) * BN;
         tma_load_3d(vdst, tm_vcur, 0, head, row, vbar);
         tma_load_3d(vdst + kHalfBytes, tm_vcur, 64, head, row, vbar);
     }
 }
 
-// Bounded wait for the last armed phase of each stage: no copy may still be
-// in flight when the CTA exits (matters only after an abort).
-__device__ __forceinline__ void drain_armed(const int (&armed_phase)[kStages], uint32_t kfull0, uint32_t vfull0) {
+// Bounded wait for the last armed phase of each K and V stage: no copy may
+// still be in flight when the CTA exits (matters only after an abort).
+__device__ __forceinline__ void drain_armed(const int (&k_armed)[kStages], const int (&v_armed)[kStages],
+                                            uint32_t kfull0, uint32_t vfull0) {
     for (int st = 0; st < kStages; ++st) {
-        if (armed_phase[st] < 0) continue;
         const uint64_t t0 = global_timer_ns();
-        while (!mbar_try_wait(kfull0 + 8u * st, armed_phase[st]) || !mbar_try_wait(vfull0 + 8u * st, armed_phase[st])) {
+        while ((k_armed[st] >= 0 && !mbar_try_wait(kfull0 + 8u * st, k_armed[st])) ||
+               (v_armed[st] >= 0 && !mbar_try_wait(vfull0 + 8u * st, v_armed[st]))) {
             if (global_timer_ns() - t0 > NOMAS_WAIT_NS) break;
         }
     }
@@ -308,7 +316,8 @@ __global__ void __launch_bounds__(kInt8 ? 512 : 384, 1)
         for (int s = 0; s < kStages; ++s) {
             mbar_init(bar(B_KFULL + s), 1);
             mbar_init(bar(B_VFULL + s), 1);
-            mbar_init(bar(B_KVEMPTY + s), 1);
+            mbar_init(bar(B_KEMPTY + s), 1);
+            mbar_init(bar(B_VEMPTY + s), 1);
         }
         for (int w = 0; w < 2; ++w) {
             mbar_init(bar(B_SFULL + w), 1);
@@ -349,15 +358,20 @@ __global__ void __launch_bounds__(kInt8 ? 512 : 384, 1)
             // (codes for cache tiles, TMA for current-segment tiles): with a single
             // filler in tile order every parity wait on the stage ring is exact.
             if (!kInt8) {
-                int armed_phase[kStages] = {-1, -1};
+                int k_armed[kStages] = {-1, -1}, v_armed[kStages] = {-1, -1};
                 for (int i = 0; i < n; ++i) {
                     const int st = i % kStages;
-                    if (i >= kStages && !mbar_wait(bar(B_KVEMPTY + st), ((i / kStages) & 1) ^ 1, ctl)) break;
-                    load_kv_tile(a, t_begin + i, head, sbase + kOffK + st * kTileBytes, sbase + kOffV + st * kTileBytes,
-                                 bar(B_KFULL + st), bar(B_VFULL + st), &tm_kc, &tm_vc, &tm_kcur, &tm_vcur);
-                    armed_phase[st] = (i / kStages) & 1;
+                    const uint32_t free_ph = ((i / kStages) & 1) ^ 1;
+                    if (i >= kStages && !mbar_wait(bar(B_KEMPTY + st), free_ph, ctl)) break;
+                    load_k_tile(a, t_begin + i, head, sbase + kOffK + st * kTileBytes, bar(B_KFULL + st), &tm_kc,
+                                &tm_kcur);
+                    k_armed[st] = (i / kStages) & 1;
+                    if (i >= kStages && !mbar_wait(bar(B_VEMPTY + st), free_ph, ctl)) break;
+                    load_v_tile(a, t_begin + i, head, sbase + kOffV + st * kTileBytes, bar(B_VFULL + st), &tm_vc,
+                                &tm_vcur);
+                    v_armed[st] = (i / kStages) & 1;
                 }
-                drain_armed(armed_phase, bar(B_KFULL), bar(B_VFULL));
+                drain_armed(k_armed, v_armed, bar(B_KFULL), bar(B_VFULL));
             }
         }
     } else if (warp == 1) {
@@ -391,6 +405,8 @@ __global__ void __launch_bounds__(kInt8 ? 512 : 384, 1)
                     issue_s(w, 0);
                     mma_commit(bar(B_SFULL + w));
                 }
+                // K of tile 0 is free once these S MMAs finish (a fill of tile 2 waits for it)
+                if (kStages < n) mma_commit(bar(B_KEMPTY + 0));
             }
             for (int i = 0; ok && i < n; ++i) {
                 const int st = i % kStages;
@@ -404,10 +420,13 @@ __global__ void __launch_bounds__(kInt8 ? 512 : 384, 1)
                     if (!(ok = mbar_wait(bar(B_PFULL + w), i & 1, ctl))) break;
                     tc_fence_after();
                     issue_pv(w, st, i == 0);
-                    if (w == nq_tiles - 1 && !last) mma_commit(bar(B_KVEMPTY + st));
+                    // each release is committed only when a later fill waits for it,
+                    // so no arrival is left pending at exit
+                    if (w == nq_tiles - 1 && i + kStages < n) mma_commit(bar(B_VEMPTY + st));
                     if (!last) {
                         issue_s(w, st1);
                         mma_commit(bar(B_SFULL + w));
+                        if (w == nq_tiles - 1 && i + 1 + kStages < n) mma_commit(bar(B_KEMPTY + st1));
                     } else {
                         mma_commit(bar(B_OFULL + w));
                     }
@@ -491,62 +510,75 @@ __global__ void __launch_bounds__(kInt8 ? 512 : 384, 1)
         // chunk slot is slot0 ^ (2j & 7) and the byte offset is a constant per j
         const uint32_t slot0 = static_cast<uint32_t>((l16 & 7) ^ half);
         const uint32_t row_off0 = chunk_off + static_cast<uint32_t>(wq * 32 + half) * 128u;
-        auto load_tile = [&](int t) {
+        auto load_codes = [&](const int8_t* base, const float* scales, int t, uint2 (&buf)[16], float& sc_own) {
             const int key0 = t * BN + wq * 32 + half;
             const int64_t grow0 = static_cast<int64_t>(head) * a.cap_tok + key0;
-            const uint2* kp = reinterpret_cast<const uint2*>(a.kc8 + grow0 * kD) + l16;
-            const uint2* vp = reinterpret_cast<const uint2*>(a.vc8 + grow0 * kD) + l16;
+            const uint2* p = reinterpret_cast<const uint2*>(base + grow0 * kD) + l16;
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
                 const bool in = key0 + 2 * j < a.nc;
-                kb[j] = in ? __ldg(kp + j * 32) : make_uint2(0u, 0u); // 2 rows = 256 B = 32 uint2
-                vb[j] = in ? __ldg(vp + j * 32) : make_uint2(0u, 0u);
+                buf[j] = in ? __ldg(p + j * 32) : make_uint2(0u, 0u); // 2 rows = 256 B = 32 uint2
             }
             const int skey = t * BN + wq * 32 + 2 * l16 + half;
-            const bool sin_ = skey < a.nc;
-            ks_own = sin_ ? __ldg(a.ksc + static_cast<int64_t>(head) * a.cap_tok + skey) : 0.0f;
-            vs_own = sin_ ? __ldg(a.vsc + static_cast<int64_t>(head) * a.cap_tok + skey) : 0.0f;
+            sc_own = skey < a.nc ? __ldg(scales + static_cast<int64_t>(head) * a.cap_tok + skey) : 0.0f;
         };
-        int armed_phase[kStages] = {-1, -1};
-        if (t_begin < a.tiles_c) load_tile(t_begin);
+        auto convert = [&](uint32_t tile, const uint2 (&buf)[16], float sc_own) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const float sc = __shfl_sync(0xFFFFFFFFu, sc_own, half * 16 + j);
+                const uint32_t off = row_off0 + j * 256u + ((slot0 ^ static_cast<uint32_t>((2 * j) & 7)) << 4);
+                st_shared_v4(tile + off, dequant8(buf[j], sc));
+            }
+        };
+        // one elected thread waits; the group learns the outcome after a named
+        // barrier, so all 128 threads take the same branch
+        auto group_wait = [&](uint32_t barrier, uint32_t parity) -> bool {
+            if (elected) *dq_go = mbar_wait(barrier, parity, ctl) ? 1 : 0;
+            named_bar_sync(1, 128);
+            return *dq_go != 0;
+        };
+        int k_armed[kStages] = {-1, -1}, v_armed[kStages] = {-1, -1};
+        if (t_begin < a.tiles_c) {
+            load_codes(a.kc8, a.ksc, t_begin, kb, ks_own);
+            load_codes(a.vc8, a.vsc, t_begin, vb, vs_own);
+        }
         for (int i = 0; i < n; ++i) {
             const int t = t_begin + i;
             const int st = i % kStages;
-            if (i >= kStages) {
-                // one elected thread waits; the group learns the outcome after a
-                // named barrier, so all 128 threads take the same branch
-                if (elected) *dq_go = mbar_wait(bar(B_KVEMPTY + st), ((i / kStages) & 1) ^ 1, ctl) ? 1 : 0;
-                named_bar_sync(1, 128);
-                if (!*dq_go) break;
-            }
+            const uint32_t free_ph = ((i / kStages) & 1) ^ 1;
             const uint32_t ktile = sbase + kOffK + st * kTileBytes;
             const uint32_t vtile = sbase + kOffV + st * kTileBytes;
+            const bool next_cached = (t + 1 < a.tiles_c && i + 1 < n);
+            // ---- K (freed early: right after the S MMAs of tile i - 2)
+            if (i >= kStages && !group_wait(bar(B_KEMPTY + st), free_ph)) break;
             if (t >= a.tiles_c) {
-                // current-segment tile: BF16 already, one TMA issue by the elected thread
                 if (elected) {
-                    load_kv_tile(a, t, head, ktile, vtile, bar(B_KFULL + st), bar(B_VFULL + st), &tm_kc, &tm_vc,
-                                 &tm_kcur, &tm_vcur);
-                    armed_phase[st] = (i / kStages) & 1;
+                    load_k_tile(a, t, head, ktile, bar(B_KFULL + st), &tm_kc, &tm_kcur);
+                    k_armed[st] = (i / kStages) & 1;
                 }
-                continue;
+            } else {
+                convert(ktile, kb, ks_own);
+                if (next_cached) load_codes(a.kc8, a.ksc, t + 1, kb, ks_own);
+                fence_proxy_async_smem();
+                named_bar_sync(1, 128);
+                if (elected) mbar_arrive(bar(B_KFULL + st));
             }
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                const float ks = __shfl_sync(0xFFFFFFFFu, ks_own, half * 16 + j);
-                const float vs = __shfl_sync(0xFFFFFFFFu, vs_own, half * 16 + j);
-                const uint32_t off = row_off0 + j * 256u + ((slot0 ^ static_cast<uint32_t>((2 * j) & 7)) << 4);
-                st_shared_v4(ktile + off, dequant8(kb[j], ks));
-                st_shared_v4(vtile + off, dequant8(vb[j], vs));
-            }
-            if (t + 1 < a.tiles_c && i + 1 < n) load_tile(t + 1);
-            fence_proxy_async_smem();
-            named_bar_sync(1, 128);
-            if (elected) {
-                mbar_arrive(bar(B_KFULL + st));
-                mbar_arrive(bar(B_VFULL + st));
+            // ---- V (freed after the P.V MMAs of tile i - 2)
+            if (i >= kStages && !group_wait(bar(B_VEMPTY + st), free_ph)) break;
+            if (t >= a.tiles_c) {
+                if (elected) {
+                    load_v_tile(a, t, head, vtile, bar(B_VFULL + st), &tm_vc, &tm_vcur);
+                    v_armed[st] = (i / kStages) & 1;
+                }
+            } else {
+                convert(vtile, vb, vs_own);
+                if (next_cached) load_codes(a.vc8, a.vsc, t + 1, vb, vs_own);
+                fence_proxy_async_smem();
+                named_bar_sync(1, 128);
+                if (elected) mbar_arrive(bar(B_VFULL + st));
             }
         }
-        if (elected) drain_armed(armed_phase, bar(B_KFULL), bar(B_VFULL));
+        if (elected) drain_armed(k_armed, v_armed, bar(B_KFULL), bar(B_VFULL));
     }
 
     // ---- teardown
