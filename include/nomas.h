@@ -187,6 +187,32 @@ int nomas_seg_attn(const nomas_cache *c, const void *q, const void *k, const voi
  */
 int nomas_device_status(void *workspace, void *stream);
 
+/*
+ * nomas_seg_attn_static -- nomas_seg_attn for callers that cannot allocate
+ * device memory. The pages have no counterpart to this call: it is a service
+ * of this library. Some callers cannot provide the device workspace that
+ * nomas_seg_attn needs: an operator plugin whose host framework passes it
+ * only its inputs and outputs, or code running where a cudaMalloc would
+ * synchronise the device or fail because all device memory is already
+ * reserved. This call takes its scratch from a fixed array in the library's
+ * device image instead: NOMAS_STATIC_SCRATCH_BYTES per GPU, held by every GPU
+ * that loads the library until the process exits.
+ *
+ * Arguments, layouts, results and errors are those of nomas_seg_attn, minus
+ * the workspace. A shape whose workspace (nomas_seg_attn_workspace_bytes)
+ * exceeds NOMAS_STATIC_SCRATCH_BYTES is rejected with NOMAS_ERR_WORKSPACE
+ * before anything is enqueued. The call allocates and frees nothing.
+ * The first call on a device (with that device current) sets the array up:
+ * it looks up its device address and clears its status header, a blocking
+ * step; make that first call before any stream capture. All calls share the
+ * one array and it keeps the last call's contents, so calls that overlap on
+ * the GPU race with each other: order them (one stream, or events). Device
+ * timeouts of this call are not reported through nomas_device_status.
+ */
+#define NOMAS_STATIC_SCRATCH_BYTES (64u << 20)
+int nomas_seg_attn_static(const nomas_cache *c, const void *q, const void *k, const void *v, int64_t token_stride,
+                          int32_t n_video_frames, int32_t n_text, void *out, float *lse, void *stream);
+
 /* Human-readable name of a status code (static storage). */
 const char *nomas_status_string(int status);
 

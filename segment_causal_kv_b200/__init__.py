@@ -35,7 +35,8 @@ HEAD_DIM = 128
 
 # exported symbols (checked against include/nomas.h by the tests)
 EXPORTS = ("nomas_cache_reset", "nomas_kv_commit", "nomas_seg_attn_workspace_bytes", "nomas_seg_attn",
-           "nomas_device_status", "nomas_status_string")
+           "nomas_device_status", "nomas_status_string", "nomas_seg_attn_static")
+NOMAS_STATIC_SCRATCH_BYTES = 64 << 20
 
 
 class NomasCacheDesc(ctypes.Structure):
@@ -89,6 +90,8 @@ def lib():
         L.nomas_seg_attn.restype = ctypes.c_int
         L.nomas_device_status.argtypes = [P, P]
         L.nomas_device_status.restype = ctypes.c_int
+        L.nomas_seg_attn_static.argtypes = [D, P, P, P, I64, I32, I32, P, P, P]
+        L.nomas_seg_attn_static.restype = ctypes.c_int
         L.nomas_status_string.argtypes = [ctypes.c_int]
         L.nomas_status_string.restype = ctypes.c_char_p
         _lib = L
@@ -119,6 +122,14 @@ def nomas_seg_attn(desc: NomasCacheDesc, q_ptr: int, k_ptr: int, v_ptr: int, tok
                    ws_bytes: int, stream: int | None) -> int:
     return lib().nomas_seg_attn(ctypes.byref(desc), q_ptr, k_ptr, v_ptr, token_stride, n_video_frames, n_text,
                                 out_ptr, lse_ptr, ws_ptr, ws_bytes, stream)
+
+
+def nomas_seg_attn_static(desc: NomasCacheDesc, q_ptr: int, k_ptr: int, v_ptr: int, token_stride: int,
+                          n_video_frames: int, n_text: int, out_ptr: int, lse_ptr: int | None,
+                          stream: int | None) -> int:
+    """nomas_seg_attn with the library's static scratch, for callers that cannot allocate a workspace."""
+    return lib().nomas_seg_attn_static(ctypes.byref(desc), q_ptr, k_ptr, v_ptr, token_stride, n_video_frames,
+                                       n_text, out_ptr, lse_ptr, stream)
 
 
 def nomas_device_status(ws_ptr: int, stream: int | None) -> int:
