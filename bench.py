@@ -52,6 +52,8 @@ def parse():
     p.add_argument("--impl", default="nomas", choices=["nomas", "reference"])
     p.add_argument("--e2e-steps", type=int, default=0, help="end-to-end steps (default: min(steps, 100))")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--workload", default=WORKLOAD,
+                   help=f"{WORKLOAD} (default: the headline line), commit_72f_int8, history_sweep, layers54_turn")
     return p.parse_args()
 
 
@@ -231,6 +233,133 @@ def run_reference(args, rank, world):
 # GPU arm
 # ---------------------------------------------------------------------------
 
+def traffic_from_profile(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, or None when the
+    kernel's source changed since those counters were taken."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        rec = json.load(open(path))[kernel]
+    except Exception:
+        return None
+    h = hashlib.sha256()
+    for f in rec["sources"]:
+        h.update(open(os.path.join(ROOT, f), "rb").read())
+    return rec["dram_bytes_per_launch"] if h.hexdigest() == rec["sources_sha256"] else None
+
+
+def device_events(torch, n):
+    return [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+
+
+def run_extra(args, torch, nm, dev):
+    """Secondary workloads (one JSON line each): large commit, history sweep, 54-layer turn."""
+    to_dev = lambda b: torch.from_numpy(np.ascontiguousarray(b).view(np.int16)).view(torch.bfloat16).to(dev)
+    flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    peaks, peak_src = load_peaks()
+    geo = synth.Geometry(16, 22, 40)
+    F = geo.tokens_per_frame
+    K, W = args.steps, args.warmup
+    if args.workload == "commit_72f_int8":
+        # one finished 72-frame segment (12 s at 24 fps) into an INT8 ring of 72 frames
+        cache = nm.KVCache("int8", 16, 22, 40, 72, 72, device=dev)
+        k, v = (to_dev(x) for x in synth.history_kv(geo, 72, 5, 0))
+        byts = 72 * F * 16 * 2 * (HEAD_DIM * 2 + HEAD_DIM + 4)
+        for _ in range(W):
+            cache.commit(k, v, 72, stream=stream)
+        ts = []
+        for _ in range(K):
+            flush.zero_()
+            a, b = device_events(torch, 2)
+            a.record(stream)
+            cache.commit(k, v, 72, stream=stream)
+            b.record(stream)
+            b.synchronize()
+            ts.append(a.elapsed_time(b))
+        ms = statistics.mean(ts)
+        hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+        print(json.dumps({"metric": "kv_commit_gbs", "value": byts / (ms * 1e-3) / 1e9, "unit": "GB/s",
+                          "ms_per_commit": ms, "steps": K, "warmup": W, "higher_is_better": True,
+                          "config": {"workload": "commit_72f_int8", "frames": 72, "tokens": 72 * F, "heads": 16,
+                                     "algorithmic_bytes": byts, "l2": "flushed before each commit"},
+                          "roofline": {"bound": "hbm", "achieved": byts / (ms * 1e-3) / 1e9, "peak": hbm,
+                                       "unit": "GB/s", "frac": byts / (ms * 1e-3) / 1e9 / hbm,
+                                       "frac_of_nominal_8000": byts / (ms * 1e-3) / 1e9 / 8000.0,
+                                       "peak_kind": peak_src}}), flush=True)
+        return 0
+    if args.workload == "history_sweep":
+        out_rows = []
+        for hist in (1, 4, 9, 18, 36, 72):
+            w = synth.sweep_workload(hist)
+            cache = nm.KVCache("int8", 16, 22, 40, hist, hist, device=dev)
+            for s_, nf in enumerate(w["hist_commits"]):
+                k, v = synth.history_kv(geo, nf, w["seed"], s_)
+                cache.commit(to_dev(k), to_dev(v), nf, stream=stream)
+            q, k, v = (to_dev(x) for x in synth.segment_qkv(geo, 3, 256, w["seed"], segment=len(w["hist_commits"])))
+            out = torch.empty_like(q)
+            ws = cache.workspace(3, 256)
+            nq, nk = 3 * F + 256, hist * F + 3 * F + 256
+            flop = 4.0 * 16 * HEAD_DIM * nq * nk
+            for _ in range(W):
+                cache.seg_attn(q, k, v, 3, 256, out=out, workspace=ws, stream=stream)
+            ts = []
+            for _ in range(K):
+                flush.zero_()
+                a, b = device_events(torch, 2)
+                a.record(stream)
+                cache.seg_attn(q, k, v, 3, 256, out=out, workspace=ws, stream=stream)
+                b.record(stream)
+                b.synchronize()
+                ts.append(a.elapsed_time(b))
+            ms = statistics.mean(ts)
+            out_rows.append({"history_frames": hist, "nk": nk, "ms": ms, "tflops": flop / (ms * 1e-3) / 1e12})
+            del cache, q, k, v, out
+        print(json.dumps({"metric": "seg_attn_tflops_vs_history", "unit": "TFLOP/s", "steps": K, "warmup": W,
+                          "config": {"workload": "history_sweep", "cache": "int8", "nq": 3 * F + 256,
+                                     "l2": "flushed before each call"}, "rows": out_rows}), flush=True)
+        return 0
+    if args.workload == "layers54_turn":
+        # per layer: commit the finished 3-frame segment, then 8 denoising steps of segment attention
+        layers = 54
+        caches = []
+        kf, vf = (to_dev(x) for x in synth.history_kv(geo, 18, 4, 0))  # same history committed to every layer
+        for L in range(layers):
+            c = nm.KVCache("int8", 16, 22, 40, 18, 18, device=dev)
+            c.commit(kf, vf, 18, stream=stream)
+            caches.append(c)
+        kseg, vseg = (to_dev(x) for x in synth.history_kv(geo, 3, 4, 999))
+        q, k, v = (to_dev(x) for x in synth.segment_qkv(geo, 3, 256, 4, segment=1000))
+        out = torch.empty_like(q)
+        ws = caches[0].workspace(3, 256)
+        flop_attn = 4.0 * 16 * HEAD_DIM * (3 * F + 256) * (18 * F + 3 * F + 256)
+
+        def turn():
+            for c in caches:
+                c.commit(kseg, vseg, 3, stream=stream)
+                for _ in range(8):
+                    c.seg_attn(q, k, v, 3, 256, out=out, workspace=ws, stream=stream)
+
+        turn()
+        torch.cuda.synchronize(dev)
+        reps = max(1, K // 100)
+        a, b = device_events(torch, 2)
+        a.record(stream)
+        for _ in range(reps):
+            turn()
+        b.record(stream)
+        b.synchronize()
+        ms = a.elapsed_time(b) / reps
+        print(json.dumps({"metric": "turn_ms", "value": ms, "unit": "ms", "higher_is_better": False,
+                          "ms_per_layer_step": ms / (layers * 8), "turns": reps,
+                          "attn_tflops": layers * 8 * flop_attn / (ms * 1e-3) / 1e12,
+                          "config": {"workload": "layers54_turn", "layers": layers, "denoising_steps": 8,
+                                     "commit_frames": 3, "history_frames": 18, "cache": "int8",
+                                     "l2": "not flushed; 54 caches (3.6 GB) exceed L2"}}), flush=True)
+        return 0
+    raise SystemExit(f"unknown workload {args.workload}")
+
+
 def main():
     args = parse()
     rank = int(os.environ.get("RANK", "0"))
@@ -238,6 +367,13 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         return run_reference(args, rank, world)
+    if args.workload != WORKLOAD:
+        import torch
+        import segment_causal_kv_b200 as nm
+        torch.cuda.set_device(local)
+        if rank != 0:
+            return 0
+        return run_extra(args, torch, nm, torch.device("cuda", local))
 
     import torch
     import segment_causal_kv_b200 as nm
@@ -383,7 +519,8 @@ def main():
         "commit_ms": cm,
         "commit_gbs": commit_bytes(w) / (cm * 1e-3) / 1e9,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": None, "peak_kind": f"bf16 dense, sustained, {peak_src}",
+                     "frac": achieved / peak, "traffic": traffic_from_profile("attn_kernel<int8>"),
+                     "peak_kind": f"bf16 dense, sustained, {peak_src}",
                      "frac_of_burst": achieved / peak_burst, "frac_of_nominal_2250": achieved / 2250.0,
                      "kernel": "nomas_seg_attn call (prep + attn_kernel + combine), CUDA events"},
         "e2e": {"value": world * flop_step * Ke / (e2e_total * 1e-3) / 1e12, "unit": "TFLOP/s",
@@ -391,6 +528,7 @@ def main():
                 "ms_per_step": e2e_total / Ke},
         # per step: commit, RoPE prep, attention, and the split combine when used
         "gpu_launches": K * (3 + _combine_launches(cache)),
+        "commit_traffic_profile": traffic_from_profile("commit_kernel<int8>"),
         "clocks": clocks,
     }
     if world == 1 and not args.no_cpu_baseline:

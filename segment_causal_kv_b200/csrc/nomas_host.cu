@@ -221,6 +221,8 @@ int nomas_kv_commit(nomas_cache* c, const void* k, const void* v, int64_t token_
     if (!aligned(k, 16) || !aligned(v, 16)) return NOMAS_ERR_ALIGN;
     const int W = c->window_frames;
     if (W == 0 && c->frames_committed + n_frames > c->capacity_frames) return NOMAS_ERR_CAPACITY;
+    if (static_cast<int64_t>(kMaxFramesPerLaunch) * c->grid_h * c->grid_w * c->heads >= (int64_t(1) << 31))
+        return NOMAS_ERR_ARG; // one launch's (token, head) rows must fit 31 bits
     if ((rc = check_device()) != NOMAS_OK) return rc;
 
     const int tpf = c->grid_h * c->grid_w;
@@ -247,7 +249,11 @@ int nomas_kv_commit(nomas_cache* c, const void* k, const void* v, int64_t token_
         a.in_frame0 = f0;
         a.abs_frame0 = c->frames_committed + f0;
         a.window = W;
+        a.slot0 = W > 0 ? static_cast<int32_t>(a.abs_frame0 % W) : 0;
         a.int8_mode = c->mode == NOMAS_CACHE_INT8;
+        a.div_heads = make_fastdiv(static_cast<uint32_t>(c->heads));
+        a.div_tpf = make_fastdiv(static_cast<uint32_t>(tpf));
+        a.div_gw = make_fastdiv(static_cast<uint32_t>(c->grid_w));
         fill_t(tab, c->rope_theta, a.abs_frame0, nf);
         if (launch_commit(a, tab, s) != cudaSuccess) return NOMAS_ERR_CUDA;
     }
@@ -275,7 +281,7 @@ int nomas_seg_attn(const nomas_cache* c, const void* q, const void* k, const voi
     if (n_video_frames < 0 || n_text < 0) return NOMAS_ERR_ARG;
     const Plan p = make_plan(c, n_video_frames, n_text);
     if (p.nq == 0) return NOMAS_OK;
-    if (p.nq > (int64_t(1) << 30)) return NOMAS_ERR_ARG;
+    if (p.nq > (int64_t(1) << 30) || p.nq * c->heads >= (int64_t(1) << 31)) return NOMAS_ERR_ARG;
     if (!q || !k || !v || !out) return NOMAS_ERR_ARG;
     if (token_stride < static_cast<int64_t>(c->heads) * kD || token_stride % 8 != 0) return NOMAS_ERR_ARG;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16)) return NOMAS_ERR_ALIGN;
@@ -312,6 +318,9 @@ int nomas_seg_attn(const nomas_cache* c, const void* q, const void* k, const voi
             const bool last = f0 + nf >= n_video_frames;
             a.tok1 = last ? static_cast<int32_t>(p.nq) : static_cast<int32_t>((f0 + nf) * p.tpf);
             a.frame0 = f0;
+            a.div_heads = make_fastdiv(static_cast<uint32_t>(c->heads));
+            a.div_tpf = make_fastdiv(static_cast<uint32_t>(p.tpf));
+            a.div_gw = make_fastdiv(static_cast<uint32_t>(c->grid_w));
             if (nf > 0) fill_t(tab, c->rope_theta, c->frames_committed + f0, nf);
             if (a.tok1 > a.tok0 && launch_prep(a, tab, s) != cudaSuccess) return NOMAS_ERR_CUDA;
             f0 += nf;

@@ -6,7 +6,7 @@
 #include <cuda_runtime.h>
 #include <cstdint>
 
-#include "../../include/nomas.h"
+#include "nomas.h" // found through -I include
 
 namespace nomas {
 
@@ -25,6 +25,26 @@ struct RopeTab {
 };
 static_assert(sizeof(RopeTab) <= 30 * 1024, "RoPE table must fit the launch-argument limit");
 
+// Unsigned division by a runtime constant d for n < 2^31 (Granlund-Montgomery
+// round-up method): q = (umulhi(n, m) + n) >> s with s = ceil(log2 d) and
+// m = floor(2^32 (2^s - d) / d) + 1.
+struct FastDiv {
+    uint32_t d, m, s;
+};
+
+inline FastDiv make_fastdiv(uint32_t d) {
+    uint32_t s = 0;
+    while ((uint64_t(1) << s) < d) ++s;
+    const uint64_t m = ((uint64_t(1) << 32) * ((uint64_t(1) << s) - d)) / d + 1;
+    return FastDiv{d, static_cast<uint32_t>(m), s};
+}
+
+#ifdef __CUDACC__
+__device__ __forceinline__ uint32_t fast_div(uint32_t n, const FastDiv& f) {
+    return (__umulhi(n, f.m) + n) >> f.s;
+}
+#endif
+
 struct CommitArgs {
     const uint16_t* k;      // segment K, BF16 bits, token-major
     const uint16_t* v;      // segment V
@@ -39,7 +59,9 @@ struct CommitArgs {
     int32_t in_frame0;      // segment-local index of the first of them
     int64_t abs_frame0;     // absolute frame index of the first of them
     int32_t window;         // ring modulus (0: slot = absolute frame)
+    int32_t slot0;          // slot of the first frame of this launch
     int32_t int8_mode;
+    FastDiv div_heads, div_tpf, div_gw;
 };
 
 struct PrepArgs {
@@ -52,6 +74,7 @@ struct PrepArgs {
     int32_t nq, nv;         // tokens in the segment, video tokens
     int32_t tok0, tok1;     // token range handled by this launch
     int32_t frame0;         // segment-local frame of table row t[0]
+    FastDiv div_heads, div_tpf, div_gw;
 };
 
 struct AttnArgs {

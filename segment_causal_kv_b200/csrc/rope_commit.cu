@@ -83,6 +83,26 @@ __device__ __forceinline__ void unpack8(const uint4 x, float (&y)[8]) {
     }
 }
 
+// INT8 code of x for the row scale `scale` (inv = rn(1/scale)): the byte of
+// round-half-even(rn(x / scale)), the IEEE quotient's rounding.
+// x * inv lies within 2^-16 of the exact quotient (two roundings of at most
+// 2^-24 relative each, |x / scale| < 128), and so does the IEEE quotient; the
+// two can round to different integers only when a half-integer lies between
+// them. Away from half-integers (farther than 2^-14) the cheap product
+// decides; next to one, the exact division does. Rounding to an integer uses
+// the sum with 1.5 * 2^23: in [2^23, 2^24) the fp32 grid is the integers, so
+// the add rounds half to even, and the low byte of the sum's bit pattern is
+// the code in two's complement. |x / scale| <= 127 (1 + 3 * 2^-24) < 127.5, so
+// the code never needs clamping to [-127, 127].
+__device__ __forceinline__ uint32_t quant_word(float x, float scale, float inv) {
+    constexpr float kMagic = 12582912.0f; // 1.5 * 2^23
+    const float q = __fmul_rn(x, inv);
+    float t = __fadd_rn(q, kMagic);
+    const float f = __fsub_rn(q, __fsub_rn(t, kMagic)); // q - rint(q), exact
+    if (fabsf(f) > 0.5f - 6.103515625e-05f) t = __fadd_rn(__fdiv_rn(x, scale), kMagic);
+    return __float_as_uint(t);
+}
+
 // Half-warp INT8 quantisation of one row: returns 8 packed codes of this lane
 // and the row scale. Both half-warps of a warp must call it together.
 __device__ __forceinline__ uint2 quantize8(const float (&y)[8], float& scale_out) {
@@ -91,24 +111,20 @@ __device__ __forceinline__ uint2 quantize8(const float (&y)[8], float& scale_out
     for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(y[i]));
 #pragma unroll
     for (int off = 8; off >= 1; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off, 16));
-    uint32_t b[8];
     if (amax == 0.0f) {
         scale_out = 0.0f;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) b[i] = 0;
-    } else {
-        const float scale = __fdiv_rn(amax, 127.0f);
-        scale_out = scale;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            int q = __float2int_rn(__fdiv_rn(y[i], scale));
-            q = max(-127, min(127, q));
-            b[i] = static_cast<uint32_t>(q) & 0xFFu;
-        }
+        return make_uint2(0u, 0u);
     }
+    const float scale = __fdiv_rn(amax, 127.0f);
+    const float inv = __fdiv_rn(1.0f, scale);
+    scale_out = scale;
+    uint32_t w[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) w[i] = quant_word(y[i], scale, inv);
+    // low bytes of w[0..7], in order
     uint2 r;
-    r.x = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
-    r.y = b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24);
+    r.x = __byte_perm(__byte_perm(w[0], w[1], 0x0040u), __byte_perm(w[2], w[3], 0x0040u), 0x5410u);
+    r.y = __byte_perm(__byte_perm(w[4], w[5], 0x0040u), __byte_perm(w[6], w[7], 0x0040u), 0x5410u);
     return r;
 }
 
@@ -121,30 +137,55 @@ __global__ void __launch_bounds__(kThreads) commit_kernel(const __grid_constant_
     const int lane = threadIdx.x & 31;
     const int half = lane >> 4;
     const int l = lane & 15;
-    const int64_t rows = static_cast<int64_t>(a.n_frames) * a.tpf * a.heads;
-    const int64_t warps = static_cast<int64_t>(gridDim.x) * (kThreads / 32);
-    for (int64_t wp = static_cast<int64_t>(blockIdx.x) * (kThreads / 32) + (threadIdx.x >> 5); wp * 2 < rows;
-         wp += warps) {
-        const int64_t r = wp * 2 + half;
+    // row r of this launch: token r / heads (frame-major), head r % heads; all
+    // index math is 32-bit with constant-divisor division (rows < 2^31)
+    const uint32_t rows = static_cast<uint32_t>(a.n_frames) * a.tpf * a.heads;
+    const uint32_t warps = gridDim.x * (kThreads / 32);
+    auto in_offset = [&](uint32_t r) {
+        const uint32_t tok = fast_div(r, a.div_heads);
+        const uint32_t h = r - tok * a.heads;
+        const int64_t in_tok = static_cast<int64_t>(a.in_frame0) * a.tpf + tok;
+        return in_tok * a.token_stride + h * kD + l * 8;
+    };
+    // software pipeline: the next row pair's K and V are in flight while this one is processed
+    uint32_t wp = blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
+    uint4 kx = make_uint4(0, 0, 0, 0), vx = kx;
+    if (wp * 2 < rows) {
+        const uint32_t r0 = min(wp * 2 + half, rows - 1);
+        kx = __ldg(reinterpret_cast<const uint4*>(a.k + in_offset(r0)));
+        vx = __ldg(reinterpret_cast<const uint4*>(a.v + in_offset(r0)));
+    }
+    for (; wp * 2 < rows; wp += warps) {
+        const uint32_t r = wp * 2 + half;
         const bool valid = r < rows;
-        const int64_t rr = valid ? r : rows - 1;
-        const int64_t tok = rr / a.heads;
-        const int h = static_cast<int>(rr % a.heads);
-        const int fi = static_cast<int>(tok / a.tpf);
-        const int rif = static_cast<int>(tok % a.tpf);
-        const int64_t in_tok = static_cast<int64_t>(a.in_frame0 + fi) * a.tpf + rif;
-        const int64_t in_off = in_tok * a.token_stride + h * kD + l * 8;
-        const uint4 kx = __ldg(reinterpret_cast<const uint4*>(a.k + in_off));
-        const uint4 vx = __ldg(reinterpret_cast<const uint4*>(a.v + in_off));
+        const uint32_t rr = valid ? r : rows - 1;
+        uint4 kn = kx, vn = vx;
+        if ((wp + warps) * 2 < rows) {
+            const uint32_t rn = min((wp + warps) * 2 + half, rows - 1);
+            kn = __ldg(reinterpret_cast<const uint4*>(a.k + in_offset(rn)));
+            vn = __ldg(reinterpret_cast<const uint4*>(a.v + in_offset(rn)));
+        }
+        const uint32_t tok = fast_div(rr, a.div_heads);
+        const uint32_t h = rr - tok * a.heads;
+        const uint32_t fi = fast_div(tok, a.div_tpf);
+        const uint32_t rif = tok - fi * a.tpf;
+        const uint32_t hh = fast_div(rif, a.div_gw);
+        const uint32_t ww = rif - hh * a.grid_w;
 
         float2 cs[4];
-        lane_coeffs(l, fi, rif / a.grid_w, rif % a.grid_w, a.grid_h, s_t, s_hw, cs);
+        lane_coeffs(l, fi, hh, ww, a.grid_h, s_t, s_hw, cs);
         float ky[8], vy[8];
         rotate8(kx, cs, ky);
         unpack8(vx, vy);
 
-        const int64_t absf = a.abs_frame0 + fi;
-        const int64_t slot = a.window > 0 ? absf % a.window : absf;
+        // slot of frame fi: ring slots advance with the frame (fi < window within a launch)
+        int64_t slot;
+        if (a.window > 0) {
+            const int32_t s0 = a.slot0 + static_cast<int32_t>(fi);
+            slot = s0 >= a.window ? s0 - a.window : s0;
+        } else {
+            slot = a.abs_frame0 + fi;
+        }
         const int64_t row = static_cast<int64_t>(h) * a.cap_tok + slot * a.tpf + rif;
         if (a.int8_mode) {
             float ks, vs;
@@ -167,6 +208,8 @@ __global__ void __launch_bounds__(kThreads) commit_kernel(const __grid_constant_
             *reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.ck) + row * kD + l * 8) = ko;
             *reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.cv) + row * kD + l * 8) = vx;
         }
+        kx = kn;
+        vx = vn;
     }
 }
 
@@ -181,21 +224,23 @@ __global__ void __launch_bounds__(kThreads) prep_kernel(const __grid_constant__ 
 
     const int lane = threadIdx.x & 31;
     const int l = lane & 15;
-    const int64_t rows = static_cast<int64_t>(a.tok1 - a.tok0) * a.heads;
-    const int64_t halves = static_cast<int64_t>(gridDim.x) * (kThreads / 16);
-    for (int64_t r = static_cast<int64_t>(blockIdx.x) * (kThreads / 16) + (threadIdx.x >> 4); r < rows;
-         r += halves) {
-        const int tok = a.tok0 + static_cast<int>(r / a.heads);
-        const int h = static_cast<int>(r % a.heads);
+    const uint32_t rows = static_cast<uint32_t>(a.tok1 - a.tok0) * a.heads;
+    const uint32_t halves = gridDim.x * (kThreads / 16);
+    for (uint32_t r = blockIdx.x * (kThreads / 16) + (threadIdx.x >> 4); r < rows; r += halves) {
+        const uint32_t tq = fast_div(r, a.div_heads);
+        const int tok = a.tok0 + static_cast<int>(tq);
+        const int h = static_cast<int>(r - tq * a.heads);
         const int64_t in_off = static_cast<int64_t>(tok) * a.token_stride + h * kD + l * 8;
         const uint4 qx = __ldg(reinterpret_cast<const uint4*>(a.q + in_off));
         const uint4 kx = __ldg(reinterpret_cast<const uint4*>(a.k + in_off));
         uint4 qo = qx, ko = kx;
         if (tok < a.nv) {
-            const int fi = tok / a.tpf - a.frame0;
-            const int rif = tok % a.tpf;
+            const uint32_t fa = fast_div(static_cast<uint32_t>(tok), a.div_tpf);
+            const int fi = static_cast<int>(fa) - a.frame0;
+            const uint32_t rif = static_cast<uint32_t>(tok) - fa * a.tpf;
+            const uint32_t hh = fast_div(rif, a.div_gw);
             float2 cs[4];
-            lane_coeffs(l, fi, rif / a.grid_w, rif % a.grid_w, a.grid_h, s_t, s_hw, cs);
+            lane_coeffs(l, fi, hh, rif - hh * a.grid_w, a.grid_h, s_t, s_hw, cs);
             float qy[8], ky[8];
             rotate8(qx, cs, qy);
             rotate8(kx, cs, ky);
