@@ -26,7 +26,8 @@
 // probabilities P overwrite the first 64 columns of their S block and feed
 // the P.V product straight from TMEM (A operand in tensor memory).
 // MMA order per KV tile j: PV0(j-1) S0(j) | PV1(j-1) S1(j) -- while one
-// softmax warpgroup exponentiates, the tensor core works for the other.
+// softmax warpgroup exponentiates, the tensor core works for the other. The
+// issuer waits for V(j-1) before PV0(j-1) and for K(j) only before S0(j).
 // Online softmax in base 2 with lazy rescaling: the running reference max is
 // raised only when a tile's max exceeds it by more than 8 (so P <= 256), and
 // only then is O rescaled in TMEM.
@@ -151,18 +152,99 @@ __device__ __forceinline__ float row_max(uint32_t t_s, int vc) {
     return mx;
 }
 
-// P = 2^(s * scale_log2 - m) of one 128-key S row, written as packed BF16 pairs
-// over the first 64 columns of the row's S block (a 32-column chunk of S is in
-// registers before the 16 P columns over it are written). Returns the fp32
-// sum, accumulated in four independent packed pairs.
-template <bool kMask>
-__device__ __forceinline__ float row_exp_store(uint32_t t_s, float sl2, float m, int vc) {
+// 2^x of two values on the FMA pipe, so that part of a row's exponentials
+// leave the MUFU unit (which alone would take as long as the tensor core needs
+// for the row's two products). Range reduction x = n + f with n = rint(x)
+// (the 1.5 * 2^23 shift puts n in the low mantissa bits of t) and f in
+// [-1/2, 1/2]; 2^f by a cubic whose coefficients minimise the maximum relative
+// error on that interval (7.5e-5, well under the 2^-9 of the BF16 rounding of P
+// that follows; fitted by exp2_poly_fit.py beside this file); 2^n by adding n
+// to the exponent field (the shift by 23 keeps exactly the low 9 bits of t,
+// i.e. n modulo 2^9). x is clamped below at -125 so the result stays normal
+// (2^-125 in place of a smaller P, far under the BF16 resolution of the row).
+constexpr float kExp2C0 = 0.9999280571937561f;
+constexpr float kExp2C1 = 0.6932608485221863f;
+constexpr float kExp2C2 = 0.24261115491390228f;
+constexpr float kExp2C3 = 0.05517221987247467f;
+__device__ __forceinline__ float2 exp2_fma2(float2 x) {
+    x.x = fmaxf(x.x, -125.0f);
+    x.y = fmaxf(x.y, -125.0f);
+    const float2 t = __fadd2_rn(x, make_float2(12582912.0f, 12582912.0f));
+    const float2 nf = __fadd2_rn(t, make_float2(-12582912.0f, -12582912.0f));
+    const float2 f = __ffma2_rn(nf, make_float2(-1.0f, -1.0f), x);
+    float2 q = __ffma2_rn(f, make_float2(kExp2C3, kExp2C3), make_float2(kExp2C2, kExp2C2));
+    q = __ffma2_rn(q, f, make_float2(kExp2C1, kExp2C1));
+    q = __ffma2_rn(q, f, make_float2(kExp2C0, kExp2C0));
+    return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
+                       __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
+}
+
+// Of every 8 column pairs of a full tile, kPoly take exp2_fma2 and the rest
+// the MUFU ex2. With an INT8 cache the dequantising warps share the FMA pipe
+// and issue slots of every SM sub-partition, so that kernel keeps all of them
+// on the MUFU.
+constexpr int kExp2PolyPairsBf16 = 3;
+constexpr int kExp2PolyPairsInt8 = 0;
+
+// One 32-column chunk of an unmasked S row -> 16 packed BF16 P columns.
+template <int kPoly>
+__device__ __forceinline__ void exp_chunk(const uint32_t (&s)[32], float2 sl2x2, float2 negm, float2 (&acc)[4],
+                                          uint32_t (&p)[16]) {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+        const float2 x = __ffma2_rn(make_float2(__uint_as_float(s[2 * e]), __uint_as_float(s[2 * e + 1])), sl2x2, negm);
+        float2 y;
+        if ((e & 7) < kPoly)
+            y = exp2_fma2(x);
+        else
+            y = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+        acc[e & 3] = __fadd2_rn(acc[e & 3], y);
+        p[e] = pack_bf16x2(y.x, y.y);
+    }
+}
+
+// P = 2^(s * scale_log2 - m) of one full 128-key S row, written as packed BF16
+// pairs over the first 64 columns of the row's S block; returns the fp32 row
+// sum (four independent packed accumulators). The TMEM loads are software
+// pipelined: chunk c + 1 is in flight while chunk c is exponentiated. P chunk c
+// lands on columns [16c, 16c + 16), all of which were read with chunks <= c.
+template <int kPoly>
+__device__ __forceinline__ float row_exp_store_full(uint32_t t_s, float sl2, float m) {
     const float2 sl2x2 = make_float2(sl2, sl2);
     const float2 negm = make_float2(-m, -m);
     float2 acc[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) acc[k] = make_float2(0.0f, 0.0f);
+    uint32_t sa[32], sb[32], p[16];
+    tmem_ld32_issue(t_s, sa);
+    tmem_ld32_wait(sa);
+    tmem_ld32_issue(t_s + 32, sb);
+    exp_chunk<kPoly>(sa, sl2x2, negm, acc, p);
+    tmem_st16(t_s, p);
+    tmem_ld32_wait(sb);
+    tmem_ld32_issue(t_s + 64, sa);
+    exp_chunk<kPoly>(sb, sl2x2, negm, acc, p);
+    tmem_st16(t_s + 16, p);
+    tmem_ld32_wait(sa);
+    tmem_ld32_issue(t_s + 96, sb);
+    exp_chunk<kPoly>(sa, sl2x2, negm, acc, p);
+    tmem_st16(t_s + 32, p);
+    tmem_ld32_wait(sb);
+    exp_chunk<kPoly>(sb, sl2x2, negm, acc, p);
+    tmem_st16(t_s + 48, p);
+    const float2 t = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+    return t.x + t.y;
+}
+
+// Masked form for a ragged last tile (columns >= vc get P = 0): MUFU only,
+// one 32-column chunk at a time.
+__device__ __forceinline__ float row_exp_store_masked_impl(uint32_t t_s, float sl2, float m, int vc) {
+    const float2 sl2x2 = make_float2(sl2, sl2);
+    const float2 negm = make_float2(-m, -m);
+    float2 acc[4];
 #pragma unroll
+    for (int k = 0; k < 4; ++k) acc[k] = make_float2(0.0f, 0.0f);
+#pragma unroll 1
     for (int c = 0; c < 4; ++c) {
         uint32_t s[32];
         tmem_ld32(t_s + c * 32, s);
@@ -170,11 +252,9 @@ __device__ __forceinline__ float row_exp_store(uint32_t t_s, float sl2, float m,
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
             float2 x = __ffma2_rn(make_float2(__uint_as_float(s[2 * e]), __uint_as_float(s[2 * e + 1])), sl2x2, negm);
-            if (kMask) {
-                const int col = c * 32 + 2 * e;
-                x.x = col < vc ? x.x : -INFINITY;
-                x.y = col + 1 < vc ? x.y : -INFINITY;
-            }
+            const int col = c * 32 + 2 * e;
+            x.x = col < vc ? x.x : -INFINITY;
+            x.y = col + 1 < vc ? x.y : -INFINITY;
             const float p0 = ex2_approx(x.x), p1 = ex2_approx(x.y);
             acc[e & 3] = __fadd2_rn(acc[e & 3], make_float2(p0, p1));
             p[e] = pack_bf16x2(p0, p1);
@@ -189,7 +269,7 @@ __device__ __forceinline__ float row_exp_store(uint32_t t_s, float sl2, float m,
 // the per-tile loop: tail tiles (masked), O rescaling, the epilogues.
 __device__ __noinline__ float row_max_masked(uint32_t t_s, int vc) { return row_max<true>(t_s, vc); }
 __device__ __noinline__ float row_exp_store_masked(uint32_t t_s, float sl2, float m, int vc) {
-    return row_exp_store<true>(t_s, sl2, m, vc);
+    return row_exp_store_masked_impl(t_s, sl2, m, vc);
 }
 
 // O *= alpha for one row (one thread), in TMEM.
@@ -415,7 +495,6 @@ __global__ void __launch_bounds__(kInt8 ? 512 : 384, 1)
                 const uint32_t ph1 = ((i + 1) / kStages) & 1;
                 const bool last = (i + 1 == n);
                 if (!(ok = mbar_wait(bar(B_VFULL + st), ph, ctl))) break;
-                if (!last && !(ok = mbar_wait(bar(B_KFULL + st1), ph1, ctl))) break;
                 for (int w = 0; w < nq_tiles; ++w) {
                     if (!(ok = mbar_wait(bar(B_PFULL + w), i & 1, ctl))) break;
                     tc_fence_after();
@@ -424,6 +503,12 @@ __global__ void __launch_bounds__(kInt8 ? 512 : 384, 1)
                     // so no arrival is left pending at exit
                     if (w == nq_tiles - 1 && i + kStages < n) mma_commit(bar(B_VEMPTY + st));
                     if (!last) {
+                        // K of tile i + 1 is needed from here on only: P.V of Q tile 0
+                        // never waits for it
+                        if (w == 0) {
+                            if (!(ok = mbar_wait(bar(B_KFULL + st1), ph1, ctl))) break;
+                            tc_fence_after();
+                        }
                         issue_s(w, st1);
                         mma_commit(bar(B_SFULL + w));
                         if (w == nq_tiles - 1 && i + 1 + kStages < n) mma_commit(bar(B_KEMPTY + st1));
@@ -467,7 +552,8 @@ __global__ void __launch_bounds__(kInt8 ? 512 : 384, 1)
                 l *= alpha;
                 m_ref = m_new;
                 // pass 2: P into TMEM, row sum in fp32
-                l += full ? row_exp_store<false>(t_s, sl2, m_ref, vc) : row_exp_store_masked(t_s, sl2, m_ref, vc);
+                l += full ? row_exp_store_full<kInt8 ? kExp2PolyPairsInt8 : kExp2PolyPairsBf16>(t_s, sl2, m_ref)
+                          : row_exp_store_masked(t_s, sl2, m_ref, vc);
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
