@@ -144,12 +144,21 @@ int nomas_kv_commit(nomas_cache *c, const void *k, const void *v, int64_t token_
                     void *stream);
 
 /*
- * nomas_seg_attn_workspace_bytes -- device workspace nomas_seg_attn needs
- * for this cache state and segment shape (0 on invalid arguments). The
- * first 256 bytes of a workspace are a status header: zero them once
- * before first use; the library only sets error bits in it.
+ * nomas_seg_attn_workspace_bytes -- device workspace for the fastest form of
+ * nomas_seg_attn for this cache state and segment shape (0 on invalid
+ * arguments). For an INT8 cache it includes a BF16 copy of the visible window
+ * (2 * heads * visible_tokens * 256 bytes): the window is then dequantised
+ * once per call and read by the BF16 attention kernel, instead of being
+ * converted in shared memory by every CTA that reads a tile.
+ * nomas_seg_attn_workspace_min_bytes -- the smallest workspace nomas_seg_attn
+ * accepts: without the copy, so an INT8 window is converted tile by tile
+ * inside the attention kernel (same results up to rounding order, slower).
+ * Both are equal for a BF16 cache. The first 256 bytes of a workspace are a
+ * status header: zero them once before first use; the library only sets
+ * error bits in it.
  */
 size_t nomas_seg_attn_workspace_bytes(const nomas_cache *c, int32_t n_video_frames, int32_t n_text);
+size_t nomas_seg_attn_workspace_min_bytes(const nomas_cache *c, int32_t n_video_frames, int32_t n_text);
 
 /*
  * nomas_seg_attn -- segment-causal joint attention of the current segment
@@ -170,8 +179,10 @@ size_t nomas_seg_attn_workspace_bytes(const nomas_cache *c, int32_t n_video_fram
  * tokens of the current segment (keys rotated with their own positions).
  * The cache is read only. Q and current K are rounded to BF16 after RoPE,
  * probabilities are BF16 for the P.V product, accumulation is fp32.
- * workspace : device, >= nomas_seg_attn_workspace_bytes(...) bytes,
- *             256-byte aligned, not shared with a call running concurrently.
+ * workspace : device, >= nomas_seg_attn_workspace_min_bytes(...) bytes
+ *             (>= nomas_seg_attn_workspace_bytes(...) selects the
+ *             dequantise-once form for an INT8 cache), 256-byte aligned, not
+ *             shared with a call running concurrently.
  * Errors: NOMAS_ERR_ARG, NOMAS_ERR_ALIGN, NOMAS_ERR_STATE,
  * NOMAS_ERR_WORKSPACE, NOMAS_ERR_DEVICE, NOMAS_ERR_CUDA.
  */
@@ -199,9 +210,12 @@ int nomas_device_status(void *workspace, void *stream);
  * that loads the library until the process exits.
  *
  * Arguments, layouts, results and errors are those of nomas_seg_attn, minus
- * the workspace. A shape whose workspace (nomas_seg_attn_workspace_bytes)
- * exceeds NOMAS_STATIC_SCRATCH_BYTES is rejected with NOMAS_ERR_WORKSPACE
- * before anything is enqueued. The call allocates and frees nothing.
+ * the workspace. The fixed array serves as a workspace of
+ * NOMAS_STATIC_SCRATCH_BYTES: the dequantise-once form runs when
+ * nomas_seg_attn_workspace_bytes fits in it, the fused form when only
+ * nomas_seg_attn_workspace_min_bytes does, and a shape whose minimum exceeds
+ * it is rejected with NOMAS_ERR_WORKSPACE before anything is enqueued. The
+ * call allocates and frees nothing.
  * The first call on a device (with that device current) sets the array up:
  * it looks up its device address and clears its status header, a blocking
  * step; make that first call before any stream capture. All calls share the
@@ -212,6 +226,26 @@ int nomas_device_status(void *workspace, void *stream);
 #define NOMAS_STATIC_SCRATCH_BYTES (64u << 20)
 int nomas_seg_attn_static(const nomas_cache *c, const void *q, const void *k, const void *v, int64_t token_stride,
                           int32_t n_video_frames, int32_t n_text, void *out, float *lse, void *stream);
+
+/*
+ * nomas_selftest_bounded_wait -- run the bounded-wait failure path of the
+ * kernels on the device, without any fault. The pages have no counterpart:
+ * this is a diagnostic of the library's failure detection. It enqueues one
+ * tiny kernel on `stream` whose first role waits on an mbarrier that nothing
+ * arrives on; after NOMAS_WAIT_NS (2 s) of device time the wait gives up,
+ * sets the status bit in word 0 of `workspace` and raises the CTA's abort
+ * flag, and the second role, waiting on another such barrier, returns on
+ * seeing that flag.
+ *   workspace  device pointer, 16-byte aligned, at least 16 bytes: word 0 is
+ *              the status word read by nomas_device_status; the call clears
+ *              words 1 and 2 and the kernel sets word 1 when the first role
+ *              gave up and word 2 when the second role returned on the abort
+ *              flag. Word 0 is not cleared first (status bits accumulate).
+ * Returns NOMAS_OK once enqueued (then nomas_device_status on the same
+ * workspace and stream returns NOMAS_ERR_DEVICE_TIMEOUT), NOMAS_ERR_ARG for a
+ * null or unaligned workspace, NOMAS_ERR_CUDA if the launch fails.
+ */
+int nomas_selftest_bounded_wait(void *workspace, void *stream);
 
 /* Human-readable name of a status code (static storage). */
 const char *nomas_status_string(int status);

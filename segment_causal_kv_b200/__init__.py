@@ -34,8 +34,9 @@ NOMAS_CACHE_INT8 = 1
 HEAD_DIM = 128
 
 # exported symbols (checked against include/nomas.h by the tests)
-EXPORTS = ("nomas_cache_reset", "nomas_kv_commit", "nomas_seg_attn_workspace_bytes", "nomas_seg_attn",
-           "nomas_device_status", "nomas_status_string", "nomas_seg_attn_static")
+EXPORTS = ("nomas_cache_reset", "nomas_kv_commit", "nomas_seg_attn_workspace_bytes",
+           "nomas_seg_attn_workspace_min_bytes", "nomas_seg_attn",
+           "nomas_device_status", "nomas_status_string", "nomas_seg_attn_static", "nomas_selftest_bounded_wait")
 NOMAS_STATIC_SCRATCH_BYTES = 64 << 20
 
 
@@ -86,12 +87,16 @@ def lib():
         L.nomas_kv_commit.restype = ctypes.c_int
         L.nomas_seg_attn_workspace_bytes.argtypes = [D, I32, I32]
         L.nomas_seg_attn_workspace_bytes.restype = ctypes.c_size_t
+        L.nomas_seg_attn_workspace_min_bytes.argtypes = [D, I32, I32]
+        L.nomas_seg_attn_workspace_min_bytes.restype = ctypes.c_size_t
         L.nomas_seg_attn.argtypes = [D, P, P, P, I64, I32, I32, P, P, P, ctypes.c_size_t, P]
         L.nomas_seg_attn.restype = ctypes.c_int
         L.nomas_device_status.argtypes = [P, P]
         L.nomas_device_status.restype = ctypes.c_int
         L.nomas_seg_attn_static.argtypes = [D, P, P, P, I64, I32, I32, P, P, P]
         L.nomas_seg_attn_static.restype = ctypes.c_int
+        L.nomas_selftest_bounded_wait.argtypes = [P, P]
+        L.nomas_selftest_bounded_wait.restype = ctypes.c_int
         L.nomas_status_string.argtypes = [ctypes.c_int]
         L.nomas_status_string.restype = ctypes.c_char_p
         _lib = L
@@ -117,6 +122,10 @@ def nomas_seg_attn_workspace_bytes(desc: NomasCacheDesc, n_video_frames: int, n_
     return int(lib().nomas_seg_attn_workspace_bytes(ctypes.byref(desc), n_video_frames, n_text))
 
 
+def nomas_seg_attn_workspace_min_bytes(desc: NomasCacheDesc, n_video_frames: int, n_text: int) -> int:
+    return int(lib().nomas_seg_attn_workspace_min_bytes(ctypes.byref(desc), n_video_frames, n_text))
+
+
 def nomas_seg_attn(desc: NomasCacheDesc, q_ptr: int, k_ptr: int, v_ptr: int, token_stride: int,
                    n_video_frames: int, n_text: int, out_ptr: int, lse_ptr: int | None, ws_ptr: int | None,
                    ws_bytes: int, stream: int | None) -> int:
@@ -130,6 +139,11 @@ def nomas_seg_attn_static(desc: NomasCacheDesc, q_ptr: int, k_ptr: int, v_ptr: i
     """nomas_seg_attn with the library's static scratch, for callers that cannot allocate a workspace."""
     return lib().nomas_seg_attn_static(ctypes.byref(desc), q_ptr, k_ptr, v_ptr, token_stride, n_video_frames,
                                        n_text, out_ptr, lse_ptr, stream)
+
+
+def nomas_selftest_bounded_wait(ws_ptr: int, stream: int | None) -> int:
+    """Enqueue the bounded-wait self-test (a wait on a barrier nothing arrives on gives up after 2 s)."""
+    return lib().nomas_selftest_bounded_wait(ws_ptr, stream)
 
 
 def nomas_device_status(ws_ptr: int, stream: int | None) -> int:
@@ -219,8 +233,11 @@ class KVCache:
     def workspace_bytes(self, n_video_frames: int, n_text: int) -> int:
         return nomas_seg_attn_workspace_bytes(self.desc, n_video_frames, n_text)
 
+    def workspace_min_bytes(self, n_video_frames: int, n_text: int) -> int:
+        return nomas_seg_attn_workspace_min_bytes(self.desc, n_video_frames, n_text)
+
     def workspace(self, n_video_frames: int, n_text: int):
-        """A cached device workspace large enough for this call (status header zeroed)."""
+        """A cached device workspace for the fastest form of this call (status header zeroed)."""
         torch = _torch()
         need = self.workspace_bytes(n_video_frames, n_text)
         if self._ws is None or self._ws.numel() < need:

@@ -149,7 +149,10 @@ bool make_tmap(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint6
 struct Plan {
     int64_t tpf, nv, nq, nc;
     int tiles_c, tiles_q, pairs, splits, tiles_per_split;
-    size_t off_qt, off_kt, off_po, off_pml, total;
+    size_t off_qt, off_kt, off_po, off_pml;
+    size_t total_min; // the fused kernel's workspace (the smallest accepted)
+    size_t off_kd, off_vd;
+    size_t total;     // with the BF16 copy of an INT8 window (dequantise once)
 };
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -176,6 +179,9 @@ void choose_splits(int units, int tiles, int& splits, int& tps) {
     }
 }
 
+// The dequantise-once kernel indexes (tensor, row, 16-code part) in 32 bits.
+bool dequant_once_fits(int heads, int64_t nc) { return static_cast<int64_t>(heads) * nc < (int64_t(1) << 28); }
+
 Plan make_plan(const nomas_cache* c, int32_t n_video_frames, int32_t n_text) {
     Plan p{};
     p.tpf = static_cast<int64_t>(c->grid_h) * c->grid_w;
@@ -192,7 +198,14 @@ Plan make_plan(const nomas_cache* c, int32_t n_video_frames, int32_t n_text) {
     p.off_kt = round_up(p.off_qt + qk_bytes, 256);
     p.off_po = round_up(p.off_kt + qk_bytes, 256);
     p.off_pml = p.off_po + (p.splits > 1 ? prow * kD * sizeof(float) : 0);
-    p.total = round_up(p.off_pml + (p.splits > 1 ? prow * sizeof(float2) : 0), 256);
+    p.total_min = round_up(p.off_pml + (p.splits > 1 ? prow * sizeof(float2) : 0), 256);
+    p.off_kd = p.off_vd = p.total = p.total_min;
+    if (c->mode == NOMAS_CACHE_INT8 && p.nc > 0 && dequant_once_fits(c->heads, p.nc)) {
+        const size_t copy = round_up(static_cast<size_t>(c->heads) * p.nc * kD * 2, 256);
+        p.off_kd = p.total_min;
+        p.off_vd = p.off_kd + copy;
+        p.total = p.off_vd + copy;
+    }
     return p;
 }
 
@@ -273,6 +286,11 @@ size_t nomas_seg_attn_workspace_bytes(const nomas_cache* c, int32_t n_video_fram
     return make_plan(c, n_video_frames, n_text).total;
 }
 
+size_t nomas_seg_attn_workspace_min_bytes(const nomas_cache* c, int32_t n_video_frames, int32_t n_text) {
+    if (validate_state(c) != NOMAS_OK || n_video_frames < 0 || n_text < 0) return 0;
+    return make_plan(c, n_video_frames, n_text).total_min;
+}
+
 int nomas_seg_attn(const nomas_cache* c, const void* q, const void* k, const void* v, int64_t token_stride,
                    int32_t n_video_frames, int32_t n_text, void* out, float* lse, void* workspace,
                    size_t workspace_bytes, void* stream) {
@@ -286,7 +304,7 @@ int nomas_seg_attn(const nomas_cache* c, const void* q, const void* k, const voi
     if (token_stride < static_cast<int64_t>(c->heads) * kD || token_stride % 8 != 0) return NOMAS_ERR_ARG;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16)) return NOMAS_ERR_ALIGN;
     if (lse && !aligned(lse, 4)) return NOMAS_ERR_ALIGN;
-    if (!workspace || workspace_bytes < p.total) return NOMAS_ERR_WORKSPACE;
+    if (!workspace || workspace_bytes < p.total_min) return NOMAS_ERR_WORKSPACE;
     if (!aligned(workspace, 256)) return NOMAS_ERR_ALIGN;
     if ((rc = check_device()) != NOMAS_OK) return rc;
 
@@ -328,7 +346,29 @@ int nomas_seg_attn(const nomas_cache* c, const void* q, const void* k, const voi
         } while (true);
     }
 
-    // 2) tensor maps
+    // 2) an INT8 window with room for its BF16 copy is dequantised once here and
+    //    read by the BF16-cache kernel; otherwise the fused kernel converts it
+    //    tile by tile in shared memory (once per CTA that reads the tile)
+    const bool int8 = c->mode == NOMAS_CACHE_INT8;
+    const bool dequant_once = int8 && p.total > p.total_min && workspace_bytes >= p.total;
+    uint16_t* kd = reinterpret_cast<uint16_t*>(ws + p.off_kd);
+    uint16_t* vd = reinterpret_cast<uint16_t*>(ws + p.off_vd);
+    if (dequant_once) {
+        DequantArgs d{};
+        d.kc = static_cast<const int8_t*>(c->k);
+        d.vc = static_cast<const int8_t*>(c->v);
+        d.ks = c->k_scale;
+        d.vs = c->v_scale;
+        d.kd = kd;
+        d.vd = vd;
+        d.cap_tok = static_cast<int64_t>(c->capacity_frames) * p.tpf;
+        d.nc = static_cast<int32_t>(p.nc);
+        d.heads = c->heads;
+        d.div_nc = make_fastdiv(static_cast<uint32_t>(p.nc));
+        if (launch_dequant_window(d, s) != cudaSuccess) return NOMAS_ERR_CUDA;
+    }
+
+    // 3) tensor maps
     CUtensorMap tm_q, tm_kcur, tm_vcur, tm_kc, tm_vc;
     const uint64_t row_bytes = kD * 2;
     bool ok = make_tmap(&tm_q, qt, kD, p.nq, c->heads, row_bytes, p.nq * row_bytes, kBM, 1) &&
@@ -339,13 +379,16 @@ int nomas_seg_attn(const nomas_cache* c, const void* q, const void* k, const voi
         const uint64_t nc_ext = p.nc > 0 ? p.nc : 1;
         ok = ok && make_tmap(&tm_kc, c->k, kD, nc_ext, c->heads, row_bytes, cap_tok * row_bytes, kBM, 1) &&
              make_tmap(&tm_vc, c->v, kD, nc_ext, c->heads, row_bytes, cap_tok * row_bytes, kBM, 1);
+    } else if (dequant_once) {
+        ok = ok && make_tmap(&tm_kc, kd, kD, p.nc, c->heads, row_bytes, p.nc * row_bytes, kBM, 1) &&
+             make_tmap(&tm_vc, vd, kD, p.nc, c->heads, row_bytes, p.nc * row_bytes, kBM, 1);
     } else {
         tm_kc = tm_q;
         tm_vc = tm_q;
     }
     if (!ok) return NOMAS_ERR_CUDA;
 
-    // 3) attention (+ combine of KV splits)
+    // 4) attention (+ combine of KV splits)
     AttnArgs a{};
     a.heads = c->heads;
     a.nq = static_cast<int32_t>(p.nq);
@@ -366,7 +409,7 @@ int nomas_seg_attn(const nomas_cache* c, const void* q, const void* k, const voi
     a.part_ml = reinterpret_cast<float2*>(ws + p.off_pml);
     a.err = reinterpret_cast<unsigned*>(ws);
     a.scale_log2 = static_cast<float>(1.4426950408889634 / sqrt(static_cast<double>(kD)));
-    if (launch_attn(a, c->mode == NOMAS_CACHE_INT8, tm_q, tm_kcur, tm_vcur, tm_kc, tm_vc, s) != cudaSuccess)
+    if (launch_attn(a, int8 && !dequant_once, tm_q, tm_kcur, tm_vcur, tm_kc, tm_vc, s) != cudaSuccess)
         return NOMAS_ERR_CUDA;
     if (p.splits > 1) {
         CombineArgs cb{};

@@ -107,6 +107,23 @@ struct CombineArgs {
     float* lse;
 };
 
+// Dequantisation of an INT8 cache's visible window into a BF16 copy, once per
+// attention call: rows [0, nc) of every head of K and V, codes * scale rounded
+// to BF16 (the same values the fused kernel converts in shared memory), written
+// head-major [heads][nc][128].
+struct DequantArgs {
+    const int8_t* kc;
+    const int8_t* vc;
+    const float* ks;
+    const float* vs;
+    uint16_t* kd;
+    uint16_t* vd;
+    int64_t cap_tok; // token capacity of one head's slab in the cache
+    int32_t nc;      // visible tokens per head
+    int32_t heads;
+    FastDiv div_nc;
+};
+
 // Kernel launchers (return cudaError_t of the launch).
 cudaError_t launch_commit(const CommitArgs& a, const RopeTab& tab, cudaStream_t s);
 cudaError_t launch_prep(const PrepArgs& a, const RopeTab& tab, cudaStream_t s);
@@ -114,5 +131,6 @@ cudaError_t launch_attn(const AttnArgs& a, bool int8_cache, const CUtensorMap& t
                         const CUtensorMap& tm_vcur, const CUtensorMap& tm_kc, const CUtensorMap& tm_vc,
                         cudaStream_t s);
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s);
+cudaError_t launch_dequant_window(const DequantArgs& a, cudaStream_t s);
 
 } // namespace nomas

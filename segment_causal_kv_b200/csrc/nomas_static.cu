@@ -61,7 +61,7 @@ int static_scratch(void** out) {
 extern "C" int nomas_seg_attn_static(const nomas_cache* c, const void* q, const void* k, const void* v,
                                      int64_t token_stride, int32_t n_video_frames, int32_t n_text, void* out,
                                      float* lse, void* stream) {
-    const size_t need = nomas_seg_attn_workspace_bytes(c, n_video_frames, n_text);
+    const size_t need = nomas_seg_attn_workspace_min_bytes(c, n_video_frames, n_text);
     if (need == 0) // invalid descriptor or sizes: report the exact reason without touching memory
         return nomas_seg_attn(c, q, k, v, token_stride, n_video_frames, n_text, out, lse, nullptr, 0, stream);
     if (need > static_cast<size_t>(NOMAS_STATIC_SCRATCH_BYTES)) return NOMAS_ERR_WORKSPACE;

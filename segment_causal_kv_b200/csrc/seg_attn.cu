@@ -14,7 +14,7 @@
 // segment's tiles):
 //   warp 0      TMA producer: Q tiles once, then (BF16 caches) every K/V tile
 //               into a 2-stage ring
-//   warp 1      TMEM allocator + single-thread tcgen05.mma issuer
+//   warp 1      TMEM allocator + tcgen05.mma issuer
 //   warps 4-7   softmax warpgroup for Q tile 0 (one thread per query row)
 //   warps 8-11  softmax warpgroup for Q tile 1
 //   warps 12-15 INT8 caches only: the one filler of the K/V ring -- cache
@@ -71,6 +71,13 @@ constexpr uint32_t kOffTmemSlot = B_COUNT * 8;
 constexpr uint32_t kOffAbort = kOffTmemSlot + 8;
 constexpr uint32_t kOffDqGo = kOffAbort + 4;
 static_assert(kOffDqGo + 4 <= 256, "barrier area overflow");
+
+// mbar_wait run by every lane of a converged warp; lane 0's outcome is
+// broadcast so the warp leaves the wait converged.
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, const WaitCtl& ctl) {
+    const bool ok = mbar_wait(bar, parity, ctl);
+    return __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
+}
 
 __device__ __forceinline__ int tile_valid(const AttnArgs& a, int t) {
     const int rem = (t < a.tiles_c) ? a.nc - t * BN : a.nq - (t - a.tiles_c) * BN;
@@ -456,37 +463,48 @@ __global__ void __launch_bounds__(kInt8 ? 512 : 384, 1)
         }
     } else if (warp == 1) {
         // ================================================================ MMA issuer
-        if (lane == 0) {
+        // BF16 caches: the whole warp runs the loop (warp-uniform waits and
+        // conditions) and one elected lane issues each MMA and commit; MMAs issued
+        // by a single lane in a divergent branch run at little more than half the
+        // tensor-core rate whenever a branch separates two groups of them. With
+        // an INT8 cache the filler warps are the bottleneck and the warp-wide
+        // polling only takes issue slots from them, so lane 0 issues alone.
+        constexpr bool kWarpIssue = !kInt8;
+        if (kWarpIssue || lane == 0) {
+#define MMA_SS(...) (kWarpIssue ? mma_ss_warp(__VA_ARGS__) : mma_ss(__VA_ARGS__))
+#define MMA_TS(...) (kWarpIssue ? mma_ts_warp(__VA_ARGS__) : mma_ts(__VA_ARGS__))
+#define MMA_COMMIT(b) (kWarpIssue ? mma_commit_warp(b) : mma_commit(b))
+#define MBAR_WAIT(b, p, c) (kWarpIssue ? mbar_wait_warp(b, p, c) : mbar_wait(b, p, c))
             constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, BN, false, false);
             constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, kD, false, true);
             const uint32_t q_tile[2] = {sbase + kOffQ, sbase + kOffQ + kTileBytes};
             const uint32_t tm_s[2] = {tmem, tmem + 128};
             const uint32_t tm_o[2] = {tmem + 256, tmem + 384};
             const int nq_tiles = has_q1 ? 2 : 1;
-            bool ok = mbar_wait(bar(B_QFULL), 0, ctl);
+            bool ok = MBAR_WAIT(bar(B_QFULL), 0, ctl);
             tc_fence_after();
             auto issue_s = [&](int w, int st) {
                 const uint32_t ktile = sbase + kOffK + st * kTileBytes;
 #pragma unroll
                 for (int kk = 0; kk < kD / 16; ++kk)
-                    mma_ss(tm_s[w], desc_kmajor(q_tile[w], kk), desc_kmajor(ktile, kk), idesc_qk, kk > 0 ? 1u : 0u);
+                    MMA_SS(tm_s[w], desc_kmajor(q_tile[w], kk), desc_kmajor(ktile, kk), idesc_qk, kk > 0 ? 1u : 0u);
             };
             auto issue_pv = [&](int w, int st, bool first_tile) {
                 const uint32_t vtile = sbase + kOffV + st * kTileBytes;
 #pragma unroll
                 for (int kk = 0; kk < BN / 16; ++kk)
-                    mma_ts(tm_o[w], tm_s[w] + kk * 8, desc_mnmajor(vtile, kk), idesc_pv,
+                    MMA_TS(tm_o[w], tm_s[w] + kk * 8, desc_mnmajor(vtile, kk), idesc_pv,
                            (first_tile && kk == 0) ? 0u : 1u);
             };
-            if (ok) ok = mbar_wait(bar(B_KFULL + 0), 0, ctl);
+            if (ok) ok = MBAR_WAIT(bar(B_KFULL + 0), 0, ctl);
             if (ok) {
                 tc_fence_after();
                 for (int w = 0; w < nq_tiles; ++w) {
                     issue_s(w, 0);
-                    mma_commit(bar(B_SFULL + w));
+                    MMA_COMMIT(bar(B_SFULL + w));
                 }
                 // K of tile 0 is free once these S MMAs finish (a fill of tile 2 waits for it)
-                if (kStages < n) mma_commit(bar(B_KEMPTY + 0));
+                if (kStages < n) MMA_COMMIT(bar(B_KEMPTY + 0));
             }
             for (int i = 0; ok && i < n; ++i) {
                 const int st = i % kStages;
@@ -494,35 +512,39 @@ __global__ void __launch_bounds__(kInt8 ? 512 : 384, 1)
                 const int st1 = (i + 1) % kStages;
                 const uint32_t ph1 = ((i + 1) / kStages) & 1;
                 const bool last = (i + 1 == n);
-                if (!(ok = mbar_wait(bar(B_VFULL + st), ph, ctl))) break;
+                if (!(ok = MBAR_WAIT(bar(B_VFULL + st), ph, ctl))) break;
                 for (int w = 0; w < nq_tiles; ++w) {
-                    if (!(ok = mbar_wait(bar(B_PFULL + w), i & 1, ctl))) break;
+                    if (!(ok = MBAR_WAIT(bar(B_PFULL + w), i & 1, ctl))) break;
                     tc_fence_after();
                     issue_pv(w, st, i == 0);
                     // each release is committed only when a later fill waits for it,
                     // so no arrival is left pending at exit
-                    if (w == nq_tiles - 1 && i + kStages < n) mma_commit(bar(B_VEMPTY + st));
+                    if (w == nq_tiles - 1 && i + kStages < n) MMA_COMMIT(bar(B_VEMPTY + st));
                     if (!last) {
                         // K of tile i + 1 is needed from here on only: P.V of Q tile 0
                         // never waits for it
                         if (w == 0) {
-                            if (!(ok = mbar_wait(bar(B_KFULL + st1), ph1, ctl))) break;
+                            if (!(ok = MBAR_WAIT(bar(B_KFULL + st1), ph1, ctl))) break;
                             tc_fence_after();
                         }
                         issue_s(w, st1);
-                        mma_commit(bar(B_SFULL + w));
-                        if (w == nq_tiles - 1 && i + 1 + kStages < n) mma_commit(bar(B_KEMPTY + st1));
+                        MMA_COMMIT(bar(B_SFULL + w));
+                        if (w == nq_tiles - 1 && i + 1 + kStages < n) MMA_COMMIT(bar(B_KEMPTY + st1));
                     } else {
-                        mma_commit(bar(B_OFULL + w));
+                        MMA_COMMIT(bar(B_OFULL + w));
                     }
                 }
             }
             // drain: every MMA issued above has completed before teardown
-            mma_commit(bar(B_DRAIN));
+            MMA_COMMIT(bar(B_DRAIN));
             const uint64_t t0 = global_timer_ns();
             while (!mbar_try_wait(bar(B_DRAIN), 0)) {
                 if (global_timer_ns() - t0 > NOMAS_WAIT_NS) break;
             }
+#undef MMA_SS
+#undef MMA_TS
+#undef MMA_COMMIT
+#undef MBAR_WAIT
         }
     } else if (warp >= 4 && warp < 12) {
         // ================================================================ softmax
@@ -708,7 +730,39 @@ __global__ void __launch_bounds__(256) combine_kernel(const __grid_constant__ Co
     if (lane == 0 && a.lse) a.lse[static_cast<int64_t>(head) * a.nq + qrow] = (mmax + log2f(L)) * 0.69314718055994531f;
 }
 
+// One work item = 16 codes (16 bytes) of one row of K or V; 8 items per row,
+// consecutive threads on consecutive items, so loads (128 B per row) and
+// stores (256 B per row) are fully coalesced. Grid-stride over both tensors.
+__global__ void __launch_bounds__(512) dequant_window_kernel(const __grid_constant__ DequantArgs a) {
+    const uint32_t rows = static_cast<uint32_t>(a.heads) * static_cast<uint32_t>(a.nc); // per tensor, < 2^31
+    const uint32_t items = 2u * rows * 8u;                                              // < 2^32 by the host check
+    for (uint32_t it = blockIdx.x * blockDim.x + threadIdx.x; it < items; it += gridDim.x * blockDim.x) {
+        const uint32_t trow = it >> 3;
+        const uint32_t part = it & 7u;
+        const bool is_v = trow >= rows;
+        const uint32_t r = is_v ? trow - rows : trow;
+        const uint32_t head = fast_div(r, a.div_nc);
+        const uint32_t tok = r - head * static_cast<uint32_t>(a.nc);
+        const int64_t src_row = static_cast<int64_t>(head) * a.cap_tok + tok;
+        const uint4 w = __ldg(reinterpret_cast<const uint4*>((is_v ? a.vc : a.kc) + src_row * kD) + part);
+        const float sc = __ldg((is_v ? a.vs : a.ks) + src_row);
+        uint4* dst = reinterpret_cast<uint4*>((is_v ? a.vd : a.kd) + static_cast<int64_t>(r) * kD) + 2 * part;
+        dst[0] = dequant8(make_uint2(w.x, w.y), sc);
+        dst[1] = dequant8(make_uint2(w.z, w.w), sc);
+    }
+}
+
 } // namespace
+
+cudaError_t launch_dequant_window(const DequantArgs& a, cudaStream_t s) {
+    const uint64_t items = 2ull * static_cast<uint64_t>(a.heads) * static_cast<uint64_t>(a.nc) * 8ull;
+    if (items == 0) return cudaSuccess;
+    uint64_t blocks = (items + 511) / 512;
+    const uint64_t cap = 148ull * 4ull; // persistent: 4 blocks of 512 threads per SM
+    if (blocks > cap) blocks = cap;
+    dequant_window_kernel<<<static_cast<unsigned>(blocks), 512, 0, s>>>(a);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_attn(const AttnArgs& a, bool int8_cache, const CUtensorMap& tm_q, const CUtensorMap& tm_kcur,
                         const CUtensorMap& tm_vcur, const CUtensorMap& tm_kc, const CUtensorMap& tm_vc,

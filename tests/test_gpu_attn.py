@@ -14,16 +14,27 @@ from harness import MAX_ABS, REL_L2, current_segment, errors, make_caches, sampl
 pytestmark = pytest.mark.gpu
 
 
-def run_case(w, rows=None, check_lse=True, rel_l2=REL_L2):
+def run_case(w, rows=None, check_lse=True, rel_l2=REL_L2, path="once"):
+    """path: "once" = the workspace of nomas_seg_attn_workspace_bytes (an INT8 window is
+    dequantised once, then the BF16-cache kernel runs); "fused" = the minimum workspace
+    (the INT8 kernel converts each tile in shared memory)."""
     torch = __import__("torch")
     gpu, orc = make_caches(w)
     q, k, v = current_segment(w)
     nq = q.shape[0]
     lse = torch.full((w["heads"], nq), float("nan"), dtype=torch.float32, device="cuda")
     out = torch.full((nq, w["heads"], 128), float("nan"), dtype=torch.bfloat16, device="cuda")
-    gpu.seg_attn(to_dev(q), to_dev(k), to_dev(v), w["cur_frames"], w["n_text"], out=out, lse=lse)
+    ws = None
+    if path == "fused":
+        need = gpu.workspace_min_bytes(w["cur_frames"], w["n_text"])
+        if w["mode"] == "int8" and gpu.valid_frames > 0:
+            assert need < gpu.workspace_bytes(w["cur_frames"], w["n_text"])
+        ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    gpu.seg_attn(to_dev(q), to_dev(k), to_dev(v), w["cur_frames"], w["n_text"], out=out, lse=lse, workspace=ws)
     torch.cuda.synchronize()
     assert gpu.device_status() == 0
+    if ws is not None:
+        assert int(ws[:4].view(torch.int32).item()) == 0
     ref, ref_lse = orc.seg_attn(q, k, v, w["cur_frames"], w["n_text"], rows=rows)
     got = to_f64(out)
     got_lse = lse.cpu().numpy().astype(np.float64)
@@ -50,22 +61,28 @@ def test_tiny_workload():
     run_case(synth.WORKLOADS["tiny"])
 
 
-def test_tiny_int8():
-    run_case(wl(mode="int8", window=4, capacity=4, hist_commits=[1, 2]))
+INT8_PATHS = ["once", "fused"]
 
 
-@pytest.mark.parametrize("mode", ["bf16", "int8"])
-def test_ragged_tiles_and_tails(mode):
+@pytest.mark.parametrize("path", INT8_PATHS)
+def test_tiny_int8(path):
+    run_case(wl(mode="int8", window=4, capacity=4, hist_commits=[1, 2]), path=path)
+
+
+@pytest.mark.parametrize("mode,path", [("bf16", "once"), ("int8", "once"), ("int8", "fused")])
+def test_ragged_tiles_and_tails(mode, path):
     # 35 tokens/frame, 4 history frames = 140 keys (128 + 12); 5 frames + 37 text = 212 queries (128 + 84)
     run_case(wl(heads=3, grid_h=5, grid_w=7, mode=mode, window=4 if mode == "int8" else 0,
-                capacity=4 if mode == "int8" else 12, hist_commits=[3, 1], cur_frames=5, n_text=37, seed=5))
+                capacity=4 if mode == "int8" else 12, hist_commits=[3, 1], cur_frames=5, n_text=37, seed=5),
+             path=path)
 
 
-@pytest.mark.parametrize("mode", ["bf16", "int8"])
-def test_multi_tile_with_kv_splits(mode):
+@pytest.mark.parametrize("mode,path", [("bf16", "once"), ("int8", "once"), ("int8", "fused")])
+def test_multi_tile_with_kv_splits(mode, path):
     # 256 tokens/frame: 1536 cached keys (12 tiles), 868 queries (7 tiles): the split-KV + combine path
     run_case(wl(heads=4, grid_h=16, grid_w=16, mode=mode, window=6 if mode == "int8" else 0,
-                capacity=6 if mode == "int8" else 10, hist_commits=[2, 2, 2], cur_frames=3, n_text=100, seed=6))
+                capacity=6 if mode == "int8" else 10, hist_commits=[2, 2, 2], cur_frames=3, n_text=100, seed=6),
+             path=path)
 
 
 def test_no_history():
@@ -84,13 +101,15 @@ def test_video_only_segment_one_token_frames():
     run_case(wl(heads=2, grid_h=1, grid_w=1, hist_commits=[3], cur_frames=5, n_text=0, seed=10))
 
 
-def test_wrapped_int8_ring():
+@pytest.mark.parametrize("path", INT8_PATHS)
+def test_wrapped_int8_ring(path):
     # 7 frames committed through a 3-frame window; the visible history is the last 3
     run_case(wl(heads=2, grid_h=6, grid_w=8, mode="int8", window=3, capacity=3, hist_commits=[2, 4, 1],
-                cur_frames=2, n_text=10, seed=11))
+                cur_frames=2, n_text=10, seed=11), path=path)
 
 
-def test_peaky_softmax():
+@pytest.mark.parametrize("path", INT8_PATHS)
+def test_peaky_softmax(path):
     """Scores three times larger exercise the running-max rescaling of O.
 
     The kernel's operands are BF16 (rotated Q and K, dequantised cache, P),
@@ -101,17 +120,19 @@ def test_peaky_softmax():
     rel-L2 <= 1e-2 while keeping the max-abs bound of 2e-2.
     """
     run_case(wl(heads=2, grid_h=8, grid_w=16, mode="int8", window=4, capacity=4, hist_commits=[2, 2],
-                cur_frames=2, n_text=30, seed=12, q_std=3.0), rel_l2=1e-2)
+                cur_frames=2, n_text=30, seed=12, q_std=3.0), rel_l2=1e-2, path=path)
 
 
-def test_int8_split_mixing_cache_and_current_tiles():
+@pytest.mark.parametrize("path", INT8_PATHS)
+def test_int8_split_mixing_cache_and_current_tiles(path):
     """160 Q-tile pairs x 38 KV tiles: three KV splits, the middle one runs five
-    dequantised cache tiles and then TMA-loaded current-segment tiles."""
+    cache tiles and then current-segment tiles (fused path: dequantised cache
+    tiles, then TMA-loaded current tiles)."""
     w = wl(heads=16, grid_h=8, grid_w=16, mode="int8", window=18, capacity=18, hist_commits=[6, 6, 6],
            cur_frames=19, n_text=64, seed=15)
     F = 128
     nq = 19 * F + 64
-    run_case(w, rows=sample_rows(nq, F, 19, per_head=24))
+    run_case(w, rows=sample_rows(nq, F, 19, per_head=24), path=path)
 
 
 def test_repeated_calls_are_deterministic():
@@ -140,13 +161,31 @@ def test_cache_is_read_only():
     assert gpu.frames_committed == 2
 
 
-def test_single_gpu_configuration_sampled_rows():
+@pytest.mark.parametrize("path", INT8_PATHS)
+def test_single_gpu_configuration_sampled_rows(path):
     w = synth.WORKLOADS["single_gpu_int8_18f"]
     F = w["grid_h"] * w["grid_w"]
     nq = w["cur_frames"] * F + w["n_text"]
     rows = sample_rows(nq, F, w["cur_frames"], per_head=48)
-    mx, rel = run_case(w, rows=rows)
-    print(f"single-GPU cfg: max-abs {mx:.3e} rel-L2 {rel:.3e}")
+    mx, rel = run_case(w, rows=rows, path=path)
+    print(f"single-GPU cfg ({path}): max-abs {mx:.3e} rel-L2 {rel:.3e}")
+
+
+def test_int8_paths_agree():
+    """Both INT8 forms feed identical BF16 K/V values to the tensor cores; they
+    differ only in the softmax exponentials (part on the FMA pipe in the BF16
+    kernel), so their outputs agree far inside the oracle tolerance."""
+    torch = __import__("torch")
+    w = wl(heads=4, grid_h=16, grid_w=16, mode="int8", window=6, capacity=6, hist_commits=[3, 3], cur_frames=3,
+           n_text=100, seed=16)
+    gpu, _ = make_caches(w, with_oracle=False)
+    q, k, v = [to_dev(x) for x in current_segment(w)]
+    a = gpu.seg_attn(q, k, v, 3, 100).clone()
+    ws = torch.zeros(gpu.workspace_min_bytes(3, 100), dtype=torch.uint8, device="cuda")
+    b = gpu.seg_attn(q, k, v, 3, 100, workspace=ws)
+    torch.cuda.synchronize()
+    d = (a.float() - b.float()).abs()
+    assert d.max().item() <= 4e-3, d.max().item()
 
 
 @pytest.mark.slow
