@@ -179,8 +179,9 @@ void choose_splits(int units, int tiles, int& splits, int& tps) {
     }
 }
 
-// The dequantise-once kernel indexes (tensor, row, 16-code part) in 32 bits.
-bool dequant_once_fits(int heads, int64_t nc) { return static_cast<int64_t>(heads) * nc < (int64_t(1) << 28); }
+// The dequantise-once kernel indexes (tensor, row, 16-code part) in 32 bits,
+// with a few grid strides of headroom.
+bool dequant_once_fits(int heads, int64_t nc) { return static_cast<int64_t>(heads) * nc < (int64_t(1) << 27); }
 
 Plan make_plan(const nomas_cache* c, int32_t n_video_frames, int32_t n_text) {
     Plan p{};

@@ -83,24 +83,33 @@ __device__ __forceinline__ void unpack8(const uint4 x, float (&y)[8]) {
     }
 }
 
-// INT8 code of x for the row scale `scale` (inv = rn(1/scale)): the byte of
-// round-half-even(rn(x / scale)), the IEEE quotient's rounding.
-// x * inv lies within 2^-16 of the exact quotient (two roundings of at most
-// 2^-24 relative each, |x / scale| < 128), and so does the IEEE quotient; the
-// two can round to different integers only when a half-integer lies between
-// them. Away from half-integers (farther than 2^-14) the cheap product
-// decides; next to one, the exact division does. Rounding to an integer uses
-// the sum with 1.5 * 2^23: in [2^23, 2^24) the fp32 grid is the integers, so
-// the add rounds half to even, and the low byte of the sum's bit pattern is
-// the code in two's complement. |x / scale| <= 127 (1 + 3 * 2^-24) < 127.5, so
-// the code never needs clamping to [-127, 127].
+// INT8 code of x for the row scale `scale`: the byte of
+// round-half-even(rn(x / scale)), the IEEE quotient's rounding. `inv` is the
+// hardware reciprocal approximation of scale (rcp.approx, at most 1 ulp off):
+// x * inv lies within 1.5 * 2^-23 relative, i.e. 1.5 * 2^-16 absolute
+// (|x / scale| < 128), of the exact quotient, and the IEEE quotient within
+// 2^-17; the two can round to different integers only when a half-integer
+// lies between them. Away from half-integers (farther than 2^-14) the cheap
+// product decides; next to one -- or when the product is not finite, as for a
+// subnormal scale whose reciprocal overflows -- the exact division does.
+// Rounding to an integer uses the sum with 1.5 * 2^23: in [2^23, 2^24) the
+// fp32 grid is the integers, so the add rounds half to even, and the low byte
+// of the sum's bit pattern is the code in two's complement.
+// |x / scale| <= 127 (1 + 3 * 2^-24) < 127.5, so the code never needs clamping
+// to [-127, 127].
 __device__ __forceinline__ uint32_t quant_word(float x, float scale, float inv) {
     constexpr float kMagic = 12582912.0f; // 1.5 * 2^23
     const float q = __fmul_rn(x, inv);
     float t = __fadd_rn(q, kMagic);
-    const float f = __fsub_rn(q, __fsub_rn(t, kMagic)); // q - rint(q), exact
-    if (fabsf(f) > 0.5f - 6.103515625e-05f) t = __fadd_rn(__fdiv_rn(x, scale), kMagic);
+    const float f = __fsub_rn(q, __fsub_rn(t, kMagic)); // q - rint(q), exact; NaN if q is not finite
+    if (!(fabsf(f) <= 0.5f - 6.103515625e-05f)) t = __fadd_rn(__fdiv_rn(x, scale), kMagic);
     return __float_as_uint(t);
+}
+
+__device__ __forceinline__ float rcp_approx(float x) {
+    float y;
+    asm("rcp.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 
 // Half-warp INT8 quantisation of one row: returns 8 packed codes of this lane
@@ -116,7 +125,7 @@ __device__ __forceinline__ uint2 quantize8(const float (&y)[8], float& scale_out
         return make_uint2(0u, 0u);
     }
     const float scale = __fdiv_rn(amax, 127.0f);
-    const float inv = __fdiv_rn(1.0f, scale);
+    const float inv = rcp_approx(scale);
     scale_out = scale;
     uint32_t w[8];
 #pragma unroll

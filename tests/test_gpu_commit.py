@@ -103,3 +103,36 @@ def test_commit_large_segment_spans_several_launches():
         gpu.commit(to_dev(k), to_dev(v), nf)
         orc.commit(k, v, nf)
     assert_cache_equal(gpu, orc)
+
+
+def test_commit_subnormal_tiny_and_large_rows():
+    """Rows whose absmax is a BF16 subnormal (the row scale is then an fp32
+    subnormal and 1/scale overflows), rows of the smallest normals, rows near
+    2^97, and single-element rows: codes and scales stay bit-exact."""
+    import segment_causal_kv_b200 as nm
+    H, gh, gw, W = 2, 3, 4, 2
+    geo = synth.Geometry(H, gh, gw)
+    k, v = synth.history_kv(geo, 2, 94, 0)
+    rng = np.random.default_rng(5)
+    sign = (rng.integers(0, 2, size=128) << 15).astype(np.uint16)
+    sub = (rng.integers(0, 0x80, size=128).astype(np.uint16) | sign)
+    sub[::7] = 0
+    k[0, 0] = sub                                   # subnormal row, with zeros and both signs
+    v[1, 1] = sub
+    one = np.zeros(128, np.uint16)
+    one[17] = 0x0001                                # a single smallest subnormal
+    k[2, 1] = one
+    v[2, 0] = one | 0x8000
+    k[3, 0] = (k[3, 0] & 0x807F) | 0x0080           # smallest normal exponent
+    k[4, 1] = (k[4, 1] & 0x807F) | (0xE0 << 7)      # around 2^97
+    v[5, 0] = (v[5, 0] & 0x807F) | (0xE0 << 7)
+    gpu = nm.KVCache("int8", H, gh, gw, W, W)
+    orc = oracle.OracleCache(oracle.MODE_INT8, H, gh, gw, W, W)
+    gpu.commit(to_dev(k), to_dev(v), 2)
+    orc.commit(k, v, 2)
+    assert_cache_equal(gpu, orc)
+    F = gh * gw
+    # the subnormal row got a subnormal (nonzero) scale and non-trivial codes
+    s = gpu.k_scale.cpu().numpy()[0, 0]
+    assert 0.0 < s < 1.17549435e-38
+    assert gpu.k[0, 0].abs().max().item() == 127
