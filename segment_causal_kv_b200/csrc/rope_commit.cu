@@ -47,19 +47,22 @@ __device__ __forceinline__ void stage_tables(const RopeTab& tab, int n_t, int n_
     __syncthreads();
 }
 
-// cos/sin of the 4 pairs a lane owns (pairs 4*l .. 4*l+3 of the head).
+// cos/sin of the 4 pairs a lane owns (pairs 4*l .. 4*l+3 of the head): 32
+// contiguous bytes of one table row (t row for lanes 0-1, h row for 2-8, w row
+// for 9-15), read as two 16-byte loads from an address picked without
+// branching, so the half-warp's three axis groups do not diverge. Row starts
+// and in-row offsets are multiples of 32 bytes (t rows 64 B, h/w rows 224 B).
 __device__ __forceinline__ void lane_coeffs(int l, int frame, int hh, int ww, int grid_h, const float2* s_t,
                                             const float2* s_hw, float2 (&cs)[4]) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int p = 4 * l + i;
-        if (l < 2)
-            cs[i] = s_t[frame * kTPairs + p];
-        else if (l < 9)
-            cs[i] = s_hw[hh * kHWPairs + (p - kTPairs)];
-        else
-            cs[i] = s_hw[(grid_h + ww) * kHWPairs + (p - kTPairs - kHWPairs)];
-    }
+    const float2* src = l < 2 ? s_t + frame * kTPairs + 4 * l
+                              : s_hw + (l < 9 ? hh * kHWPairs + (4 * l - kTPairs)
+                                              : (grid_h + ww) * kHWPairs + (4 * l - kTPairs - kHWPairs));
+    const float4 a = reinterpret_cast<const float4*>(src)[0];
+    const float4 b = reinterpret_cast<const float4*>(src)[1];
+    cs[0] = make_float2(a.x, a.y);
+    cs[1] = make_float2(a.z, a.w);
+    cs[2] = make_float2(b.x, b.y);
+    cs[3] = make_float2(b.z, b.w);
 }
 
 // y0 = fma(x0, c, -rn(x1*s)), y1 = fma(x0, s, rn(x1*c)) on 4 pairs.
@@ -113,7 +116,11 @@ __device__ __forceinline__ float rcp_approx(float x) {
 }
 
 // Half-warp INT8 quantisation of one row: returns 8 packed codes of this lane
-// and the row scale. Both half-warps of a warp must call it together.
+// and the row scale. Both half-warps of a warp must call it together. The
+// fast path of quant_word runs on packed pairs for all 8 values with a single
+// branch to the exact per-value path when any of them is near a half-integer
+// (or not finite); packed fp32 operations round each half exactly as the
+// scalar ones do.
 __device__ __forceinline__ uint2 quantize8(const float (&y)[8], float& scale_out) {
     float amax = 0.0f;
 #pragma unroll
@@ -127,9 +134,24 @@ __device__ __forceinline__ uint2 quantize8(const float (&y)[8], float& scale_out
     const float scale = __fdiv_rn(amax, 127.0f);
     const float inv = rcp_approx(scale);
     scale_out = scale;
+    constexpr float kMagic = 12582912.0f; // 1.5 * 2^23
+    constexpr float kNear = 0.5f - 6.103515625e-05f;
     uint32_t w[8];
+    bool near = false;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) w[i] = quant_word(y[i], scale, inv);
+    for (int i = 0; i < 4; ++i) {
+        const float2 q = __fmul2_rn(make_float2(y[2 * i], y[2 * i + 1]), make_float2(inv, inv));
+        const float2 t = __fadd2_rn(q, make_float2(kMagic, kMagic));
+        const float2 r = __fadd2_rn(t, make_float2(-kMagic, -kMagic));
+        const float2 f = __ffma2_rn(r, make_float2(-1.0f, -1.0f), q); // q - rint(q), exact; NaN if q is not finite
+        near |= !(fabsf(f.x) <= kNear && fabsf(f.y) <= kNear);
+        w[2 * i] = __float_as_uint(t.x);
+        w[2 * i + 1] = __float_as_uint(t.y);
+    }
+    if (near) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) w[i] = quant_word(y[i], scale, inv);
+    }
     // low bytes of w[0..7], in order
     uint2 r;
     r.x = __byte_perm(__byte_perm(w[0], w[1], 0x0040u), __byte_perm(w[2], w[3], 0x0040u), 0x5410u);
@@ -139,8 +161,8 @@ __device__ __forceinline__ uint2 quantize8(const float (&y)[8], float& scale_out
 
 __global__ void __launch_bounds__(kThreads) commit_kernel(const __grid_constant__ CommitArgs a,
                                                           const __grid_constant__ RopeTab tab) {
-    __shared__ float2 s_t[kMaxFramesPerLaunch * kTPairs];
-    __shared__ float2 s_hw[NOMAS_MAX_GRID_HW * kHWPairs];
+    __shared__ __align__(16) float2 s_t[kMaxFramesPerLaunch * kTPairs];
+    __shared__ __align__(16) float2 s_hw[NOMAS_MAX_GRID_HW * kHWPairs];
     stage_tables(tab, a.n_frames, a.grid_h + a.grid_w, s_t, s_hw);
 
     const int lane = threadIdx.x & 31;
@@ -224,8 +246,8 @@ __global__ void __launch_bounds__(kThreads) commit_kernel(const __grid_constant_
 
 __global__ void __launch_bounds__(kThreads) prep_kernel(const __grid_constant__ PrepArgs a,
                                                         const __grid_constant__ RopeTab tab) {
-    __shared__ float2 s_t[kMaxFramesPerLaunch * kTPairs];
-    __shared__ float2 s_hw[NOMAS_MAX_GRID_HW * kHWPairs];
+    __shared__ __align__(16) float2 s_t[kMaxFramesPerLaunch * kTPairs];
+    __shared__ __align__(16) float2 s_hw[NOMAS_MAX_GRID_HW * kHWPairs];
     const int vid_lo = a.tok0 < a.nv ? a.tok0 : a.nv;
     const int vid_hi = a.tok1 < a.nv ? a.tok1 : a.nv;
     const int n_t = vid_hi > vid_lo ? (vid_hi - 1) / a.tpf - a.frame0 + 1 : 0;
