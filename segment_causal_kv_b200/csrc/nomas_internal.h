@@ -62,6 +62,8 @@ struct CommitArgs {
     int32_t slot0;          // slot of the first frame of this launch
     int32_t int8_mode;
     FastDiv div_heads, div_tpf, div_gw;
+    int32_t head_group;     // heads of one token handled by one warp task (set by launch_commit)
+    FastDiv div_groups;     // ceil(heads / head_group)
 };
 
 struct PrepArgs {

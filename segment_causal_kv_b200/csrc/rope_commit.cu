@@ -7,14 +7,15 @@
 //  * prep_kernel: RoPE of the current segment's Q and K, BF16 out, relayout
 //    token-major -> head-major for the attention kernel's TMA loads.
 //
-// Work split: a half-warp owns one (token, head) row of 128 elements; each
-// lane moves 16 bytes (8 BF16 = 4 RoPE pairs) with one 128-bit load per
-// tensor. The 16 lanes of a row fall into exactly one RoPE axis block each
-// (lanes 0-1: t, 2-8: h, 9-15: w). Rows are visited in token-major order so
-// reads are contiguous; every row write is one full 128-byte (codes) or
-// 256-byte (BF16) run. The RoPE tables arrive as launch arguments and are
-// staged once per block into shared memory; the grid is persistent (two
-// blocks per SM) so the staging is paid a few hundred times, not per row.
+// Work split: a half-warp owns one (token, head) row of 128 elements at a
+// time; each lane moves 16 bytes (8 BF16 = 4 RoPE pairs) with one 128-bit load
+// per tensor. The 16 lanes of a row fall into exactly one RoPE axis block each
+// (lanes 0-1: t, 2-8: h, 9-15: w). In the commit a warp walks the heads of one
+// token (or of a group of its heads), so position, RoPE coefficients and ring
+// slot are set up once per token; every row write is one full 128-byte
+// (codes) or 256-byte (BF16) run. The RoPE tables arrive as launch arguments
+// and are staged once per block into shared memory; the grid is persistent
+// (two blocks per SM) so the staging is paid a few hundred times, not per row.
 //
 // Commit arithmetic is fixed bit for bit: products and fused multiply-adds
 // use the _rn intrinsics (no contraction freedom), the scale is an IEEE
@@ -115,40 +116,56 @@ __device__ __forceinline__ float rcp_approx(float x) {
     return y;
 }
 
+// RN(x / 127) for a finite x >= 0, by Markstein's division (P. Markstein,
+// "Computation of elementary functions on the IBM RISC System/6000
+// processor", IBM J. Res. Dev. 34(1), 1990): with r = RN(1/127) and
+// q0 = RN(x * r) within an ulp of x / 127, the remainder e = x - 127 q0 is
+// exact in one fma and q1 = RN(q0 + e * r) is the correctly rounded quotient
+// while nothing underflows. Below 2^-100, and for a non-finite x, the IEEE
+// division is used instead. Checked against the IEEE division for every
+// non-negative fp32 x.
+__device__ __forceinline__ float div127_rn(float x) {
+    if (!(x >= 7.8886090522101181e-31f && x <= 3.4028234663852886e38f)) return __fdiv_rn(x, 127.0f); // 2^-100
+    constexpr float r = 1.0f / 127.0f;                            // RN(1/127), folded at compile time
+    const float q0 = __fmul_rn(x, r);
+    const float e = __fmaf_rn(-q0, 127.0f, x);
+    return __fmaf_rn(e, r, q0);
+}
+
 // Half-warp INT8 quantisation of one row: returns 8 packed codes of this lane
 // and the row scale. Both half-warps of a warp must call it together. The
-// fast path of quant_word runs on packed pairs for all 8 values with a single
-// branch to the exact per-value path when any of them is near a half-integer
-// (or not finite); packed fp32 operations round each half exactly as the
-// scalar ones do.
+// fast path of quant_word runs on packed pairs for all 8 values; one test of
+// the largest distance to the nearest integer (and of the reciprocal being
+// finite, which makes every product finite) sends the lane to the exact
+// per-value path when any value needs it. Packed fp32 operations round each
+// half exactly as the scalar ones do.
 __device__ __forceinline__ uint2 quantize8(const float (&y)[8], float& scale_out) {
-    float amax = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(y[i]));
+    float amax = fmaxf(fmaxf(fmaxf(fabsf(y[0]), fabsf(y[1])), fmaxf(fabsf(y[2]), fabsf(y[3]))),
+                       fmaxf(fmaxf(fabsf(y[4]), fabsf(y[5])), fmaxf(fabsf(y[6]), fabsf(y[7]))));
 #pragma unroll
     for (int off = 8; off >= 1; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off, 16));
     if (amax == 0.0f) {
         scale_out = 0.0f;
         return make_uint2(0u, 0u);
     }
-    const float scale = __fdiv_rn(amax, 127.0f);
+    const float scale = div127_rn(amax);
     const float inv = rcp_approx(scale);
     scale_out = scale;
     constexpr float kMagic = 12582912.0f; // 1.5 * 2^23
     constexpr float kNear = 0.5f - 6.103515625e-05f;
     uint32_t w[8];
-    bool near = false;
+    float fmax_abs = 0.0f;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const float2 q = __fmul2_rn(make_float2(y[2 * i], y[2 * i + 1]), make_float2(inv, inv));
         const float2 t = __fadd2_rn(q, make_float2(kMagic, kMagic));
         const float2 r = __fadd2_rn(t, make_float2(-kMagic, -kMagic));
-        const float2 f = __ffma2_rn(r, make_float2(-1.0f, -1.0f), q); // q - rint(q), exact; NaN if q is not finite
-        near |= !(fabsf(f.x) <= kNear && fabsf(f.y) <= kNear);
+        const float2 f = __ffma2_rn(r, make_float2(-1.0f, -1.0f), q); // q - rint(q), exact
+        fmax_abs = fmaxf(fmax_abs, fmaxf(fabsf(f.x), fabsf(f.y)));
         w[2 * i] = __float_as_uint(t.x);
         w[2 * i + 1] = __float_as_uint(t.y);
     }
-    if (near) {
+    if (!(fmax_abs <= kNear && inv <= 3.4028234663852886e38f)) {
 #pragma unroll
         for (int i = 0; i < 8; ++i) w[i] = quant_word(y[i], scale, inv);
     }
@@ -159,56 +176,59 @@ __device__ __forceinline__ uint2 quantize8(const float (&y)[8], float& scale_out
     return r;
 }
 
+template <bool kGrouped>
 __global__ void __launch_bounds__(kThreads) commit_kernel(const __grid_constant__ CommitArgs a,
                                                           const __grid_constant__ RopeTab tab) {
     __shared__ __align__(16) float2 s_t[kMaxFramesPerLaunch * kTPairs];
     __shared__ __align__(16) float2 s_hw[NOMAS_MAX_GRID_HW * kHWPairs];
     stage_tables(tab, a.n_frames, a.grid_h + a.grid_w, s_t, s_hw);
 
+    // A warp task is one token and a group of `head_group` of its heads; the
+    // two half-warps walk the group's heads h = g0 + half, g0 + half + 2, ...
+    // (one (token, head) row per half-warp per step). Position, RoPE
+    // coefficients and ring slot depend only on the token, so they are set up
+    // once per task. The next row's K and V are loaded while the current one
+    // is processed, across task boundaries too. Large commits use all heads
+    // per task; a commit with too few tokens to fill the GPU splits them.
+    // All index math is 32-bit (rows of one launch < 2^31).
     const int lane = threadIdx.x & 31;
     const int half = lane >> 4;
     const int l = lane & 15;
-    // row r of this launch: token r / heads (frame-major), head r % heads; all
-    // index math is 32-bit with constant-divisor division (rows < 2^31)
-    const uint32_t rows = static_cast<uint32_t>(a.n_frames) * a.tpf * a.heads;
+    const uint32_t groups = kGrouped ? a.div_groups.d : 1u;
+    const uint32_t tasks = static_cast<uint32_t>(a.n_frames) * a.tpf * groups;
     const uint32_t warps = gridDim.x * (kThreads / 32);
-    auto in_offset = [&](uint32_t r) {
-        const uint32_t tok = fast_div(r, a.div_heads);
-        const uint32_t h = r - tok * a.heads;
-        const int64_t in_tok = static_cast<int64_t>(a.in_frame0) * a.tpf + tok;
-        return in_tok * a.token_stride + h * kD + l * 8;
+    const int steps = ((kGrouped ? a.head_group : a.heads) + 1) >> 1; // rows per half-warp per task
+    const int64_t tok0 = static_cast<int64_t>(a.in_frame0) * a.tpf;
+    auto row_ptr = [&](const uint16_t* base, uint32_t tok, int h) {
+        return reinterpret_cast<const uint4*>(base + (tok0 + tok) * a.token_stride + h * kD + l * 8);
     };
-    // software pipeline: the next row pair's K and V are in flight while this one is processed
-    uint32_t wp = blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
-    uint4 kx = make_uint4(0, 0, 0, 0), vx = kx;
-    if (wp * 2 < rows) {
-        const uint32_t r0 = min(wp * 2 + half, rows - 1);
-        kx = __ldg(reinterpret_cast<const uint4*>(a.k + in_offset(r0)));
-        vx = __ldg(reinterpret_cast<const uint4*>(a.v + in_offset(r0)));
-    }
-    for (; wp * 2 < rows; wp += warps) {
-        const uint32_t r = wp * 2 + half;
-        const bool valid = r < rows;
-        const uint32_t rr = valid ? r : rows - 1;
-        uint4 kn = kx, vn = vx;
-        if ((wp + warps) * 2 < rows) {
-            const uint32_t rn = min((wp + warps) * 2 + half, rows - 1);
-            kn = __ldg(reinterpret_cast<const uint4*>(a.k + in_offset(rn)));
-            vn = __ldg(reinterpret_cast<const uint4*>(a.v + in_offset(rn)));
+    // token of a task and the first head of its group
+    auto task_token = [&](uint32_t t, uint32_t& tk) {
+        if (!kGrouped) {
+            tk = t;
+            return 0;
         }
-        const uint32_t tok = fast_div(rr, a.div_heads);
-        const uint32_t h = rr - tok * a.heads;
+        tk = fast_div(t, a.div_groups);
+        return static_cast<int>(t - tk * groups) * a.head_group;
+    };
+    uint32_t task = blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
+    uint4 kx = make_uint4(0, 0, 0, 0), vx = kx;
+    if (task < tasks) {
+        uint32_t tk;
+        const int h0 = min(task_token(task, tk) + half, a.heads - 1); // out-of-range heads load a valid row, not stored
+        kx = __ldg(row_ptr(a.k, tk, h0));
+        vx = __ldg(row_ptr(a.v, tk, h0));
+    }
+    for (; task < tasks; task += warps) {
+        uint32_t tok;
+        const int g0 = task_token(task, tok);
+        const int g1 = kGrouped ? min(g0 + a.head_group, a.heads) : a.heads; // heads [g0, g1) in this task
         const uint32_t fi = fast_div(tok, a.div_tpf);
         const uint32_t rif = tok - fi * a.tpf;
         const uint32_t hh = fast_div(rif, a.div_gw);
         const uint32_t ww = rif - hh * a.grid_w;
-
         float2 cs[4];
         lane_coeffs(l, fi, hh, ww, a.grid_h, s_t, s_hw, cs);
-        float ky[8], vy[8];
-        rotate8(kx, cs, ky);
-        unpack8(vx, vy);
-
         // slot of frame fi: ring slots advance with the frame (fi < window within a launch)
         int64_t slot;
         if (a.window > 0) {
@@ -217,30 +237,51 @@ __global__ void __launch_bounds__(kThreads) commit_kernel(const __grid_constant_
         } else {
             slot = a.abs_frame0 + fi;
         }
-        const int64_t row = static_cast<int64_t>(h) * a.cap_tok + slot * a.tpf + rif;
-        if (a.int8_mode) {
-            float ks, vs;
-            const uint2 kc = quantize8(ky, ks);
-            const uint2 vc = quantize8(vy, vs);
-            if (valid) {
-                *reinterpret_cast<uint2*>(static_cast<int8_t*>(a.ck) + row * kD + l * 8) = kc;
-                *reinterpret_cast<uint2*>(static_cast<int8_t*>(a.cv) + row * kD + l * 8) = vc;
-                if (l == 0) {
-                    a.cks[row] = ks;
-                    a.cvs[row] = vs;
-                }
+        const int64_t row0 = slot * a.tpf + rif; // row of head 0; head h adds h * cap_tok
+        const uint32_t task_next = task + warps;
+        for (int j = 0; j < steps; ++j) {
+            const int h = g0 + 2 * j + half;
+            const bool valid = h < g1;
+            // next row of this half-warp: the following head, or the first of the next task
+            uint4 kn = kx, vn = vx;
+            if (j + 1 < steps) {
+                const int hn = min(h + 2, a.heads - 1);
+                kn = __ldg(row_ptr(a.k, tok, hn));
+                vn = __ldg(row_ptr(a.v, tok, hn));
+            } else if (task_next < tasks) {
+                uint32_t tn;
+                const int hn = min(task_token(task_next, tn) + half, a.heads - 1);
+                kn = __ldg(row_ptr(a.k, tn, hn));
+                vn = __ldg(row_ptr(a.v, tn, hn));
             }
-        } else if (valid) {
-            uint4 ko;
-            ko.x = rne_bf16x2(ky[0], ky[1]);
-            ko.y = rne_bf16x2(ky[2], ky[3]);
-            ko.z = rne_bf16x2(ky[4], ky[5]);
-            ko.w = rne_bf16x2(ky[6], ky[7]);
-            *reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.ck) + row * kD + l * 8) = ko;
-            *reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.cv) + row * kD + l * 8) = vx;
+            float ky[8], vy[8];
+            rotate8(kx, cs, ky);
+            unpack8(vx, vy);
+            const int64_t row = static_cast<int64_t>(valid ? h : 0) * a.cap_tok + row0;
+            if (a.int8_mode) {
+                float ks, vs;
+                const uint2 kc = quantize8(ky, ks);
+                const uint2 vc = quantize8(vy, vs);
+                if (valid) {
+                    *reinterpret_cast<uint2*>(static_cast<int8_t*>(a.ck) + row * kD + l * 8) = kc;
+                    *reinterpret_cast<uint2*>(static_cast<int8_t*>(a.cv) + row * kD + l * 8) = vc;
+                    if (l == 0) {
+                        a.cks[row] = ks;
+                        a.cvs[row] = vs;
+                    }
+                }
+            } else if (valid) {
+                uint4 ko;
+                ko.x = rne_bf16x2(ky[0], ky[1]);
+                ko.y = rne_bf16x2(ky[2], ky[3]);
+                ko.z = rne_bf16x2(ky[4], ky[5]);
+                ko.w = rne_bf16x2(ky[6], ky[7]);
+                *reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.ck) + row * kD + l * 8) = ko;
+                *reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.cv) + row * kD + l * 8) = vx;
+            }
+            kx = kn;
+            vx = vn;
         }
-        kx = kn;
-        vx = vn;
     }
 }
 
@@ -308,9 +349,22 @@ int grid_for(int64_t work_items, int items_per_block) {
 
 } // namespace
 
-cudaError_t launch_commit(const CommitArgs& a, const RopeTab& tab, cudaStream_t s) {
-    const int64_t rows = static_cast<int64_t>(a.n_frames) * a.tpf * a.heads;
-    commit_kernel<<<grid_for(rows, kThreads / 16), kThreads, 0, s>>>(a, tab);
+cudaError_t launch_commit(const CommitArgs& a_in, const RopeTab& tab, cudaStream_t s) {
+    // heads per warp task: all of a token's heads when there are enough tokens
+    // to give every resident warp several tasks, else halves of that, down to 2,
+    // so that small commits still spread over the GPU
+    CommitArgs a = a_in;
+    const int64_t tokens = static_cast<int64_t>(a.n_frames) * a.tpf;
+    const int64_t want = 4ll * 148 * 2 * (kThreads / 32);
+    int hg = a.heads;
+    while (hg > 2 && tokens * ((a.heads + hg - 1) / hg) < want) hg = (hg + 1) / 2;
+    a.head_group = hg;
+    a.div_groups = make_fastdiv(static_cast<uint32_t>((a.heads + hg - 1) / hg));
+    const int64_t tasks = tokens * a.div_groups.d;
+    if (hg < a.heads)
+        commit_kernel<true><<<grid_for(tasks, kThreads / 32), kThreads, 0, s>>>(a, tab);
+    else
+        commit_kernel<false><<<grid_for(tasks, kThreads / 32), kThreads, 0, s>>>(a, tab);
     return cudaGetLastError();
 }
 
