@@ -176,7 +176,7 @@ __device__ __forceinline__ uint2 quantize8(const float (&y)[8], float& scale_out
     return r;
 }
 
-template <bool kGrouped>
+template <bool kGrouped, bool kInt8>
 __global__ void __launch_bounds__(kThreads) commit_kernel(const __grid_constant__ CommitArgs a,
                                                           const __grid_constant__ RopeTab tab) {
     __shared__ __align__(16) float2 s_t[kMaxFramesPerLaunch * kTPairs];
@@ -258,7 +258,7 @@ __global__ void __launch_bounds__(kThreads) commit_kernel(const __grid_constant_
             rotate8(kx, cs, ky);
             unpack8(vx, vy);
             const int64_t row = static_cast<int64_t>(valid ? h : 0) * a.cap_tok + row0;
-            if (a.int8_mode) {
+            if (kInt8) {
                 float ks, vs;
                 const uint2 kc = quantize8(ky, ks);
                 const uint2 vc = quantize8(vy, vs);
@@ -361,10 +361,14 @@ cudaError_t launch_commit(const CommitArgs& a_in, const RopeTab& tab, cudaStream
     a.head_group = hg;
     a.div_groups = make_fastdiv(static_cast<uint32_t>((a.heads + hg - 1) / hg));
     const int64_t tasks = tokens * a.div_groups.d;
-    if (hg < a.heads)
-        commit_kernel<true><<<grid_for(tasks, kThreads / 32), kThreads, 0, s>>>(a, tab);
-    else
-        commit_kernel<false><<<grid_for(tasks, kThreads / 32), kThreads, 0, s>>>(a, tab);
+    const int grid = grid_for(tasks, kThreads / 32);
+    if (hg < a.heads) {
+        if (a.int8_mode) commit_kernel<true, true><<<grid, kThreads, 0, s>>>(a, tab);
+        else commit_kernel<true, false><<<grid, kThreads, 0, s>>>(a, tab);
+    } else {
+        if (a.int8_mode) commit_kernel<false, true><<<grid, kThreads, 0, s>>>(a, tab);
+        else commit_kernel<false, false><<<grid, kThreads, 0, s>>>(a, tab);
+    }
     return cudaGetLastError();
 }
 
