@@ -144,6 +144,26 @@ int nomas_kv_commit(nomas_cache *c, const void *k, const void *v, int64_t token_
                     void *stream);
 
 /*
+ * nomas_kv_commit_layers -- nomas_kv_commit of one finished segment into
+ * n_layers per-layer caches at once (one launch per 24 layers instead of one
+ * per layer). The pages describe the per-layer commit; batching the layers of
+ * a model step is a service of this library.
+ *   caches : host array of n_layers descriptors (distinct caches) that share
+ *            mode, heads, grid, window, capacity, theta and ring state
+ *            (frames_committed, valid_frames, head_slot), e.g. the layers of
+ *            one model advanced in lockstep.
+ *   k, v   : host arrays of n_layers device pointers, each laid out as for
+ *            nomas_kv_commit, all with the same token_stride.
+ * Every layer's cache receives exactly what nomas_kv_commit would write, and
+ * every descriptor's state advances by n_frames.
+ * Errors: as nomas_kv_commit, plus NOMAS_ERR_ARG (n_layers < 1, a NULL entry,
+ * one cache given twice) and NOMAS_ERR_STATE (descriptors that differ in
+ * configuration or state). All checks happen before anything is enqueued.
+ */
+int nomas_kv_commit_layers(nomas_cache *const *caches, const void *const *k, const void *const *v,
+                           int64_t token_stride, int32_t n_layers, int32_t n_frames, void *stream);
+
+/*
  * nomas_seg_attn_workspace_bytes -- device workspace for the fastest form of
  * nomas_seg_attn for this cache state and segment shape (0 on invalid
  * arguments). For an INT8 cache it includes a BF16 copy of the visible window

@@ -34,7 +34,7 @@ NOMAS_CACHE_INT8 = 1
 HEAD_DIM = 128
 
 # exported symbols (checked against include/nomas.h by the tests)
-EXPORTS = ("nomas_cache_reset", "nomas_kv_commit", "nomas_seg_attn_workspace_bytes",
+EXPORTS = ("nomas_cache_reset", "nomas_kv_commit", "nomas_kv_commit_layers", "nomas_seg_attn_workspace_bytes",
            "nomas_seg_attn_workspace_min_bytes", "nomas_seg_attn",
            "nomas_device_status", "nomas_status_string", "nomas_seg_attn_static", "nomas_selftest_bounded_wait")
 NOMAS_STATIC_SCRATCH_BYTES = 64 << 20
@@ -85,6 +85,8 @@ def lib():
         L.nomas_cache_reset.restype = ctypes.c_int
         L.nomas_kv_commit.argtypes = [D, P, P, I64, I32, P]
         L.nomas_kv_commit.restype = ctypes.c_int
+        L.nomas_kv_commit_layers.argtypes = [ctypes.POINTER(D), ctypes.POINTER(P), ctypes.POINTER(P), I64, I32, I32, P]
+        L.nomas_kv_commit_layers.restype = ctypes.c_int
         L.nomas_seg_attn_workspace_bytes.argtypes = [D, I32, I32]
         L.nomas_seg_attn_workspace_bytes.restype = ctypes.c_size_t
         L.nomas_seg_attn_workspace_min_bytes.argtypes = [D, I32, I32]
@@ -116,6 +118,28 @@ def nomas_cache_reset(desc: NomasCacheDesc) -> int:
 def nomas_kv_commit(desc: NomasCacheDesc, k_ptr: int, v_ptr: int, token_stride: int, n_frames: int,
                     stream: int | None) -> int:
     return lib().nomas_kv_commit(ctypes.byref(desc), k_ptr, v_ptr, token_stride, n_frames, stream)
+
+
+def nomas_kv_commit_layers(descs, k_ptrs, v_ptrs, token_stride: int, n_frames: int, stream: int | None) -> int:
+    """Commit one segment into several layer caches in one call (descs: NomasCacheDesc objects)."""
+    n = len(descs)
+    if not (len(k_ptrs) == len(v_ptrs) == n):
+        raise ValueError("one K and one V pointer per cache")
+    D = ctypes.POINTER(NomasCacheDesc)
+    darr = (D * n)(*[ctypes.pointer(d) for d in descs])
+    karr = (ctypes.c_void_p * n)(*k_ptrs)
+    varr = (ctypes.c_void_p * n)(*v_ptrs)
+    return lib().nomas_kv_commit_layers(darr, karr, varr, token_stride, n, n_frames, stream)
+
+
+def commit_layers(caches, ks, vs, n_frames: int, stream=None) -> None:
+    """nomas_kv_commit_layers for KVCache objects and per-layer BF16 K/V tensors sharing one layout."""
+    assert len(caches) == len(ks) == len(vs) and len(caches) > 0
+    torch = _torch()
+    for k, v in zip(ks, vs):
+        assert k.dtype == torch.bfloat16 and v.dtype == k.dtype and k.stride() == v.stride() == ks[0].stride()
+    _check(nomas_kv_commit_layers([c.desc for c in caches], [k.data_ptr() for k in ks], [v.data_ptr() for v in vs],
+                                  ks[0].stride(0), n_frames, _stream_handle(stream)), "nomas_kv_commit_layers")
 
 
 def nomas_seg_attn_workspace_bytes(desc: NomasCacheDesc, n_video_frames: int, n_text: int) -> int:

@@ -224,19 +224,42 @@ int nomas_cache_reset(nomas_cache* c) {
     return NOMAS_OK;
 }
 
-int nomas_kv_commit(nomas_cache* c, const void* k, const void* v, int64_t token_stride, int32_t n_frames,
-                    void* stream) {
+// Commit of one finished segment into n layer caches that share configuration
+// and state (the single-layer call is n == 1). Everything is validated before
+// anything is enqueued; the host counters of every cache advance together.
+static int commit_layers(nomas_cache* const* cs, const void* const* ks, const void* const* vs, int64_t token_stride,
+                         int32_t n_layers, int32_t n_frames, void* stream) {
+    if (!cs || n_layers < 1) return NOMAS_ERR_ARG;
+    for (int i = 0; i < n_layers; ++i)
+        if (!cs[i]) return NOMAS_ERR_ARG;
+    const nomas_cache* c = cs[0];
     int rc = validate_state(c);
     if (rc != NOMAS_OK) return rc;
+    for (int i = 1; i < n_layers; ++i) {
+        const nomas_cache* o = cs[i];
+        if ((rc = validate_state(o)) != NOMAS_OK) return rc;
+        if (o->mode != c->mode || o->heads != c->heads || o->grid_h != c->grid_h || o->grid_w != c->grid_w ||
+            o->window_frames != c->window_frames || o->capacity_frames != c->capacity_frames ||
+            o->rope_theta != c->rope_theta || o->frames_committed != c->frames_committed ||
+            o->valid_frames != c->valid_frames || o->head_slot != c->head_slot)
+            return NOMAS_ERR_STATE;
+        for (int j = 0; j < i; ++j)
+            if (cs[j] == o || cs[j]->k == o->k || cs[j]->v == o->v) return NOMAS_ERR_ARG; // one cache twice
+    }
     if (n_frames < 0) return NOMAS_ERR_ARG;
     if (n_frames == 0) return NOMAS_OK;
-    if (!k || !v) return NOMAS_ERR_ARG;
+    if (!ks || !vs) return NOMAS_ERR_ARG;
     if (token_stride < static_cast<int64_t>(c->heads) * kD || token_stride % 8 != 0) return NOMAS_ERR_ARG;
-    if (!aligned(k, 16) || !aligned(v, 16)) return NOMAS_ERR_ALIGN;
+    for (int i = 0; i < n_layers; ++i) {
+        if (!ks[i] || !vs[i]) return NOMAS_ERR_ARG;
+        if (!aligned(ks[i], 16) || !aligned(vs[i], 16)) return NOMAS_ERR_ALIGN;
+    }
     const int W = c->window_frames;
     if (W == 0 && c->frames_committed + n_frames > c->capacity_frames) return NOMAS_ERR_CAPACITY;
-    if (static_cast<int64_t>(kMaxFramesPerLaunch) * c->grid_h * c->grid_w * c->heads >= (int64_t(1) << 31))
-        return NOMAS_ERR_ARG; // one launch's (token, head) rows must fit 31 bits
+    const int64_t layers_per_launch = n_layers < kMaxLayersPerLaunch ? n_layers : kMaxLayersPerLaunch;
+    if (static_cast<int64_t>(kMaxFramesPerLaunch) * c->grid_h * c->grid_w * c->heads * layers_per_launch >=
+        (int64_t(1) << 31))
+        return NOMAS_ERR_ARG; // one launch's (layer, token, head) rows must fit 31 bits
     if ((rc = check_device()) != NOMAS_OK) return rc;
 
     const int tpf = c->grid_h * c->grid_w;
@@ -247,13 +270,7 @@ int nomas_kv_commit(nomas_cache* c, const void* k, const void* v, int64_t token_
     for (int f0 = first; f0 < n_frames; f0 += kMaxFramesPerLaunch) {
         const int nf = (n_frames - f0) < kMaxFramesPerLaunch ? (n_frames - f0) : kMaxFramesPerLaunch;
         CommitArgs a{};
-        a.k = static_cast<const uint16_t*>(k);
-        a.v = static_cast<const uint16_t*>(v);
         a.token_stride = token_stride;
-        a.ck = c->k;
-        a.cv = c->v;
-        a.cks = c->k_scale;
-        a.cvs = c->v_scale;
         a.cap_tok = static_cast<int64_t>(c->capacity_frames) * tpf;
         a.heads = c->heads;
         a.tpf = tpf;
@@ -269,17 +286,47 @@ int nomas_kv_commit(nomas_cache* c, const void* k, const void* v, int64_t token_
         a.div_tpf = make_fastdiv(static_cast<uint32_t>(tpf));
         a.div_gw = make_fastdiv(static_cast<uint32_t>(c->grid_w));
         fill_t(tab, c->rope_theta, a.abs_frame0, nf);
-        if (launch_commit(a, tab, s) != cudaSuccess) return NOMAS_ERR_CUDA;
+        // launches of equal size (54 layers: 3 x 18, not 24 + 24 + 6)
+        const int n_launch = (n_layers + kMaxLayersPerLaunch - 1) / kMaxLayersPerLaunch;
+        const int per_launch = (n_layers + n_launch - 1) / n_launch;
+        for (int l0 = 0; l0 < n_layers; l0 += per_launch) {
+            const int nl = (n_layers - l0) < per_launch ? (n_layers - l0) : per_launch;
+            CommitLayers L{};
+            for (int i = 0; i < nl; ++i) {
+                const nomas_cache* ci = cs[l0 + i];
+                L.l[i].k = static_cast<const uint16_t*>(ks[l0 + i]);
+                L.l[i].v = static_cast<const uint16_t*>(vs[l0 + i]);
+                L.l[i].ck = ci->k;
+                L.l[i].cv = ci->v;
+                L.l[i].cks = ci->k_scale;
+                L.l[i].cvs = ci->v_scale;
+            }
+            a.n_layers = nl;
+            if (launch_commit(a, L, tab, s) != cudaSuccess) return NOMAS_ERR_CUDA;
+        }
     }
-    c->frames_committed += n_frames;
-    if (W > 0) {
-        c->valid_frames = static_cast<int32_t>(c->frames_committed < W ? c->frames_committed : W);
-        c->head_slot = static_cast<int32_t>(c->frames_committed % W);
-    } else {
-        c->valid_frames = static_cast<int32_t>(c->frames_committed);
-        c->head_slot = static_cast<int32_t>(c->frames_committed);
+    for (int i = 0; i < n_layers; ++i) {
+        nomas_cache* ci = cs[i];
+        ci->frames_committed += n_frames;
+        if (W > 0) {
+            ci->valid_frames = static_cast<int32_t>(ci->frames_committed < W ? ci->frames_committed : W);
+            ci->head_slot = static_cast<int32_t>(ci->frames_committed % W);
+        } else {
+            ci->valid_frames = static_cast<int32_t>(ci->frames_committed);
+            ci->head_slot = static_cast<int32_t>(ci->frames_committed);
+        }
     }
     return NOMAS_OK;
+}
+
+int nomas_kv_commit(nomas_cache* c, const void* k, const void* v, int64_t token_stride, int32_t n_frames,
+                    void* stream) {
+    return commit_layers(&c, &k, &v, token_stride, 1, n_frames, stream);
+}
+
+int nomas_kv_commit_layers(nomas_cache* const* caches, const void* const* k, const void* const* v,
+                           int64_t token_stride, int32_t n_layers, int32_t n_frames, void* stream) {
+    return commit_layers(caches, k, v, token_stride, n_layers, n_frames, stream);
 }
 
 size_t nomas_seg_attn_workspace_bytes(const nomas_cache* c, int32_t n_video_frames, int32_t n_text) {

@@ -45,14 +45,23 @@ __device__ __forceinline__ uint32_t fast_div(uint32_t n, const FastDiv& f) {
 }
 #endif
 
-struct CommitArgs {
+// Per-layer pointers of one commit launch (layers share every other argument).
+struct CommitLayer {
     const uint16_t* k;      // segment K, BF16 bits, token-major
     const uint16_t* v;      // segment V
-    int64_t token_stride;   // elements between tokens
     void* ck;               // cache K (int8 codes or BF16 bits), head-major
     void* cv;
     float* cks;             // cache K scales (INT8 mode)
     float* cvs;
+};
+constexpr int kMaxLayersPerLaunch = 24; // keeps RopeTab + CommitArgs + CommitLayers under the 32 KB argument limit
+struct CommitLayers {
+    CommitLayer l[kMaxLayersPerLaunch];
+};
+
+struct CommitArgs {
+    int32_t n_layers;       // layers of this launch (entries of CommitLayers)
+    int64_t token_stride;   // elements between tokens
     int64_t cap_tok;        // capacity_frames * tokens_per_frame
     int32_t heads, tpf, grid_h, grid_w;
     int32_t n_frames;       // frames written by this launch
@@ -64,7 +73,10 @@ struct CommitArgs {
     FastDiv div_heads, div_tpf, div_gw;
     int32_t head_group;     // heads of one token handled by one warp task (set by launch_commit)
     FastDiv div_groups;     // ceil(heads / head_group)
+    FastDiv div_layer_tasks; // warp tasks per layer (set by launch_commit)
 };
+static_assert(sizeof(RopeTab) + sizeof(CommitArgs) + sizeof(CommitLayers) <= 32764,
+              "commit launch arguments exceed the 32,764-byte limit");
 
 struct PrepArgs {
     const uint16_t* q;      // segment Q, BF16 bits, token-major
@@ -127,7 +139,7 @@ struct DequantArgs {
 };
 
 // Kernel launchers (return cudaError_t of the launch).
-cudaError_t launch_commit(const CommitArgs& a, const RopeTab& tab, cudaStream_t s);
+cudaError_t launch_commit(const CommitArgs& a, const CommitLayers& layers, const RopeTab& tab, cudaStream_t s);
 cudaError_t launch_prep(const PrepArgs& a, const RopeTab& tab, cudaStream_t s);
 cudaError_t launch_attn(const AttnArgs& a, bool int8_cache, const CUtensorMap& tm_q, const CUtensorMap& tm_kcur,
                         const CUtensorMap& tm_vcur, const CUtensorMap& tm_kc, const CUtensorMap& tm_vc,

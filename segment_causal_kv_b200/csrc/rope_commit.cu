@@ -178,12 +178,13 @@ __device__ __forceinline__ uint2 quantize8(const float (&y)[8], float& scale_out
 
 template <bool kGrouped, bool kInt8>
 __global__ void __launch_bounds__(kThreads) commit_kernel(const __grid_constant__ CommitArgs a,
+                                                          const __grid_constant__ CommitLayers L,
                                                           const __grid_constant__ RopeTab tab) {
     __shared__ __align__(16) float2 s_t[kMaxFramesPerLaunch * kTPairs];
     __shared__ __align__(16) float2 s_hw[NOMAS_MAX_GRID_HW * kHWPairs];
     stage_tables(tab, a.n_frames, a.grid_h + a.grid_w, s_t, s_hw);
 
-    // A warp task is one token and a group of `head_group` of its heads; the
+    // A warp task is one layer's token and a group of `head_group` of its heads; the
     // two half-warps walk the group's heads h = g0 + half, g0 + half + 2, ...
     // (one (token, head) row per half-warp per step). Position, RoPE
     // coefficients and ring slot depend only on the token, so they are set up
@@ -195,15 +196,18 @@ __global__ void __launch_bounds__(kThreads) commit_kernel(const __grid_constant_
     const int half = lane >> 4;
     const int l = lane & 15;
     const uint32_t groups = kGrouped ? a.div_groups.d : 1u;
-    const uint32_t tasks = static_cast<uint32_t>(a.n_frames) * a.tpf * groups;
+    const uint32_t layer_tasks = static_cast<uint32_t>(a.n_frames) * a.tpf * groups;
+    const uint32_t tasks = layer_tasks * static_cast<uint32_t>(a.n_layers);
     const uint32_t warps = gridDim.x * (kThreads / 32);
     const int steps = ((kGrouped ? a.head_group : a.heads) + 1) >> 1; // rows per half-warp per task
     const int64_t tok0 = static_cast<int64_t>(a.in_frame0) * a.tpf;
     auto row_ptr = [&](const uint16_t* base, uint32_t tok, int h) {
         return reinterpret_cast<const uint4*>(base + (tok0 + tok) * a.token_stride + h * kD + l * 8);
     };
-    // token of a task and the first head of its group
-    auto task_token = [&](uint32_t t, uint32_t& tk) {
+    // layer and token of a task, and the first head of its group
+    auto task_token = [&](uint32_t t, uint32_t& ly, uint32_t& tk) {
+        ly = a.n_layers > 1 ? fast_div(t, a.div_layer_tasks) : 0u;
+        t -= ly * layer_tasks;
         if (!kGrouped) {
             tk = t;
             return 0;
@@ -214,14 +218,15 @@ __global__ void __launch_bounds__(kThreads) commit_kernel(const __grid_constant_
     uint32_t task = blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
     uint4 kx = make_uint4(0, 0, 0, 0), vx = kx;
     if (task < tasks) {
-        uint32_t tk;
-        const int h0 = min(task_token(task, tk) + half, a.heads - 1); // out-of-range heads load a valid row, not stored
-        kx = __ldg(row_ptr(a.k, tk, h0));
-        vx = __ldg(row_ptr(a.v, tk, h0));
+        uint32_t ly, tk;
+        const int h0 = min(task_token(task, ly, tk) + half, a.heads - 1); // out-of-range heads load a valid row, not stored
+        kx = __ldg(row_ptr(L.l[ly].k, tk, h0));
+        vx = __ldg(row_ptr(L.l[ly].v, tk, h0));
     }
     for (; task < tasks; task += warps) {
-        uint32_t tok;
-        const int g0 = task_token(task, tok);
+        uint32_t layer, tok;
+        const int g0 = task_token(task, layer, tok);
+        const CommitLayer& P = L.l[layer];
         const int g1 = kGrouped ? min(g0 + a.head_group, a.heads) : a.heads; // heads [g0, g1) in this task
         const uint32_t fi = fast_div(tok, a.div_tpf);
         const uint32_t rif = tok - fi * a.tpf;
@@ -246,13 +251,13 @@ __global__ void __launch_bounds__(kThreads) commit_kernel(const __grid_constant_
             uint4 kn = kx, vn = vx;
             if (j + 1 < steps) {
                 const int hn = min(h + 2, a.heads - 1);
-                kn = __ldg(row_ptr(a.k, tok, hn));
-                vn = __ldg(row_ptr(a.v, tok, hn));
+                kn = __ldg(row_ptr(P.k, tok, hn));
+                vn = __ldg(row_ptr(P.v, tok, hn));
             } else if (task_next < tasks) {
-                uint32_t tn;
-                const int hn = min(task_token(task_next, tn) + half, a.heads - 1);
-                kn = __ldg(row_ptr(a.k, tn, hn));
-                vn = __ldg(row_ptr(a.v, tn, hn));
+                uint32_t ln, tn;
+                const int hn = min(task_token(task_next, ln, tn) + half, a.heads - 1);
+                kn = __ldg(row_ptr(L.l[ln].k, tn, hn));
+                vn = __ldg(row_ptr(L.l[ln].v, tn, hn));
             }
             float ky[8], vy[8];
             rotate8(kx, cs, ky);
@@ -263,11 +268,11 @@ __global__ void __launch_bounds__(kThreads) commit_kernel(const __grid_constant_
                 const uint2 kc = quantize8(ky, ks);
                 const uint2 vc = quantize8(vy, vs);
                 if (valid) {
-                    *reinterpret_cast<uint2*>(static_cast<int8_t*>(a.ck) + row * kD + l * 8) = kc;
-                    *reinterpret_cast<uint2*>(static_cast<int8_t*>(a.cv) + row * kD + l * 8) = vc;
+                    *reinterpret_cast<uint2*>(static_cast<int8_t*>(P.ck) + row * kD + l * 8) = kc;
+                    *reinterpret_cast<uint2*>(static_cast<int8_t*>(P.cv) + row * kD + l * 8) = vc;
                     if (l == 0) {
-                        a.cks[row] = ks;
-                        a.cvs[row] = vs;
+                        P.cks[row] = ks;
+                        P.cvs[row] = vs;
                     }
                 }
             } else if (valid) {
@@ -276,8 +281,8 @@ __global__ void __launch_bounds__(kThreads) commit_kernel(const __grid_constant_
                 ko.y = rne_bf16x2(ky[2], ky[3]);
                 ko.z = rne_bf16x2(ky[4], ky[5]);
                 ko.w = rne_bf16x2(ky[6], ky[7]);
-                *reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.ck) + row * kD + l * 8) = ko;
-                *reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.cv) + row * kD + l * 8) = vx;
+                *reinterpret_cast<uint4*>(static_cast<uint16_t*>(P.ck) + row * kD + l * 8) = ko;
+                *reinterpret_cast<uint4*>(static_cast<uint16_t*>(P.cv) + row * kD + l * 8) = vx;
             }
             kx = kn;
             vx = vn;
@@ -349,25 +354,26 @@ int grid_for(int64_t work_items, int items_per_block) {
 
 } // namespace
 
-cudaError_t launch_commit(const CommitArgs& a_in, const RopeTab& tab, cudaStream_t s) {
+cudaError_t launch_commit(const CommitArgs& a_in, const CommitLayers& layers, const RopeTab& tab, cudaStream_t s) {
     // heads per warp task: all of a token's heads when there are enough tokens
     // to give every resident warp several tasks, else halves of that, down to 2,
     // so that small commits still spread over the GPU
     CommitArgs a = a_in;
-    const int64_t tokens = static_cast<int64_t>(a.n_frames) * a.tpf;
+    const int64_t tokens = static_cast<int64_t>(a.n_frames) * a.tpf * a.n_layers;
     const int64_t want = 4ll * 148 * 2 * (kThreads / 32);
     int hg = a.heads;
     while (hg > 2 && tokens * ((a.heads + hg - 1) / hg) < want) hg = (hg + 1) / 2;
     a.head_group = hg;
     a.div_groups = make_fastdiv(static_cast<uint32_t>((a.heads + hg - 1) / hg));
-    const int64_t tasks = tokens * a.div_groups.d;
-    const int grid = grid_for(tasks, kThreads / 32);
+    const int64_t layer_tasks = static_cast<int64_t>(a.n_frames) * a.tpf * a.div_groups.d;
+    a.div_layer_tasks = make_fastdiv(static_cast<uint32_t>(layer_tasks));
+    const int grid = grid_for(layer_tasks * a.n_layers, kThreads / 32);
     if (hg < a.heads) {
-        if (a.int8_mode) commit_kernel<true, true><<<grid, kThreads, 0, s>>>(a, tab);
-        else commit_kernel<true, false><<<grid, kThreads, 0, s>>>(a, tab);
+        if (a.int8_mode) commit_kernel<true, true><<<grid, kThreads, 0, s>>>(a, layers, tab);
+        else commit_kernel<true, false><<<grid, kThreads, 0, s>>>(a, layers, tab);
     } else {
-        if (a.int8_mode) commit_kernel<false, true><<<grid, kThreads, 0, s>>>(a, tab);
-        else commit_kernel<false, false><<<grid, kThreads, 0, s>>>(a, tab);
+        if (a.int8_mode) commit_kernel<false, true><<<grid, kThreads, 0, s>>>(a, layers, tab);
+        else commit_kernel<false, false><<<grid, kThreads, 0, s>>>(a, layers, tab);
     }
     return cudaGetLastError();
 }

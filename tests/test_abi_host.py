@@ -160,3 +160,47 @@ def test_workspace_size_is_a_function_of_the_shape():
     assert a == b and a % 256 == 0
     assert nm.nomas_seg_attn_workspace_bytes(d, 6, 256) > a
     assert nm.nomas_seg_attn_workspace_bytes(d, -1, 0) == 0
+
+
+def test_min_workspace_selects_the_fused_form_and_bounds_the_call():
+    d = desc()
+    assert nm.nomas_cache_reset(d) == nm.NOMAS_OK
+    d.valid_frames = 18  # as after 18 committed frames (state is not part of the stamp)
+    full = nm.nomas_seg_attn_workspace_bytes(d, 3, 256)
+    low = nm.nomas_seg_attn_workspace_min_bytes(d, 3, 256)
+    # the full workspace adds the BF16 copy of the window: 2 x 16 heads x 15,840 tokens x 256 B
+    assert full - low >= 2 * 16 * 18 * 880 * 256
+    call = lambda wsb: nm.nomas_seg_attn(d, FAKE, FAKE, FAKE, 2048, 3, 256, FAKE, None, FAKE, wsb, None)
+    assert call(low - 1) == nm.NOMAS_ERR_WORKSPACE
+    # with low or more bytes validation passes; without a GPU the call then stops at the device check
+    assert call(low) in (nm.NOMAS_ERR_DEVICE, nm.NOMAS_ERR_CUDA)
+    bf = desc(mode=nm.NOMAS_CACHE_BF16, window=0, cap=20)
+    assert nm.nomas_cache_reset(bf) == nm.NOMAS_OK
+    bf.valid_frames = 18
+    assert nm.nomas_seg_attn_workspace_bytes(bf, 3, 256) == nm.nomas_seg_attn_workspace_min_bytes(bf, 3, 256)
+
+
+def test_layered_commit_argument_checks():
+    ds = [desc(k=FAKE + (i << 32), v=FAKE + (i << 32) + (1 << 30), ks=FAKE + (i << 32) + (2 << 30),
+               vs=FAKE + (i << 32) + (3 << 30)) for i in range(3)]
+    for d in ds:
+        assert nm.nomas_cache_reset(d) == nm.NOMAS_OK
+    ptrs = [FAKE] * 3
+    c = lambda dd, k=ptrs, v=ptrs, ts=2048, nf=3: nm.nomas_kv_commit_layers(dd, k, v, ts, nf, None)
+    assert c(ds, nf=0) == nm.NOMAS_OK  # no-op
+    assert c(ds, nf=-1) == nm.NOMAS_ERR_ARG
+    assert c([ds[0], ds[1], ds[0]]) == nm.NOMAS_ERR_ARG  # one cache twice
+    assert c(ds, k=[FAKE, None, FAKE]) == nm.NOMAS_ERR_ARG
+    assert c(ds, v=[FAKE, FAKE, FAKE + 8]) == nm.NOMAS_ERR_ALIGN
+    assert c(ds, ts=2052) == nm.NOMAS_ERR_ARG
+    ds[2].grid_w = 41  # changed configuration: the stamp no longer matches
+    assert c(ds) == nm.NOMAS_ERR_STATE
+    ds[2].grid_w = 40
+    ds[1].valid_frames = 2  # same configuration, different ring state
+    assert c(ds) == nm.NOMAS_ERR_STATE
+    ds[1].valid_frames = 0
+    other = desc(window=9, cap=9, k=FAKE + (7 << 32))
+    assert nm.nomas_cache_reset(other) == nm.NOMAS_OK
+    assert c([ds[0], other, ds[2]]) == nm.NOMAS_ERR_STATE
+    assert all(d.frames_committed == 0 for d in ds)
+    assert nm.nomas_kv_commit_layers([], [], [], 2048, 3, None) == nm.NOMAS_ERR_ARG

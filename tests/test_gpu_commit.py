@@ -136,3 +136,22 @@ def test_commit_subnormal_tiny_and_large_rows():
     s = gpu.k_scale.cpu().numpy()[0, 0]
     assert 0.0 < s < 1.17549435e-38
     assert gpu.k[0, 0].abs().max().item() == 127
+
+
+@pytest.mark.parametrize("mode,n_layers", [("int8", 3), ("bf16", 3), ("int8", 26)])
+def test_layered_commit_matches_per_layer_commits(mode, n_layers):
+    """nomas_kv_commit_layers writes into every layer cache exactly what the
+    oracle's commit of that layer's segment writes (26 layers: two launches)."""
+    import segment_causal_kv_b200 as nm
+    H, gh, gw, W = 2, 3, 5, 4
+    geo = synth.Geometry(H, gh, gw)
+    om = oracle.MODE_INT8 if mode == "int8" else oracle.MODE_BF16
+    gpus = [nm.KVCache(mode, H, gh, gw, W, W) for _ in range(n_layers)]
+    orcs = [oracle.OracleCache(om, H, gh, gw, W, W) for _ in range(n_layers)]
+    for s, nf in enumerate([3, 2, 4]):  # wraps the 4-frame ring
+        kv = [synth.history_kv(geo, nf, 200 + layer, s) for layer in range(n_layers)]
+        nm.commit_layers(gpus, [to_dev(k) for k, _ in kv], [to_dev(v) for _, v in kv], nf)
+        for o, (k, v) in zip(orcs, kv):
+            o.commit(k, v, nf)
+        for g, o in zip(gpus, orcs):
+            assert_cache_equal(g, o)
