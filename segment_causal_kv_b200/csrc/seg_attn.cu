@@ -92,6 +92,14 @@ __device__ __forceinline__ uint64_t desc_kmajor(uint32_t tile, int kk) {
 __device__ __forceinline__ uint64_t desc_mnmajor(uint32_t tile, int kk) {
     return smem_desc(tile + kk * 2048, kHalfBytes, 1024, kSwizzle128B);
 }
+// The start address sits in the low 14 bits of a descriptor in 16-byte units;
+// shared addresses stay below 256 KB, so a k-step's descriptor is the tile's
+// k-step-0 descriptor plus the step's byte offset / 16 (no carry out of the
+// field). The issuer builds the k-step-0 descriptors once and adds these.
+__host__ __device__ constexpr uint64_t kstep_kmajor(int kk) {
+    return static_cast<uint64_t>(((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4);
+}
+__host__ __device__ constexpr uint64_t kstep_mnmajor(int kk) { return static_cast<uint64_t>((kk * 2048) >> 4); }
 
 // 8 INT8 codes -> 8 BF16 values code * scale. A code c is read exactly as the
 // float 2^23 + (c + 128) (the byte of c ^ 0x80 placed under the exponent of 2^23),
@@ -478,22 +486,30 @@ __global__ void __launch_bounds__(kInt8 ? 512 : 384, 1)
             constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, BN, false, false);
             constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, kD, false, true);
             const uint32_t q_tile[2] = {sbase + kOffQ, sbase + kOffQ + kTileBytes};
-            const uint32_t tm_s[2] = {tmem, tmem + 128};
-            const uint32_t tm_o[2] = {tmem + 256, tmem + 384};
+            // TMEM columns: S of Q tile w at 128 w, O of Q tile w at 256 + 128 w
+            auto tm_s = [&](int w) { return tmem + 128u * static_cast<uint32_t>(w); };
+            auto tm_o = [&](int w) { return tmem + 256u + 128u * static_cast<uint32_t>(w); };
             const int nq_tiles = has_q1 ? 2 : 1;
             bool ok = MBAR_WAIT(bar(B_QFULL), 0, ctl);
             tc_fence_after();
+            // k-step-0 descriptors of the Q tiles and of the K and V stages (scalars:
+            // selected, not indexed, so they stay in registers)
+            static_assert(kStages == 2, "the stage descriptors below assume two stages");
+            const uint64_t q_desc0 = desc_kmajor(q_tile[0], 0), q_desc1 = desc_kmajor(q_tile[1], 0);
+            const uint64_t k_desc0 = desc_kmajor(sbase + kOffK, 0), k_desc1 = desc_kmajor(sbase + kOffK + kTileBytes, 0);
+            const uint64_t v_desc0 = desc_mnmajor(sbase + kOffV, 0);
+            const uint64_t v_desc1 = desc_mnmajor(sbase + kOffV + kTileBytes, 0);
             auto issue_s = [&](int w, int st) {
-                const uint32_t ktile = sbase + kOffK + st * kTileBytes;
+                const uint64_t qd = w ? q_desc1 : q_desc0, kd = st ? k_desc1 : k_desc0;
 #pragma unroll
                 for (int kk = 0; kk < kD / 16; ++kk)
-                    MMA_SS(tm_s[w], desc_kmajor(q_tile[w], kk), desc_kmajor(ktile, kk), idesc_qk, kk > 0 ? 1u : 0u);
+                    MMA_SS(tm_s(w), qd + kstep_kmajor(kk), kd + kstep_kmajor(kk), idesc_qk, kk > 0 ? 1u : 0u);
             };
             auto issue_pv = [&](int w, int st, bool first_tile) {
-                const uint32_t vtile = sbase + kOffV + st * kTileBytes;
+                const uint64_t vd = st ? v_desc1 : v_desc0;
 #pragma unroll
                 for (int kk = 0; kk < BN / 16; ++kk)
-                    MMA_TS(tm_o[w], tm_s[w] + kk * 8, desc_mnmajor(vtile, kk), idesc_pv,
+                    MMA_TS(tm_o(w), tm_s(w) + kk * 8, vd + kstep_mnmajor(kk), idesc_pv,
                            (first_tile && kk == 0) ? 0u : 1u);
             };
             if (ok) ok = MBAR_WAIT(bar(B_KFULL + 0), 0, ctl);
