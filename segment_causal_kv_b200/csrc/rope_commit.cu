@@ -337,13 +337,15 @@ __global__ void __launch_bounds__(kThreads) prep_kernel(const __grid_constant__ 
 }
 
 int grid_for(int64_t work_items, int items_per_block) {
-    static int sms = 0;
-    if (sms == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        if (sms <= 0) sms = 148;
-    }
+    // SM count of the first device that launches (every device of this library is a B200);
+    // a function-local static is initialised once, thread-safely
+    static const int sms = [] {
+        int dev = 0, n = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+        return n;
+    }();
     // a persistent grid: every block stages the RoPE rows once and then loops
     int64_t want = (work_items + items_per_block - 1) / items_per_block;
     const int64_t cap = static_cast<int64_t>(sms) * 2;

@@ -36,6 +36,8 @@
 #include "nomas_internal.h"
 #include "nomas_ptx.cuh"
 
+#include <atomic>
+
 namespace nomas {
 
 namespace {
@@ -780,27 +782,34 @@ cudaError_t launch_dequant_window(const DequantArgs& a, cudaStream_t s) {
     return cudaGetLastError();
 }
 
+// The dynamic shared-memory limit of a kernel is an attribute of the kernel in
+// one device's context: it is raised once per device (and per kernel), the
+// first time that device launches it. Concurrent first launches may both set
+// it, which is harmless.
+template <bool kInt8>
+cudaError_t ensure_smem_attr() {
+    constexpr int kMaxDev = 64;
+    static std::atomic<bool> done[kMaxDev];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < kMaxDev && done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+    e = cudaFuncSetAttribute(attn_kernel<kInt8>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e == cudaSuccess && dev >= 0 && dev < kMaxDev) done[dev].store(true, std::memory_order_release);
+    return e;
+}
+
 cudaError_t launch_attn(const AttnArgs& a, bool int8_cache, const CUtensorMap& tm_q, const CUtensorMap& tm_kcur,
                         const CUtensorMap& tm_vcur, const CUtensorMap& tm_kc, const CUtensorMap& tm_vc,
                         cudaStream_t s) {
     const int grid = a.heads * a.pairs * a.splits;
     if (int8_cache) {
-        static bool attr_set = false;
-        if (!attr_set) {
-            cudaError_t e = cudaFuncSetAttribute(attn_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 kSmemBytes);
-            if (e != cudaSuccess) return e;
-            attr_set = true;
-        }
+        cudaError_t e = ensure_smem_attr<true>();
+        if (e != cudaSuccess) return e;
         attn_kernel<true><<<grid, 512, kSmemBytes, s>>>(a, tm_q, tm_kcur, tm_vcur, tm_kc, tm_vc);
     } else {
-        static bool attr_set = false;
-        if (!attr_set) {
-            cudaError_t e = cudaFuncSetAttribute(attn_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 kSmemBytes);
-            if (e != cudaSuccess) return e;
-            attr_set = true;
-        }
+        cudaError_t e = ensure_smem_attr<false>();
+        if (e != cudaSuccess) return e;
         attn_kernel<false><<<grid, 384, kSmemBytes, s>>>(a, tm_q, tm_kcur, tm_vcur, tm_kc, tm_vc);
     }
     return cudaGetLastError();
