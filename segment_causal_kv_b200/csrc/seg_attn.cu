@@ -81,6 +81,27 @@ __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, co
     return __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
 }
 
+// How the MMA issuer issues: kWarp = the whole warp runs the loop and one
+// elected lane issues each instruction; otherwise lane 0 alone runs it.
+template <bool kWarp>
+struct Issuer {
+    static __device__ __forceinline__ void ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+        if (kWarp) mma_ss_warp(d, a, b, idesc, acc);
+        else mma_ss(d, a, b, idesc, acc);
+    }
+    static __device__ __forceinline__ void ts(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+        if (kWarp) mma_ts_warp(d, a, b, idesc, acc);
+        else mma_ts(d, a, b, idesc, acc);
+    }
+    static __device__ __forceinline__ void commit(uint32_t bar) {
+        if (kWarp) mma_commit_warp(bar);
+        else mma_commit(bar);
+    }
+    static __device__ __forceinline__ bool wait(uint32_t bar, uint32_t parity, const WaitCtl& ctl) {
+        return kWarp ? mbar_wait_warp(bar, parity, ctl) : mbar_wait(bar, parity, ctl);
+    }
+};
+
 __device__ __forceinline__ int tile_valid(const AttnArgs& a, int t) {
     const int rem = (t < a.tiles_c) ? a.nc - t * BN : a.nq - (t - a.tiles_c) * BN;
     return rem < BN ? rem : BN;
@@ -481,10 +502,7 @@ __global__ void __launch_bounds__(kInt8 ? 512 : 384, 1)
         // polling only takes issue slots from them, so lane 0 issues alone.
         constexpr bool kWarpIssue = !kInt8;
         if (kWarpIssue || lane == 0) {
-#define MMA_SS(...) (kWarpIssue ? mma_ss_warp(__VA_ARGS__) : mma_ss(__VA_ARGS__))
-#define MMA_TS(...) (kWarpIssue ? mma_ts_warp(__VA_ARGS__) : mma_ts(__VA_ARGS__))
-#define MMA_COMMIT(b) (kWarpIssue ? mma_commit_warp(b) : mma_commit(b))
-#define MBAR_WAIT(b, p, c) (kWarpIssue ? mbar_wait_warp(b, p, c) : mbar_wait(b, p, c))
+            using I = Issuer<kWarpIssue>;
             constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, BN, false, false);
             constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, kD, false, true);
             const uint32_t q_tile[2] = {sbase + kOffQ, sbase + kOffQ + kTileBytes};
@@ -492,7 +510,7 @@ __global__ void __launch_bounds__(kInt8 ? 512 : 384, 1)
             auto tm_s = [&](int w) { return tmem + 128u * static_cast<uint32_t>(w); };
             auto tm_o = [&](int w) { return tmem + 256u + 128u * static_cast<uint32_t>(w); };
             const int nq_tiles = has_q1 ? 2 : 1;
-            bool ok = MBAR_WAIT(bar(B_QFULL), 0, ctl);
+            bool ok = I::wait(bar(B_QFULL), 0, ctl);
             tc_fence_after();
             // k-step-0 descriptors of the Q tiles and of the K and V stages (scalars:
             // selected, not indexed, so they stay in registers)
@@ -505,24 +523,24 @@ __global__ void __launch_bounds__(kInt8 ? 512 : 384, 1)
                 const uint64_t qd = w ? q_desc1 : q_desc0, kd = st ? k_desc1 : k_desc0;
 #pragma unroll
                 for (int kk = 0; kk < kD / 16; ++kk)
-                    MMA_SS(tm_s(w), qd + kstep_kmajor(kk), kd + kstep_kmajor(kk), idesc_qk, kk > 0 ? 1u : 0u);
+                    I::ss(tm_s(w), qd + kstep_kmajor(kk), kd + kstep_kmajor(kk), idesc_qk, kk > 0 ? 1u : 0u);
             };
             auto issue_pv = [&](int w, int st, bool first_tile) {
                 const uint64_t vd = st ? v_desc1 : v_desc0;
 #pragma unroll
                 for (int kk = 0; kk < BN / 16; ++kk)
-                    MMA_TS(tm_o(w), tm_s(w) + kk * 8, vd + kstep_mnmajor(kk), idesc_pv,
+                    I::ts(tm_o(w), tm_s(w) + kk * 8, vd + kstep_mnmajor(kk), idesc_pv,
                            (first_tile && kk == 0) ? 0u : 1u);
             };
-            if (ok) ok = MBAR_WAIT(bar(B_KFULL + 0), 0, ctl);
+            if (ok) ok = I::wait(bar(B_KFULL + 0), 0, ctl);
             if (ok) {
                 tc_fence_after();
                 for (int w = 0; w < nq_tiles; ++w) {
                     issue_s(w, 0);
-                    MMA_COMMIT(bar(B_SFULL + w));
+                    I::commit(bar(B_SFULL + w));
                 }
                 // K of tile 0 is free once these S MMAs finish (a fill of tile 2 waits for it)
-                if (kStages < n) MMA_COMMIT(bar(B_KEMPTY + 0));
+                if (kStages < n) I::commit(bar(B_KEMPTY + 0));
             }
             for (int i = 0; ok && i < n; ++i) {
                 const int st = i % kStages;
@@ -530,39 +548,35 @@ __global__ void __launch_bounds__(kInt8 ? 512 : 384, 1)
                 const int st1 = (i + 1) % kStages;
                 const uint32_t ph1 = ((i + 1) / kStages) & 1;
                 const bool last = (i + 1 == n);
-                if (!(ok = MBAR_WAIT(bar(B_VFULL + st), ph, ctl))) break;
+                if (!(ok = I::wait(bar(B_VFULL + st), ph, ctl))) break;
                 for (int w = 0; w < nq_tiles; ++w) {
-                    if (!(ok = MBAR_WAIT(bar(B_PFULL + w), i & 1, ctl))) break;
+                    if (!(ok = I::wait(bar(B_PFULL + w), i & 1, ctl))) break;
                     tc_fence_after();
                     issue_pv(w, st, i == 0);
                     // each release is committed only when a later fill waits for it,
                     // so no arrival is left pending at exit
-                    if (w == nq_tiles - 1 && i + kStages < n) MMA_COMMIT(bar(B_VEMPTY + st));
+                    if (w == nq_tiles - 1 && i + kStages < n) I::commit(bar(B_VEMPTY + st));
                     if (!last) {
                         // K of tile i + 1 is needed from here on only: P.V of Q tile 0
                         // never waits for it
                         if (w == 0) {
-                            if (!(ok = MBAR_WAIT(bar(B_KFULL + st1), ph1, ctl))) break;
+                            if (!(ok = I::wait(bar(B_KFULL + st1), ph1, ctl))) break;
                             tc_fence_after();
                         }
                         issue_s(w, st1);
-                        MMA_COMMIT(bar(B_SFULL + w));
-                        if (w == nq_tiles - 1 && i + 1 + kStages < n) MMA_COMMIT(bar(B_KEMPTY + st1));
+                        I::commit(bar(B_SFULL + w));
+                        if (w == nq_tiles - 1 && i + 1 + kStages < n) I::commit(bar(B_KEMPTY + st1));
                     } else {
-                        MMA_COMMIT(bar(B_OFULL + w));
+                        I::commit(bar(B_OFULL + w));
                     }
                 }
             }
             // drain: every MMA issued above has completed before teardown
-            MMA_COMMIT(bar(B_DRAIN));
+            I::commit(bar(B_DRAIN));
             const uint64_t t0 = global_timer_ns();
             while (!mbar_try_wait(bar(B_DRAIN), 0)) {
                 if (global_timer_ns() - t0 > NOMAS_WAIT_NS) break;
             }
-#undef MMA_SS
-#undef MMA_TS
-#undef MMA_COMMIT
-#undef MBAR_WAIT
         }
     } else if (warp >= 4 && warp < 12) {
         // ================================================================ softmax
