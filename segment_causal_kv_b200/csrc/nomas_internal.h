@@ -4,6 +4,7 @@
 
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <utility>
 #include <cstdint>
 
 #include "nomas.h" // found through -I include
@@ -137,6 +138,25 @@ struct DequantArgs {
     int32_t heads;
     FastDiv div_nc;
 };
+
+// Launch `kernel` with programmatic stream serialisation: it may begin while
+// the previous kernel on `s` finishes and must call grid_dep_wait before it
+// reads anything that kernel (or an earlier one) wrote.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                             Args&&... args) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // Kernel launchers (return cudaError_t of the launch).
 cudaError_t launch_commit(const CommitArgs& a, const CommitLayers& layers, const RopeTab& tab, cudaStream_t s);

@@ -21,6 +21,7 @@
 // use the _rn intrinsics (no contraction freedom), the scale is an IEEE
 // division absmax / 127, codes are round-half-even of an IEEE division.
 #include "nomas_internal.h"
+#include "nomas_ptx.cuh"
 
 #include <cuda_bf16.h>
 
@@ -292,6 +293,9 @@ __global__ void __launch_bounds__(kThreads) commit_kernel(const __grid_constant_
 
 __global__ void __launch_bounds__(kThreads) prep_kernel(const __grid_constant__ PrepArgs a,
                                                         const __grid_constant__ RopeTab tab) {
+    // the next kernel of the call (the window dequantisation, or the attention
+    // kernel, which waits for this one) may start launching right away
+    grid_dep_launch();
     __shared__ __align__(16) float2 s_t[kMaxFramesPerLaunch * kTPairs];
     __shared__ __align__(16) float2 s_hw[NOMAS_MAX_GRID_HW * kHWPairs];
     const int vid_lo = a.tok0 < a.nv ? a.tok0 : a.nv;

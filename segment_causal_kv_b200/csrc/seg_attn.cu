@@ -455,6 +455,9 @@ __global__ void __launch_bounds__(kInt8 ? 512 : 384, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // launched dependent on the previous kernel of the call: barriers and TMEM
+    // are set up while it finishes; nothing it wrote is read before this point
+    grid_dep_wait();
 
     if (warp == 0) {
         // ================================================================ producer
@@ -731,6 +734,7 @@ __global__ void __launch_bounds__(kInt8 ? 512 : 384, 1)
 }
 
 __global__ void __launch_bounds__(256) combine_kernel(const __grid_constant__ CombineArgs a) {
+    grid_dep_wait(); // launched dependent on the attention kernel
     // one warp per (head, query row); each lane owns 4 of the 128 dims
     const int64_t gw = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
@@ -766,6 +770,11 @@ __global__ void __launch_bounds__(256) combine_kernel(const __grid_constant__ Co
 // consecutive threads on consecutive items, so loads (128 B per row) and
 // stores (256 B per row) are fully coalesced. Grid-stride over both tensors.
 __global__ void __launch_bounds__(512) dequant_window_kernel(const __grid_constant__ DequantArgs a) {
+    // Launched dependent on the RoPE prep kernel and overlapping it: it reads
+    // only the cache, which was complete before prep started. It lets the
+    // attention kernel launch early, and before it exits it waits for prep, so
+    // the attention kernel's wait on it covers prep too.
+    grid_dep_launch();
     const uint32_t rows = static_cast<uint32_t>(a.heads) * static_cast<uint32_t>(a.nc); // per tensor, < 2^31
     const uint32_t items = 2u * rows * 8u;                                              // < 2^32 by the host check
     for (uint32_t it = blockIdx.x * blockDim.x + threadIdx.x; it < items; it += gridDim.x * blockDim.x) {
@@ -782,6 +791,7 @@ __global__ void __launch_bounds__(512) dequant_window_kernel(const __grid_consta
         dst[0] = dequant8(make_uint2(w.x, w.y), sc);
         dst[1] = dequant8(make_uint2(w.z, w.w), sc);
     }
+    grid_dep_wait();
 }
 
 } // namespace
@@ -792,8 +802,7 @@ cudaError_t launch_dequant_window(const DequantArgs& a, cudaStream_t s) {
     uint64_t blocks = (items + 511) / 512;
     const uint64_t cap = 148ull * 4ull; // persistent: 4 blocks of 512 threads per SM
     if (blocks > cap) blocks = cap;
-    dequant_window_kernel<<<static_cast<unsigned>(blocks), 512, 0, s>>>(a);
-    return cudaGetLastError();
+    return launch_dependent(dequant_window_kernel, dim3(static_cast<unsigned>(blocks)), dim3(512), 0, s, a);
 }
 
 // The dynamic shared-memory limit of a kernel is an attribute of the kernel in
@@ -820,11 +829,13 @@ cudaError_t launch_attn(const AttnArgs& a, bool int8_cache, const CUtensorMap& t
     if (int8_cache) {
         cudaError_t e = ensure_smem_attr<true>();
         if (e != cudaSuccess) return e;
-        attn_kernel<true><<<grid, 512, kSmemBytes, s>>>(a, tm_q, tm_kcur, tm_vcur, tm_kc, tm_vc);
+        return launch_dependent(attn_kernel<true>, dim3(grid), dim3(512), kSmemBytes, s, a, tm_q, tm_kcur, tm_vcur,
+                                tm_kc, tm_vc);
     } else {
         cudaError_t e = ensure_smem_attr<false>();
         if (e != cudaSuccess) return e;
-        attn_kernel<false><<<grid, 384, kSmemBytes, s>>>(a, tm_q, tm_kcur, tm_vcur, tm_kc, tm_vc);
+        return launch_dependent(attn_kernel<false>, dim3(grid), dim3(384), kSmemBytes, s, a, tm_q, tm_kcur, tm_vcur,
+                                tm_kc, tm_vc);
     }
     return cudaGetLastError();
 }
@@ -832,8 +843,7 @@ cudaError_t launch_attn(const AttnArgs& a, bool int8_cache, const CUtensorMap& t
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s) {
     const int64_t warps = static_cast<int64_t>(a.heads) * a.nq;
     const int64_t blocks = (warps * 32 + 255) / 256;
-    combine_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(a);
-    return cudaGetLastError();
+    return launch_dependent(combine_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, a);
 }
 
 } // namespace nomas
