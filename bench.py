@@ -19,8 +19,17 @@ is outside the per-step CUDA-event windows.
 
 --impl reference times the CPU oracle (oracle/) as it stands, on a bounded
 sample of the same workload (rank 0 only), as the reference arm.
-With torchrun (N > 1) every rank runs an independent layer cache on its GPU
-(weak scaling, no data-path collective); the time is the max over ranks.
+With torchrun (N > 1) the ranks split the work one of three ways (--shard):
+  replica  every rank runs an independent layer cache on its GPU (default;
+           weak scaling, no data-path collective);
+  heads    one layer-step split by head: each rank owns the cache of its
+           heads and receives the Q/K/V of its heads (strong scaling, no
+           collective);
+  ulysses  one layer-step with token-sharded inputs: all-to-alls turn them
+           into head shards before the commit and the attention and turn the
+           output back (strong scaling; the exchanges are inside the timed
+           step).
+Times are the max over ranks.
 """
 
 from __future__ import annotations
@@ -55,6 +64,8 @@ def parse():
     p.add_argument("--impl", default="nomas", choices=["nomas", "reference"])
     p.add_argument("--e2e-steps", type=int, default=0, help="end-to-end steps (default: min(steps, 100))")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--shard", default="replica", choices=["replica", "heads", "ulysses"],
+                   help="how N > 1 ranks split the work (see the module docstring)")
     p.add_argument("--workload", default=WORKLOAD,
                    help=f"{WORKLOAD} (default: the headline line), commit_72f_int8, history_sweep, layers54_turn")
     return p.parse_args()
@@ -400,6 +411,7 @@ def main():
 
     import torch
     import segment_causal_kv_b200 as nm
+    from segment_causal_kv_b200 import shard as shd
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
@@ -414,22 +426,60 @@ def main():
     geo = synth.Geometry(w["heads"], w["grid_h"], w["grid_w"])
     to_dev = lambda b: torch.from_numpy(np.ascontiguousarray(b).view(np.int16)).view(torch.bfloat16).to(dev)
 
-    cache = nm.KVCache("int8", w["heads"], w["grid_h"], w["grid_w"], w["window"], w["capacity"], device=dev)
+    # Work split: a replica rank owns a whole layer cache with its own inputs;
+    # heads/ulysses ranks own the cache of their heads of one shared layer-step.
+    H = w["heads"]
+    shard_mode = args.shard
+    h0, nh = (0, H) if shard_mode == "replica" else shd.head_range(H, world, rank)
+    seed = w["seed"] + rank if shard_mode == "replica" else w["seed"]
+    jobs = world if shard_mode == "replica" else 1  # layer-steps the whole job does per step
+    counts_f = shd.split_counts(w["cur_frames"] * F, world)
+    counts_q = shd.split_counts(nq, world)
+    cache = nm.KVCache("int8", nh, w["grid_h"], w["grid_w"], w["window"], w["capacity"], device=dev)
     for s, nf in enumerate(w["hist_commits"]):
-        k, v = synth.history_kv(geo, nf, w["seed"] + rank, s)
-        cache.commit(to_dev(k), to_dev(v), nf)
+        k, v = synth.history_kv(geo, nf, seed, s)
+        cache.commit(to_dev(k[:, h0:h0 + nh]), to_dev(v[:, h0:h0 + nh]), nf)
     n_seg = len(w["hist_commits"])
-    kf_h, vf_h = synth.history_kv(geo, w["cur_frames"], w["seed"] + rank, n_seg)
-    q_h, k_h, v_h = synth.segment_qkv(geo, w["cur_frames"], w["n_text"], w["seed"] + rank, segment=n_seg + 1)
+    kf_h, vf_h = synth.history_kv(geo, w["cur_frames"], seed, n_seg)
+    q_h, k_h, v_h = synth.segment_qkv(geo, w["cur_frames"], w["n_text"], seed, segment=n_seg + 1)
+    # what arrives at this rank each step
+    if shard_mode == "heads":
+        kf_h, vf_h, q_h, k_h, v_h = (x[:, h0:h0 + nh] for x in (kf_h, vf_h, q_h, k_h, v_h))
+    elif shard_mode == "ulysses":
+        f0, nf_r = shd.split_range(w["cur_frames"] * F, world, rank)
+        t0, nq_r = shd.split_range(nq, world, rank)
+        kf_h, vf_h = kf_h[f0:f0 + nf_r], vf_h[f0:f0 + nf_r]
+        q_h, k_h, v_h = q_h[t0:t0 + nq_r], k_h[t0:t0 + nq_r], v_h[t0:t0 + nq_r]
     kf, vf, q, k, v = (to_dev(x) for x in (kf_h, vf_h, q_h, k_h, v_h))
-    out = torch.empty((nq, w["heads"], HEAD_DIM), dtype=torch.bfloat16, device=dev)
+    out_rows, out_heads = (counts_q[rank], H) if shard_mode == "ulysses" else (nq, nh)
+    out = torch.empty((out_rows, out_heads, HEAD_DIM), dtype=torch.bfloat16, device=dev)
+    out_h = torch.empty((nq, nh, HEAD_DIM), dtype=torch.bfloat16, device=dev) if shard_mode == "ulysses" else None
     ws = cache.workspace(w["cur_frames"], w["n_text"])
     flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
+    def run_step(d, out_buf, ev=None):
+        """One layer-step on this rank from device inputs d = (kf, vf, q, k, v) into out_buf;
+        ev, if given, gets three events: start, commit done, attention done."""
+        kf_d, vf_d, q_d, k_d, v_d = d
+        if ev is not None:
+            ev[0].record(stream)
+        if shard_mode == "ulysses":
+            kf_d, vf_d = (shd.seq_to_heads(x, H, counts_f) for x in (kf_d, vf_d))
+        cache.commit(kf_d, vf_d, w["cur_frames"], stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        if shard_mode == "ulysses":
+            q_d, k_d, v_d = (shd.seq_to_heads(x, H, counts_q) for x in (q_d, k_d, v_d))
+            cache.seg_attn(q_d, k_d, v_d, w["cur_frames"], w["n_text"], out=out_h, workspace=ws, stream=stream)
+            out_buf.copy_(shd.heads_to_seq(out_h, H, counts_q))
+        else:
+            cache.seg_attn(q_d, k_d, v_d, w["cur_frames"], w["n_text"], out=out_buf, workspace=ws, stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+
     def step():
-        cache.commit(kf, vf, w["cur_frames"], stream=stream)
-        cache.seg_attn(q, k, v, w["cur_frames"], w["n_text"], out=out, workspace=ws, stream=stream)
+        run_step((kf, vf, q, k, v), out)
 
     sampler = ClockSampler(local)
     sampler.start()
@@ -447,11 +497,7 @@ def main():
         dist.barrier()
     for i in range(K):
         flush.zero_()
-        ev[i][0].record(stream)
-        cache.commit(kf, vf, w["cur_frames"], stream=stream)
-        ev[i][1].record(stream)
-        cache.seg_attn(q, k, v, w["cur_frames"], w["n_text"], out=out, workspace=ws, stream=stream)
-        ev[i][2].record(stream)
+        run_step((kf, vf, q, k, v), out, ev[i])
     torch.cuda.synchronize(dev)
     if dist:
         dist.barrier()
@@ -459,12 +505,7 @@ def main():
     commit_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K)]
     attn_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]
     step_ms_total = sum(commit_ms) + sum(attn_ms)
-    if dist:
-        t = torch.tensor([step_ms_total, sum(attn_ms)], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        step_ms_total, attn_total = float(t[0]), float(t[1])
-    else:
-        attn_total = sum(attn_ms)
+    step_ms_total, attn_total = shd.max_over_ranks([step_ms_total, sum(attn_ms)], device=dev)
     if cache.device_status(stream) != nm.NOMAS_OK:
         raise RuntimeError("a kernel reported a timed-out wait")
 
@@ -484,10 +525,10 @@ def main():
     host_in = [torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16).pin_memory()
                for x in (kf_h, vf_h, q_h, k_h, v_h)]
     h2d = sum(x.numel() * x.element_size() for x in host_in)
-    d2h = nq * w["heads"] * HEAD_DIM * 2
+    d2h = out.numel() * out.element_size()
     sets = [[torch.empty_like(x, device=dev) for x in host_in] for _ in range(2)]
     outs = [torch.empty_like(out) for _ in range(2)]
-    host_outs = [torch.empty((nq, w["heads"], HEAD_DIM), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    host_outs = [torch.empty(out.shape, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
     up = torch.cuda.Stream(dev)
     down = torch.cuda.Stream(dev)
     ev_in = [torch.cuda.Event() for _ in range(2)]    # set s is on the device
@@ -509,9 +550,7 @@ def main():
         if not fresh["out"][s]:
             stream.wait_event(ev_out[s])
         fresh["out"][s] = False
-        d = sets[s]
-        cache.commit(d[0], d[1], w["cur_frames"], stream=stream)
-        cache.seg_attn(d[2], d[3], d[4], w["cur_frames"], w["n_text"], out=outs[s], workspace=ws, stream=stream)
+        run_step(sets[s], outs[s])
         ev_used[s].record(stream)
         with torch.cuda.stream(down):
             down.wait_event(ev_used[s])
@@ -547,20 +586,15 @@ def main():
         flush.zero_()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        d = sets[0]
-        for hsrc, ddst in zip(host_in, d):
+        for hsrc, ddst in zip(host_in, sets[0]):
             ddst.copy_(hsrc, non_blocking=True)
-        cache.commit(d[0], d[1], w["cur_frames"], stream=stream)
-        cache.seg_attn(d[2], d[3], d[4], w["cur_frames"], w["n_text"], out=outs[0], workspace=ws, stream=stream)
+        run_step(sets[0], outs[0])
         host_outs[0].copy_(outs[0], non_blocking=True)
         b.record(stream)
         b.synchronize()
         serial_ms.append(a.elapsed_time(b))
     serial_avg = statistics.mean(serial_ms)
-    if dist:
-        t = torch.tensor([e2e_total, serial_avg], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_total, serial_avg = float(t[0]), float(t[1])
+    e2e_total, serial_avg = shd.max_over_ranks([e2e_total, serial_avg], device=dev)
     clocks = sampler.stop()
 
     if dist:
@@ -571,9 +605,10 @@ def main():
 
     peaks, peak_src = load_peaks()
     ms_step = step_ms_total / K
-    value = world * flop_step * K / (step_ms_total * 1e-3) / 1e12
+    value = jobs * flop_step * K / (step_ms_total * 1e-3) / 1e12
     attn_avg_ms = attn_total / K
-    achieved = flop_step / (attn_avg_ms * 1e-3) / 1e12
+    flop_rank = flop_step * nh / H  # attention FLOPs of this rank's heads
+    achieved = flop_rank / (attn_avg_ms * 1e-3) / 1e12
     peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     peak_burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     cm = statistics.mean(commit_ms)
@@ -586,7 +621,7 @@ def main():
         "warmup": args.warmup,
         "ms_per_step": ms_step,
         "higher_is_better": True,
-        "scaling": "weak",
+        "scaling": "weak" if shard_mode == "replica" else "strong",
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
@@ -594,21 +629,24 @@ def main():
                    "history_frames": w["window"], "cache": "int8", "n_video_frames": w["cur_frames"],
                    "n_text": w["n_text"], "nq": nq, "nk": nk, "flop_per_step": flop_step,
                    "step": "kv_commit(3 frames) + seg_attn", "l2": "flushed: 512 MB written before each step",
-                   "parallelism": f"replica x{world}"},
+                   "parallelism": {"replica": f"replica x{world}",
+                                   "heads": f"heads x{world} ({nh} heads on rank 0, no collective)",
+                                   "ulysses": f"ulysses x{world} (token-sharded inputs; all-to-all to heads "
+                                              f"and back inside the step)"}[shard_mode]},
         "attn_ms": attn_avg_ms,
         "commit_ms": cm,
-        "commit_gbs": commit_bytes(w) / (cm * 1e-3) / 1e9,
+        "commit_gbs": commit_bytes(w) * nh / H / (cm * 1e-3) / 1e9,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": traffic_from_profile("attn_kernel<bf16>"),
                      "peak_kind": f"bf16 dense, sustained, {peak_src}",
                      "frac_of_burst": achieved / peak_burst, "frac_of_nominal_2250": achieved / 2250.0,
                      "kernel": "nomas_seg_attn call (INT8 window dequantised once + RoPE prep + BF16-cache "
                                "attn_kernel + split combine), CUDA events; the ncu launch list gives the split"},
-        "e2e": {"value": world * flop_step * Ke / (e2e_total * 1e-3) / 1e12, "unit": "TFLOP/s",
+        "e2e": {"value": jobs * flop_step * Ke / (e2e_total * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": Ke,
                 "ms_per_step": e2e_total / Ke,
                 "form": "pipelined: step i+1 upload and step i-1 readback overlap step i; L2 not flushed"},
-        "e2e_serial": {"value": world * flop_step / (serial_avg * 1e-3) / 1e12, "unit": "TFLOP/s",
+        "e2e_serial": {"value": jobs * flop_step / (serial_avg * 1e-3) / 1e12, "unit": "TFLOP/s",
                        "ms_per_step": serial_avg, "form": "one step at a time, L2 flushed before each"},
         # per step: commit, RoPE prep, attention, the INT8 window dequantisation and the
         # split combine when used
