@@ -164,6 +164,48 @@ int nomas_kv_commit_layers(nomas_cache *const *caches, const void *const *k, con
                            int64_t token_stride, int32_t n_layers, int32_t n_frames, void *stream);
 
 /*
+ * Archive of frames leaving a window (model card, "Segment-Autoregressive
+ * Diffusion Transformer" and "Single-GPU Low-Memory Inference": the single-GPU
+ * configuration attends over a bounded set of history frames on the GPU and
+ * keeps earlier history in an archive in system memory).
+ *
+ * nomas_kv_evicted_frames -- the frames that the next nomas_kv_commit(c, ...,
+ * n_frames) drops from the window: *count frames, absolute indices
+ * *first_frame, *first_frame + 1, ... (the oldest frames of the window, in
+ * order). Host only: no GPU work, no device needed. With no window
+ * (window_frames == 0) nothing is ever dropped (*count = 0). Frames of the
+ * segment being committed that fall out of the window by its end (a segment
+ * longer than the window) never enter the cache and are not counted.
+ * Errors: NOMAS_ERR_ARG (n_frames < 0, NULL outputs), NOMAS_ERR_STATE, and
+ * the descriptor checks of nomas_cache_reset.
+ */
+int nomas_kv_evicted_frames(const nomas_cache *c, int32_t n_frames, int32_t *count, int64_t *first_frame);
+
+/*
+ * nomas_kv_archive_evicted -- enqueue on `stream` device-to-host copies of the
+ * frames nomas_kv_evicted_frames reports, out of the cache, as they are now.
+ * Call it before that commit, on the commit's stream (or order the two
+ * streams with an event), so that the copies read the frames before the
+ * commit overwrites their slots. The caller owns the host buffers (pinned
+ * memory makes the copies asynchronous; pageable memory works but the call
+ * then waits for them). Archived frame i (0 <= i < *count) is stored
+ * frame-major, in the cache's own encoding:
+ *   host_k, host_v             : [count][heads][tokens_per_frame][128]
+ *                                int8 codes (INT8 mode) or BF16 bits;
+ *   host_k_scale, host_v_scale : [count][heads][tokens_per_frame] fp32
+ *                                (INT8 mode; ignored and may be NULL in BF16 mode).
+ * max_frames : frames the host buffers hold. *count and *first_frame are set
+ * whenever the descriptor validates, also when the call then fails with
+ * NOMAS_ERR_CAPACITY (*count > max_frames), so a caller can size its buffers.
+ * *count == 0 enqueues nothing and needs no buffers.
+ * Errors: NOMAS_ERR_ARG, NOMAS_ERR_STATE, NOMAS_ERR_CAPACITY,
+ * NOMAS_ERR_DEVICE, NOMAS_ERR_CUDA; all checks happen before any copy.
+ */
+int nomas_kv_archive_evicted(const nomas_cache *c, int32_t n_frames, void *host_k, void *host_v,
+                             float *host_k_scale, float *host_v_scale, int32_t max_frames, int32_t *count,
+                             int64_t *first_frame, void *stream);
+
+/*
  * nomas_seg_attn_workspace_bytes -- device workspace for the fastest form of
  * nomas_seg_attn for this cache state and segment shape (0 on invalid
  * arguments). For an INT8 cache it includes a BF16 copy of the visible window

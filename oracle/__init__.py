@@ -7,7 +7,7 @@ and the CPU-baseline leg of ``bench.py``; never by the library in
 fp32 commit expression is evaluated exactly as written.
 
 What each C function follows is cited in the C file's header; the readings
-taken where the pages are silent are listed there and in the design doc.
+taken where the pages are silent are listed there.
 """
 
 from __future__ import annotations
@@ -173,6 +173,28 @@ class OracleCache:
         if rc != 0:
             raise MemoryError(f"oracle attention failed ({rc})")
         return out, lse
+
+    def window_frames(self) -> list[int]:
+        """Absolute indices of the frames the cache holds now, read from the slots' frame labels.
+
+        A frame leaves the window exactly when a commit overwrites its slot, so the
+        frames a commit evicts are window_frames() before it minus window_frames() after it."""
+        return sorted(int(f) for f in self.slot_frame if f >= 0)
+
+    def frame_rows(self, f: int):
+        """Stored rows of absolute frame f: (k, v, k_scale, v_scale) as [H][F][128] codes or
+        BF16 bits and [H][F] fp32 scales (None in BF16 mode), copied."""
+        slots = np.nonzero(self.slot_frame == f)[0]
+        if len(slots) != 1:
+            raise KeyError(f)
+        F = self.tokens_per_frame
+        r = slice(int(slots[0]) * F, (int(slots[0]) + 1) * F)
+        if self.mode == MODE_INT8:
+            return (self.k_code[:, r].copy(), self.v_code[:, r].copy(), self.k_scale[:, r].copy(),
+                    self.v_scale[:, r].copy())
+        if self.mode == MODE_BF16:
+            return self.k_bf16[:, r].copy(), self.v_bf16[:, r].copy(), None, None
+        return self.k_f64[:, r].copy(), self.v_f64[:, r].copy(), None, None
 
     def dequantized(self):
         """fp64 K and V of every slot row, [H][cap*F][128] (oracle dequantisation rule)."""

@@ -27,7 +27,7 @@
  *    queries and keys (RoFormer formulation).
  *  - blog "Step 3: The Video Latent": 22 x 40 = 880 tokens per latent frame.
  *
- * Readings where the pages are silent (each listed in the design doc):
+ * Readings where the pages are silent:
  *  - RoPE pairs are interleaved (2j, 2j+1) inside each axis block; block t
  *    = dims [0,16), h = [16,72), w = [72,128); pair j of a block of width d
  *    turns by pos * theta^(-2j/d). Text tokens are not rotated.

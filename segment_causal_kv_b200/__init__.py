@@ -36,7 +36,8 @@ HEAD_DIM = 128
 # exported symbols (checked against include/nomas.h by the tests)
 EXPORTS = ("nomas_cache_reset", "nomas_kv_commit", "nomas_kv_commit_layers", "nomas_seg_attn_workspace_bytes",
            "nomas_seg_attn_workspace_min_bytes", "nomas_seg_attn",
-           "nomas_device_status", "nomas_status_string", "nomas_seg_attn_static", "nomas_selftest_bounded_wait")
+           "nomas_device_status", "nomas_status_string", "nomas_seg_attn_static", "nomas_selftest_bounded_wait",
+           "nomas_kv_evicted_frames", "nomas_kv_archive_evicted")
 NOMAS_STATIC_SCRATCH_BYTES = 64 << 20
 
 
@@ -99,6 +100,10 @@ def lib():
         L.nomas_seg_attn_static.restype = ctypes.c_int
         L.nomas_selftest_bounded_wait.argtypes = [P, P]
         L.nomas_selftest_bounded_wait.restype = ctypes.c_int
+        L.nomas_kv_evicted_frames.argtypes = [D, I32, ctypes.POINTER(I32), ctypes.POINTER(I64)]
+        L.nomas_kv_evicted_frames.restype = ctypes.c_int
+        L.nomas_kv_archive_evicted.argtypes = [D, I32, P, P, P, P, I32, ctypes.POINTER(I32), ctypes.POINTER(I64), P]
+        L.nomas_kv_archive_evicted.restype = ctypes.c_int
         L.nomas_status_string.argtypes = [ctypes.c_int]
         L.nomas_status_string.restype = ctypes.c_char_p
         _lib = L
@@ -130,6 +135,23 @@ def nomas_kv_commit_layers(descs, k_ptrs, v_ptrs, token_stride: int, n_frames: i
     karr = (ctypes.c_void_p * n)(*k_ptrs)
     varr = (ctypes.c_void_p * n)(*v_ptrs)
     return lib().nomas_kv_commit_layers(darr, karr, varr, token_stride, n, n_frames, stream)
+
+
+def nomas_kv_evicted_frames(desc: NomasCacheDesc, n_frames: int) -> tuple[int, int, int]:
+    """(status, count, first_frame) of the frames the next commit of n_frames drops from the window."""
+    count, first = ctypes.c_int32(-1), ctypes.c_int64(-1)
+    rc = lib().nomas_kv_evicted_frames(ctypes.byref(desc), n_frames, ctypes.byref(count), ctypes.byref(first))
+    return rc, int(count.value), int(first.value)
+
+
+def nomas_kv_archive_evicted(desc: NomasCacheDesc, n_frames: int, hk: int | None, hv: int | None,
+                             hks: int | None, hvs: int | None, max_frames: int,
+                             stream: int | None) -> tuple[int, int, int]:
+    """(status, count, first_frame); enqueues the device-to-host copies of those frames."""
+    count, first = ctypes.c_int32(-1), ctypes.c_int64(-1)
+    rc = lib().nomas_kv_archive_evicted(ctypes.byref(desc), n_frames, hk, hv, hks, hvs, max_frames,
+                                        ctypes.byref(count), ctypes.byref(first), stream)
+    return rc, int(count.value), int(first.value)
 
 
 def commit_layers(caches, ks, vs, n_frames: int, stream=None) -> None:
@@ -247,12 +269,45 @@ class KVCache:
     def reset(self) -> None:
         _check(nomas_cache_reset(self.desc), "nomas_cache_reset")
 
-    def commit(self, k, v, n_frames: int, stream=None) -> None:
-        """k, v: BF16 [n_frames * F][heads][128] (token stride taken from the tensor)."""
+    def commit(self, k, v, n_frames: int, stream=None, archive: "FrameArchive | None" = None) -> None:
+        """k, v: BF16 [n_frames * F][heads][128] (token stride taken from the tensor).
+
+        With an archive, the frames this commit drops from the window are first
+        copied into it (on the same stream, so before they are overwritten)."""
+        if archive is not None:
+            archive.add(self.archive_evicted(n_frames, stream=stream))
         assert k.dtype == _torch().bfloat16 and v.dtype == k.dtype and k.stride() == v.stride()
         assert k.shape[0] >= n_frames * self.tokens_per_frame and k.stride(2) == 1 and k.stride(1) == HEAD_DIM
         _check(nomas_kv_commit(self.desc, k.data_ptr(), v.data_ptr(), k.stride(0), n_frames,
                                _stream_handle(stream)), "nomas_kv_commit")
+
+    def evicted_frames(self, n_frames: int) -> tuple[int, int]:
+        """(first_frame, count): the frames the next commit of n_frames drops from the window."""
+        rc, count, first = nomas_kv_evicted_frames(self.desc, n_frames)
+        _check(rc, "nomas_kv_evicted_frames")
+        return first, count
+
+    def archive_evicted(self, n_frames: int, stream=None) -> "ArchivedFrames":
+        """Enqueue device-to-host copies of the frames the next commit of n_frames drops.
+
+        Returns pinned host tensors that hold them once `stream` has passed this point."""
+        torch = _torch()
+        first, count = self.evicted_frames(n_frames)
+        F = self.tokens_per_frame
+        code_t = torch.int8 if self.mode == "int8" else torch.bfloat16
+        host = lambda shape, dt: torch.empty(shape, dtype=dt, pin_memory=count > 0)
+        k = host((count, self.heads, F, HEAD_DIM), code_t)
+        v = host((count, self.heads, F, HEAD_DIM), code_t)
+        ks = vs = None
+        if self.mode == "int8":
+            ks = host((count, self.heads, F), torch.float32)
+            vs = host((count, self.heads, F), torch.float32)
+        ptr = lambda t: t.data_ptr() if t is not None and t.numel() else None
+        rc, got, first2 = nomas_kv_archive_evicted(self.desc, n_frames, ptr(k), ptr(v), ptr(ks), ptr(vs), count,
+                                                   _stream_handle(stream))
+        _check(rc, "nomas_kv_archive_evicted")
+        assert (got, first2) == (count, first)
+        return ArchivedFrames(first, k, v, ks, vs)
 
     def workspace_bytes(self, n_video_frames: int, n_text: int) -> int:
         return nomas_seg_attn_workspace_bytes(self.desc, n_video_frames, n_text)
@@ -289,3 +344,48 @@ class KVCache:
         if self._ws is None:
             return NOMAS_OK
         return nomas_device_status(self._ws.data_ptr(), _stream_handle(stream))
+
+
+class ArchivedFrames:
+    """Frames [first, first + count) copied out of a cache's window, frame-major in the
+    cache's encoding: k, v [count][heads][F][128] (int8 codes or BF16), k_scale,
+    v_scale [count][heads][F] fp32 (INT8 mode, else None). Pinned host tensors."""
+
+    def __init__(self, first: int, k, v, k_scale, v_scale):
+        self.first, self.k, self.v, self.k_scale, self.v_scale = first, k, v, k_scale, v_scale
+
+    @property
+    def count(self) -> int:
+        return int(self.k.shape[0])
+
+
+class FrameArchive:
+    """Host archive of every frame dropped from a cache's window (pass it to KVCache.commit).
+
+    It grows without bound, one entry per archived frame; frame(f) returns the
+    stored (k, v, k_scale, v_scale) of absolute frame f. Read it only after the
+    stream of the commits has been synchronised."""
+
+    def __init__(self):
+        self._chunks: list[ArchivedFrames] = []
+        self._index: dict[int, tuple[int, int]] = {}
+
+    def add(self, chunk: ArchivedFrames) -> None:
+        if chunk.count == 0:
+            return
+        self._chunks.append(chunk)
+        for i in range(chunk.count):
+            self._index[chunk.first + i] = (len(self._chunks) - 1, i)
+
+    def frames(self) -> list[int]:
+        return sorted(self._index)
+
+    def frame(self, f: int):
+        c, i = self._index[f]
+        ch = self._chunks[c]
+        pick = lambda t: t[i] if t is not None else None
+        return pick(ch.k), pick(ch.v), pick(ch.k_scale), pick(ch.v_scale)
+
+    def host_bytes(self) -> int:
+        return sum(t.numel() * t.element_size() for ch in self._chunks
+                   for t in (ch.k, ch.v, ch.k_scale, ch.v_scale) if t is not None)

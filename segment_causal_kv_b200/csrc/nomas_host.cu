@@ -329,6 +329,70 @@ int nomas_kv_commit_layers(nomas_cache* const* caches, const void* const* k, con
     return commit_layers(caches, k, v, token_stride, n_layers, n_frames, stream);
 }
 
+// ------------------------------------------------- archive of evicted frames
+// A commit of n frames into a window of W leaves the last min(W, committed)
+// frames of the whole sequence in the window. The frames it drops are those of
+// the current window [committed - valid, committed) that precede the new
+// window's first frame: consecutive, oldest first.
+static void evicted_range(const nomas_cache* c, int32_t n_frames, int32_t* count, int64_t* first) {
+    const int64_t fc = c->frames_committed, W = c->window_frames;
+    *first = fc - c->valid_frames;
+    *count = 0;
+    if (W == 0 || n_frames <= 0) return;
+    const int64_t after = fc + n_frames;
+    const int64_t kept_from = after - (after < W ? after : W);
+    const int64_t end = fc < kept_from ? fc : kept_from;
+    if (end > *first) *count = static_cast<int32_t>(end - *first);
+}
+
+int nomas_kv_evicted_frames(const nomas_cache* c, int32_t n_frames, int32_t* count, int64_t* first_frame) {
+    int rc = validate_state(c);
+    if (rc != NOMAS_OK) return rc;
+    if (n_frames < 0 || !count || !first_frame) return NOMAS_ERR_ARG;
+    evicted_range(c, n_frames, count, first_frame);
+    return NOMAS_OK;
+}
+
+int nomas_kv_archive_evicted(const nomas_cache* c, int32_t n_frames, void* host_k, void* host_v,
+                             float* host_k_scale, float* host_v_scale, int32_t max_frames, int32_t* count,
+                             int64_t* first_frame, void* stream) {
+    int rc = validate_state(c);
+    if (rc != NOMAS_OK) return rc;
+    if (n_frames < 0 || max_frames < 0 || !count || !first_frame) return NOMAS_ERR_ARG;
+    evicted_range(c, n_frames, count, first_frame);
+    const int32_t m = *count;
+    if (m > max_frames) return NOMAS_ERR_CAPACITY;
+    if (m == 0) return NOMAS_OK;
+    const bool int8 = c->mode == NOMAS_CACHE_INT8;
+    if (!host_k || !host_v || (int8 && (!host_k_scale || !host_v_scale))) return NOMAS_ERR_ARG;
+    if ((rc = check_device()) != NOMAS_OK) return rc;
+    // One frame of one head is tokens_per_frame consecutive rows of that head's
+    // slab, so a frame is `heads` equal runs pitched by the slab: one 2D copy per
+    // frame and tensor, gathered by the copy engine into the frame-major archive.
+    const size_t tpf = static_cast<size_t>(c->grid_h) * c->grid_w;
+    const size_t cap_tok = static_cast<size_t>(c->capacity_frames) * tpf;
+    const size_t es = int8 ? 1 : 2;
+    const size_t run = tpf * kD * es, pitch = cap_tok * kD * es;
+    const size_t srun = tpf * sizeof(float), spitch = cap_tok * sizeof(float);
+    const size_t H = static_cast<size_t>(c->heads);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    for (int32_t i = 0; i < m; ++i) {
+        const size_t slot = static_cast<size_t>((*first_frame + i) % c->window_frames);
+        const auto d2h = [&](void* dst, size_t dst_frame_bytes, const void* src, size_t width, size_t src_pitch) {
+            return cudaMemcpy2DAsync(static_cast<char*>(dst) + static_cast<size_t>(i) * dst_frame_bytes, width,
+                                     static_cast<const char*>(src) + slot * width, src_pitch, width, H,
+                                     cudaMemcpyDeviceToHost, s);
+        };
+        if (d2h(host_k, H * run, c->k, run, pitch) != cudaSuccess ||
+            d2h(host_v, H * run, c->v, run, pitch) != cudaSuccess)
+            return NOMAS_ERR_CUDA;
+        if (int8 && (d2h(host_k_scale, H * srun, c->k_scale, srun, spitch) != cudaSuccess ||
+                     d2h(host_v_scale, H * srun, c->v_scale, srun, spitch) != cudaSuccess))
+            return NOMAS_ERR_CUDA;
+    }
+    return NOMAS_OK;
+}
+
 size_t nomas_seg_attn_workspace_bytes(const nomas_cache* c, int32_t n_video_frames, int32_t n_text) {
     if (validate_state(c) != NOMAS_OK || n_video_frames < 0 || n_text < 0) return 0;
     return make_plan(c, n_video_frames, n_text).total;

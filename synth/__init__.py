@@ -153,7 +153,7 @@ def history_kv(geo: Geometry, n_frames: int, seed: int, segment: int, kv_std: fl
 
 
 # ---------------------------------------------------------------------------
-# Workloads (shapes from the pages; see the design doc for the recipe)
+# Workloads (shapes and value distributions from the pages)
 # ---------------------------------------------------------------------------
 
 WORKLOADS = {
