@@ -82,6 +82,8 @@ def lib():
         _lib.orc_rope_rotate_f64.argtypes = [P, P, ctypes.c_double, P]
         _lib.orc_rope_rotate_f32.argtypes = [P, P, ctypes.c_double, P]
         _lib.orc_quantize_row.argtypes = [P, P, P]
+        _lib.orc_camera_attn.argtypes = [P, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P,
+                                         ctypes.c_int, ctypes.c_int, P]
         _lib.orc_f32_to_bf16.argtypes = [ctypes.c_float]
         _lib.orc_f32_to_bf16.restype = ctypes.c_uint16
     return _lib
@@ -205,6 +207,26 @@ class OracleCache:
             return (self.k_code.astype(np.float64) * self.k_scale[..., None].astype(np.float64),
                     self.v_code.astype(np.float64) * self.v_scale[..., None].astype(np.float64))
         return self.k_f64.copy(), self.v_f64.copy()
+
+
+def camera_attn(q, n_frames: int, tpf: int, k_cam, v_cam, chunk_frames: int = 1) -> np.ndarray:
+    """fp64 per-latent-frame camera cross-attention (orc_camera_attn).
+
+    q: BF16 bits [n_frames * tpf][heads][128] (video tokens); k_cam, v_cam: BF16 bits
+    [n_chunks][n_cam][heads][128]. Returns out [n_frames * tpf][heads][128] fp64."""
+    q = np.ascontiguousarray(q, np.uint16)
+    k_cam = np.ascontiguousarray(k_cam, np.uint16)
+    v_cam = np.ascontiguousarray(v_cam, np.uint16)
+    heads = q.shape[1]
+    n_chunks, n_cam = k_cam.shape[0], k_cam.shape[1]
+    assert q.shape == (n_frames * tpf, heads, HEAD_DIM) and v_cam.shape == k_cam.shape
+    assert k_cam.shape[2:] == (heads, HEAD_DIM) and n_chunks == -(-n_frames // chunk_frames)
+    out = np.zeros(q.shape, np.float64)
+    rc = lib().orc_camera_attn(_ptr(q), heads * HEAD_DIM, n_frames, tpf, heads, _ptr(k_cam), _ptr(v_cam), n_cam,
+                               chunk_frames, _ptr(out))
+    if rc != 0:
+        raise ValueError(f"oracle camera attention rejected its arguments ({rc})")
+    return out
 
 
 def full_seq_attn(segments, heads: int, grid_h: int, grid_w: int, window: int, target: int,

@@ -26,6 +26,12 @@
  *    causal between segments, bidirectional inside one; RoPE rotates
  *    queries and keys (RoFormer formulation).
  *  - blog "Step 3: The Video Latent": 22 x 40 = 880 tokens per latent frame.
+ *  - model card, "Text and Camera Conditioning", and the blog's "Camera
+ *    conditioning": video tokens query projected camera features by
+ *    cross-attention; with per-chunk camera attention and a chunk of one
+ *    latent frame, each latent frame's video tokens see only the camera
+ *    tokens of their own chunk (one token per latent frame in the blog's
+ *    reading of the 64-d grouped extrinsics).
  *
  * Readings where the pages are silent:
  *  - RoPE pairs are interleaved (2j, 2j+1) inside each axis block; block t
@@ -46,6 +52,9 @@
  *  - eviction: keep the last `window` committed latent frames (FIFO, frame
  *    granularity); frame f lives in slot f mod window. window 0 = keep all
  *    (full history) and commits beyond capacity are an error.
+ *  - camera cross-attention: no RoPE, softmax scale 1/sqrt(128), only video
+ *    tokens take part; video token i belongs to latent frame i / F and to
+ *    chunk (i / F) / chunk_frames; each chunk has n_cam camera tokens.
  *
  * Mode 2 (ORC_MODE_F64) is oracle-only: the cache keeps fp64 rotated keys
  * and exact values, so incremental attention can be compared with a masked
@@ -545,5 +554,46 @@ int orc_full_seq_attn(int n_seg, const uint16_t *const *qs, const uint16_t *cons
         }
     }
     free(keys); free(vals); free(qr); free(ob); free(lb); free(tmp);
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* Per-latent-frame camera cross-attention                             */
+/* ------------------------------------------------------------------ */
+
+/* out[i][h] = softmax_j(<q_i,h, k_c,j,h> / sqrt(128)) . v_c,j,h over the
+ * n_cam camera tokens j of chunk c = (i / tpf) / chunk_frames, for every
+ * video token i < n_frames * tpf and head h. q: BF16 [n_video][heads][128]
+ * with token stride q_stride; k_cam, v_cam: BF16 [n_chunks][n_cam][heads][128];
+ * out: fp64 [n_video][heads][128]. fp64 two-pass softmax (attend_row). */
+int orc_camera_attn(const uint16_t *q, int64_t q_stride, int n_frames, int tpf, int heads,
+                    const uint16_t *k_cam, const uint16_t *v_cam, int n_cam, int chunk_frames, double *out) {
+    if (n_frames < 0 || tpf <= 0 || heads <= 0 || n_cam <= 0 || chunk_frames <= 0) return -1;
+    double *keys = malloc(sizeof(double) * (size_t)n_cam * ORC_D);
+    double *vals = malloc(sizeof(double) * (size_t)n_cam * ORC_D);
+    double *scores = malloc(sizeof(double) * (size_t)n_cam);
+    double qd[ORC_D];
+    if (!keys || !vals || !scores) {
+        free(keys); free(vals); free(scores);
+        return -2;
+    }
+    const int64_t nv = (int64_t)n_frames * tpf;
+    for (int64_t i = 0; i < nv; ++i) {
+        const int64_t chunk = (i / tpf) / chunk_frames;
+        for (int h = 0; h < heads; ++h) {
+            for (int j = 0; j < n_cam; ++j) {
+                const int64_t base = ((chunk * n_cam + j) * heads + h) * ORC_D;
+                for (int e = 0; e < ORC_D; ++e) {
+                    keys[(int64_t)j * ORC_D + e] = bf16_to_f32(k_cam[base + e]);
+                    vals[(int64_t)j * ORC_D + e] = bf16_to_f32(v_cam[base + e]);
+                }
+            }
+            for (int e = 0; e < ORC_D; ++e) qd[e] = bf16_to_f32(q[i * q_stride + (int64_t)h * ORC_D + e]);
+            key_set ks = {n_cam, keys, vals};
+            double lse;
+            attend_row(qd, &ks, out + (i * heads + h) * ORC_D, &lse, scores);
+        }
+    }
+    free(keys); free(vals); free(scores);
     return 0;
 }

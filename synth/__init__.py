@@ -40,6 +40,7 @@ _M2 = np.uint64(0x94D049BB133111EB)
 # tensor ids: one stream per role
 TID_Q, TID_K, TID_V = 1, 2, 3
 TID_HIST_K, TID_HIST_V = 4, 5
+TID_CAM_K, TID_CAM_V = 6, 7
 
 
 def _mix(z: np.ndarray) -> np.ndarray:
@@ -150,6 +151,13 @@ def history_kv(geo: Geometry, n_frames: int, seed: int, segment: int, kv_std: fl
     shape = (n_frames * geo.tokens_per_frame, geo.heads, geo.head_dim)
     return (bf16_normal(seed, TID_HIST_K, shape, kv_std, segment),
             bf16_normal(seed, TID_HIST_V, shape, kv_std, segment))
+
+
+def camera_kv(geo: Geometry, n_chunks: int, n_cam: int, seed: int, segment: int = 0, std: float = 1.0):
+    """Projected camera K, V BF16 bits [n_chunks][n_cam][heads][128] (n_cam tokens per camera chunk)."""
+    shape = (n_chunks, n_cam, geo.heads, geo.head_dim)
+    return (bf16_normal(seed, TID_CAM_K, shape, std, segment),
+            bf16_normal(seed, TID_CAM_V, shape, std, segment))
 
 
 # ---------------------------------------------------------------------------
