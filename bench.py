@@ -67,7 +67,8 @@ def parse():
     p.add_argument("--shard", default="replica", choices=["replica", "heads", "ulysses"],
                    help="how N > 1 ranks split the work (see the module docstring)")
     p.add_argument("--workload", default=WORKLOAD,
-                   help=f"{WORKLOAD} (default: the headline line), commit_72f_int8, history_sweep, layers54_turn")
+                   help=f"{WORKLOAD} (default: the headline line), commit_72f_int8, history_sweep, layers54_turn, "
+                        "camera_xattn")
     return p.parse_args()
 
 
@@ -301,6 +302,40 @@ def run_extra(args, torch, nm, dev):
                                        "unit": "GB/s", "frac": byts / (ms * 1e-3) / 1e9 / hbm,
                                        "frac_of_nominal_8000": byts / (ms * 1e-3) / 1e9 / 8000.0,
                                        "peak_kind": peak_src}}), flush=True)
+        return 0
+    if args.workload == "camera_xattn":
+        # per-latent-frame camera cross-attention of a segment's video tokens (16 heads, 880
+        # tokens per frame), one camera token per frame and 4 per frame, 3- and 72-frame segments;
+        # HBM-bound: algorithmic bytes = Q read + O write + camera K/V read
+        hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+        rows = []
+        for n_frames, n_cam in ((3, 1), (72, 1), (72, 4)):
+            q, _, _ = synth.segment_qkv(geo, n_frames, 0, 6)
+            kc, vc = synth.camera_kv(geo, n_frames, n_cam, 6)
+            qd, kcd, vcd = to_dev(q), to_dev(kc), to_dev(vc)
+            out = torch.empty_like(qd)
+            byts = 2 * qd.numel() * 2 + 2 * kcd.numel() * 2
+            for _ in range(W):
+                nm.camera_attn(qd, kcd, vcd, n_frames, F, 1, out=out, stream=stream)
+            ts = []
+            for _ in range(K):
+                flush.zero_()
+                a, b = device_events(torch, 2)
+                a.record(stream)
+                nm.camera_attn(qd, kcd, vcd, n_frames, F, 1, out=out, stream=stream)
+                b.record(stream)
+                b.synchronize()
+                ts.append(a.elapsed_time(b))
+            ms = statistics.median(ts)
+            rows.append({"frames": n_frames, "camera_tokens_per_frame": n_cam, "us": ms * 1e3,
+                         "gbs": byts / (ms * 1e-3) / 1e9, "frac_of_hbm": byts / (ms * 1e-3) / 1e9 / hbm,
+                         "bytes": byts})
+        print(json.dumps({"metric": "camera_xattn_gbs", "value": rows[1]["gbs"], "unit": "GB/s",
+                          "higher_is_better": True, "steps": K, "warmup": W, "rows": rows,
+                          "peak_hbm_gbs": hbm, "peak_kind": peak_src,
+                          "config": {"workload": "camera_xattn", "heads": 16, "grid": [22, 40], "chunk_frames": 1,
+                                     "l2": "flushed before each launch", "value": "72 frames, 1 camera token"}}),
+              flush=True)
         return 0
     if args.workload == "history_sweep":
         out_rows = []

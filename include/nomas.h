@@ -67,6 +67,7 @@ extern "C" {
 
 #define NOMAS_HEAD_DIM 128
 #define NOMAS_MAX_GRID_HW 96 /* grid_h + grid_w limit (RoPE tables travel as launch arguments) */
+#define NOMAS_MAX_CAMERA_TOKENS 4096 /* camera tokens per chunk accepted by nomas_camera_attn */
 
 /*
  * One layer's K/V cache. The caller fills the configuration fields and the
@@ -162,6 +163,33 @@ int nomas_kv_commit(nomas_cache *c, const void *k, const void *v, int64_t token_
  */
 int nomas_kv_commit_layers(nomas_cache *const *caches, const void *const *k, const void *const *v,
                            int64_t token_stride, int32_t n_layers, int32_t n_frames, void *stream);
+
+/*
+ * nomas_camera_attn -- per-latent-frame camera cross-attention (model card,
+ * "Text and Camera Conditioning": after the video MLP of each double-stream
+ * block the video tokens query the projected camera features; with per-chunk
+ * camera attention and a chunk of one latent frame, each latent frame's
+ * tokens see only their own chunk's camera tokens -- one token per latent
+ * frame in the blog's reading, "Camera conditioning").
+ *   out[i][h] = softmax_j(<q[i][h], k_cam[c][j][h]> / sqrt(128)) . v_cam[c][j][h]
+ *   for video token i < n_frames * tokens_per_frame, head h, c = (i /
+ *   tokens_per_frame) / chunk_frames, j < n_cam. No RoPE, no mask inside a
+ *   chunk; fp32 arithmetic, BF16 output rounded to nearest even. With
+ *   n_cam == 1 the output is that chunk's V exactly.
+ * q     : device, BF16 bits, video tokens only, token-major [n_video][heads][128],
+ *         q_stride elements between tokens (>= heads * 128, a multiple of 8).
+ * k_cam, v_cam : device, BF16 bits, [ceil(n_frames / chunk_frames)][n_cam][heads][128],
+ *         contiguous (projected camera keys and values).
+ * out   : device, BF16 bits, [n_video][heads][128], out_stride elements between
+ *         tokens (>= heads * 128, a multiple of 8); must not overlap the inputs.
+ * All device pointers 16-byte aligned; 1 <= n_cam <= NOMAS_MAX_CAMERA_TOKENS;
+ * chunk_frames >= 1; n_video * heads < 2^31. n_frames == 0 is a no-op.
+ * Errors: NOMAS_ERR_ARG, NOMAS_ERR_ALIGN, NOMAS_ERR_DEVICE, NOMAS_ERR_CUDA;
+ * all checks happen before the launch.
+ */
+int nomas_camera_attn(const void *q, int64_t q_stride, int32_t n_frames, int32_t tokens_per_frame, int32_t heads,
+                      const void *k_cam, const void *v_cam, int32_t n_cam, int32_t chunk_frames, void *out,
+                      int64_t out_stride, void *stream);
 
 /*
  * Archive of frames leaving a window (model card, "Segment-Autoregressive

@@ -37,7 +37,7 @@ HEAD_DIM = 128
 EXPORTS = ("nomas_cache_reset", "nomas_kv_commit", "nomas_kv_commit_layers", "nomas_seg_attn_workspace_bytes",
            "nomas_seg_attn_workspace_min_bytes", "nomas_seg_attn",
            "nomas_device_status", "nomas_status_string", "nomas_seg_attn_static", "nomas_selftest_bounded_wait",
-           "nomas_kv_evicted_frames", "nomas_kv_archive_evicted")
+           "nomas_kv_evicted_frames", "nomas_kv_archive_evicted", "nomas_camera_attn")
 NOMAS_STATIC_SCRATCH_BYTES = 64 << 20
 
 
@@ -104,6 +104,8 @@ def lib():
         L.nomas_kv_evicted_frames.restype = ctypes.c_int
         L.nomas_kv_archive_evicted.argtypes = [D, I32, P, P, P, P, I32, ctypes.POINTER(I32), ctypes.POINTER(I64), P]
         L.nomas_kv_archive_evicted.restype = ctypes.c_int
+        L.nomas_camera_attn.argtypes = [P, I64, I32, I32, I32, P, P, I32, I32, P, I64, P]
+        L.nomas_camera_attn.restype = ctypes.c_int
         L.nomas_status_string.argtypes = [ctypes.c_int]
         L.nomas_status_string.restype = ctypes.c_char_p
         _lib = L
@@ -152,6 +154,32 @@ def nomas_kv_archive_evicted(desc: NomasCacheDesc, n_frames: int, hk: int | None
     rc = lib().nomas_kv_archive_evicted(ctypes.byref(desc), n_frames, hk, hv, hks, hvs, max_frames,
                                         ctypes.byref(count), ctypes.byref(first), stream)
     return rc, int(count.value), int(first.value)
+
+
+def nomas_camera_attn(q_ptr: int, q_stride: int, n_frames: int, tokens_per_frame: int, heads: int, kc_ptr: int,
+                      vc_ptr: int, n_cam: int, chunk_frames: int, out_ptr: int, out_stride: int,
+                      stream: int | None) -> int:
+    return lib().nomas_camera_attn(q_ptr, q_stride, n_frames, tokens_per_frame, heads, kc_ptr, vc_ptr, n_cam,
+                                   chunk_frames, out_ptr, out_stride, stream)
+
+
+def camera_attn(q, k_cam, v_cam, n_frames: int, tokens_per_frame: int, chunk_frames: int = 1, out=None,
+                stream=None):
+    """Per-latent-frame camera cross-attention of the video tokens q [n_frames*F][heads][128]
+    (BF16, any token stride) over k_cam, v_cam [n_chunks][n_cam][heads][128]. Returns out."""
+    torch = _torch()
+    heads = k_cam.shape[2]
+    nv = n_frames * tokens_per_frame
+    assert q.dtype == torch.bfloat16 and k_cam.dtype == q.dtype and v_cam.dtype == q.dtype
+    assert q.shape[0] == nv and q.shape[1] == heads and q.stride(1) == HEAD_DIM and q.stride(2) == 1
+    assert k_cam.is_contiguous() and v_cam.is_contiguous() and k_cam.shape == v_cam.shape
+    if out is None:
+        out = torch.empty((nv, heads, HEAD_DIM), dtype=torch.bfloat16, device=q.device)
+    assert out.shape == (nv, heads, HEAD_DIM) and out.stride(1) == HEAD_DIM and out.stride(2) == 1
+    _check(nomas_camera_attn(q.data_ptr(), q.stride(0), n_frames, tokens_per_frame, heads, k_cam.data_ptr(),
+                             v_cam.data_ptr(), k_cam.shape[1], chunk_frames, out.data_ptr(), out.stride(0),
+                             _stream_handle(stream)), "nomas_camera_attn")
+    return out
 
 
 def commit_layers(caches, ks, vs, n_frames: int, stream=None) -> None:

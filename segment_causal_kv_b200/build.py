@@ -13,7 +13,8 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
-SOURCES = ["nomas_host.cu", "rope_commit.cu", "seg_attn.cu", "nomas_static.cu", "nomas_selftest.cu"]
+SOURCES = ["nomas_host.cu", "rope_commit.cu", "seg_attn.cu", "camera_attn.cu", "nomas_static.cu",
+           "nomas_selftest.cu"]
 HEADERS = ["nomas_internal.h", "nomas_ptx.cuh"]
 LIB = os.path.join(HERE, "libnomas.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

@@ -329,6 +329,40 @@ int nomas_kv_commit_layers(nomas_cache* const* caches, const void* const* k, con
     return commit_layers(caches, k, v, token_stride, n_layers, n_frames, stream);
 }
 
+// ------------------------------------------- camera cross-attention per frame
+int nomas_camera_attn(const void* q, int64_t q_stride, int32_t n_frames, int32_t tokens_per_frame, int32_t heads,
+                      const void* k_cam, const void* v_cam, int32_t n_cam, int32_t chunk_frames, void* out,
+                      int64_t out_stride, void* stream) {
+    if (n_frames < 0 || tokens_per_frame <= 0 || heads <= 0 || n_cam < 1 || n_cam > NOMAS_MAX_CAMERA_TOKENS ||
+        chunk_frames < 1)
+        return NOMAS_ERR_ARG;
+    const int64_t rows = static_cast<int64_t>(n_frames) * tokens_per_frame * heads;
+    if (rows > (int64_t(1) << 31) - 1) return NOMAS_ERR_ARG;
+    if (rows == 0) return NOMAS_OK;
+    if (!q || !k_cam || !v_cam || !out) return NOMAS_ERR_ARG;
+    const int64_t row_elems = static_cast<int64_t>(heads) * kD;
+    if (q_stride < row_elems || out_stride < row_elems) return NOMAS_ERR_ARG;
+    if (q_stride % 8 != 0 || out_stride % 8 != 0) return NOMAS_ERR_ALIGN;
+    if (!aligned(q, 16) || !aligned(k_cam, 16) || !aligned(v_cam, 16) || !aligned(out, 16)) return NOMAS_ERR_ALIGN;
+    int rc = check_device();
+    if (rc != NOMAS_OK) return rc;
+    CamArgs a{};
+    a.q = static_cast<const uint16_t*>(q);
+    a.q_stride = q_stride;
+    a.k_cam = static_cast<const uint16_t*>(k_cam);
+    a.v_cam = static_cast<const uint16_t*>(v_cam);
+    a.out = static_cast<uint16_t*>(out);
+    a.out_stride = out_stride;
+    a.rows = rows;
+    a.heads = heads;
+    a.n_cam = n_cam;
+    a.div_heads = make_fastdiv(static_cast<uint32_t>(heads));
+    a.div_tpf = make_fastdiv(static_cast<uint32_t>(tokens_per_frame));
+    a.div_chunk = make_fastdiv(static_cast<uint32_t>(chunk_frames));
+    a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(kD)));
+    return launch_camera_attn(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? NOMAS_OK : NOMAS_ERR_CUDA;
+}
+
 // ------------------------------------------------- archive of evicted frames
 // A commit of n frames into a window of W leaves the last min(W, committed)
 // frames of the whole sequence in the window. The frames it drops are those of

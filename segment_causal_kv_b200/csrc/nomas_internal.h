@@ -139,6 +139,21 @@ struct DequantArgs {
     FastDiv div_nc;
 };
 
+// Per-latent-frame camera cross-attention: rows are (video token, head) pairs,
+// row = token * heads + head; token i uses camera chunk (i / tpf) / chunk_frames.
+struct CamArgs {
+    const uint16_t* q;      // video Q, BF16 bits, token-major
+    int64_t q_stride;       // elements between tokens
+    const uint16_t* k_cam;  // [n_chunks][n_cam][heads][128]
+    const uint16_t* v_cam;
+    uint16_t* out;          // BF16 bits, token-major
+    int64_t out_stride;
+    int64_t rows;           // n_video * heads (< 2^31)
+    int32_t heads, n_cam;
+    FastDiv div_heads, div_tpf, div_chunk;
+    float scale_log2;       // log2(e) / sqrt(128)
+};
+
 // Launch `kernel` with programmatic stream serialisation: it may begin while
 // the previous kernel on `s` finishes and must call grid_dep_wait before it
 // reads anything that kernel (or an earlier one) wrote.
@@ -166,5 +181,6 @@ cudaError_t launch_attn(const AttnArgs& a, bool int8_cache, const CUtensorMap& t
                         cudaStream_t s);
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s);
 cudaError_t launch_dequant_window(const DequantArgs& a, cudaStream_t s);
+cudaError_t launch_camera_attn(const CamArgs& a, cudaStream_t s);
 
 } // namespace nomas

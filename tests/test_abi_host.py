@@ -204,3 +204,29 @@ def test_layered_commit_argument_checks():
     assert c([ds[0], other, ds[2]]) == nm.NOMAS_ERR_STATE
     assert all(d.frames_committed == 0 for d in ds)
     assert nm.nomas_kv_commit_layers([], [], [], 2048, 3, None) == nm.NOMAS_ERR_ARG
+
+
+def test_camera_attn_argument_checks():
+    A = FAKE
+    ok = dict(q=A, qs=16 * 128, nf=3, tpf=880, h=16, kc=A, vc=A, m=1, ch=1, o=A, os=16 * 128)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return nm.nomas_camera_attn(a["q"], a["qs"], a["nf"], a["tpf"], a["h"], a["kc"], a["vc"], a["m"], a["ch"],
+                                    a["o"], a["os"], None)
+
+    assert call(nf=0) == nm.NOMAS_OK  # nothing to do, no device touched
+    assert call(nf=-1) == nm.NOMAS_ERR_ARG
+    assert call(m=0) == nm.NOMAS_ERR_ARG
+    assert call(m=4097) == nm.NOMAS_ERR_ARG
+    assert call(ch=0) == nm.NOMAS_ERR_ARG
+    assert call(h=0) == nm.NOMAS_ERR_ARG
+    assert call(tpf=0) == nm.NOMAS_ERR_ARG
+    assert call(q=None) == nm.NOMAS_ERR_ARG
+    assert call(o=None) == nm.NOMAS_ERR_ARG
+    assert call(qs=15 * 128) == nm.NOMAS_ERR_ARG
+    assert call(os=16 * 128 - 8) == nm.NOMAS_ERR_ARG
+    assert call(qs=16 * 128 + 4) == nm.NOMAS_ERR_ALIGN
+    assert call(q=A + 8) == nm.NOMAS_ERR_ALIGN
+    assert call(vc=A + 2) == nm.NOMAS_ERR_ALIGN
+    assert call(nf=1 << 20, tpf=1 << 10, h=16) == nm.NOMAS_ERR_ARG  # rows beyond 31 bits
