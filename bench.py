@@ -90,6 +90,15 @@ def workload_shape(w):
     return F, nq, nc, nk, flop
 
 
+def workload_config(w):
+    """The workload keys of the headline line's config, shared by both arms."""
+    _, nq, _, nk, flop = workload_shape(w)
+    return {"workload": WORKLOAD, "heads": w["heads"], "grid": [w["grid_h"], w["grid_w"]],
+            "history_frames": w["window"], "cache": "int8", "n_video_frames": w["cur_frames"],
+            "n_text": w["n_text"], "nq": nq, "nk": nk, "flop_per_step": flop,
+            "step": "kv_commit(3 frames) + seg_attn"}
+
+
 def commit_bytes(w):
     """Algorithmic bytes of one commit: read K, V BF16; write codes + fp32 scales."""
     F = w["grid_h"] * w["grid_w"]
@@ -229,13 +238,11 @@ def run_reference(args, rank, world):
         tot_t += dt
     value = tot_flop / tot_t / 1e12
     ms_full = flop_step / (value * 1e12) * 1e3
-    F, _, nc, _, _ = workload_shape(w)
     line = {"metric": "seg_attn_tflops", "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_full, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {"workload": WORKLOAD, "heads": w["heads"], "grid": [w["grid_h"], w["grid_w"]],
-                       "history_frames": w["window"], "cache": "int8", "n_video_frames": w["cur_frames"],
-                       "n_text": w["n_text"], "nq": nq, "nk": nk},
+            "config": dict(workload_config(w), parallelism="host oracle, rank 0 only",
+                           l2="n/a (host cores)"),
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": nthreads, "kind": "oracle",
                              "sample": f"{rows_per_step} query rows x {w['heads']} heads per step; ms_per_step "
                                        f"extrapolates to all {nq} rows"},
@@ -718,14 +725,11 @@ def main():
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": WORKLOAD, "heads": w["heads"], "grid": [w["grid_h"], w["grid_w"]],
-                   "history_frames": w["window"], "cache": "int8", "n_video_frames": w["cur_frames"],
-                   "n_text": w["n_text"], "nq": nq, "nk": nk, "flop_per_step": flop_step,
-                   "step": "kv_commit(3 frames) + seg_attn", "l2": "flushed: 512 MB written before each step",
-                   "parallelism": {"replica": f"replica x{world}",
-                                   "heads": f"heads x{world} ({nh} heads on rank 0, no collective)",
-                                   "ulysses": f"ulysses x{world} (token-sharded inputs; all-to-all to heads "
-                                              f"and back inside the step)"}[shard_mode]},
+        "config": dict(workload_config(w), l2="flushed: 512 MB written before each step",
+                       parallelism={"replica": f"replica x{world}",
+                                    "heads": f"heads x{world} ({nh} heads on rank 0, no collective)",
+                                    "ulysses": f"ulysses x{world} (token-sharded inputs; all-to-all to heads "
+                                               f"and back inside the step)"}[shard_mode]),
         "attn_ms": attn_avg_ms,
         "commit_ms": cm,
         "commit_gbs": commit_bytes(w) * nh / H / (cm * 1e-3) / 1e9,
