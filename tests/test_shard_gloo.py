@@ -154,7 +154,7 @@ def test_single_rank_exchange_is_the_identity():
     assert shard.max_over_ranks([1.0, 2.0]) == [1.0, 2.0]
 
 
-@pytest.mark.parametrize("heads,n_tokens", [(16, 80), (3, 81), (2, 7)])
+@pytest.mark.parametrize("heads,n_tokens", [(16, 80), (3, 81), (2, 7), (4, 1)])  # (4, 1): rank 1 holds no token
 def test_exchange_is_exact_and_invertible_over_two_gloo_ranks(heads, n_tokens):
     _run(_exchange_body, 2, heads, n_tokens)
 
