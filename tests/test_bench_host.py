@@ -32,3 +32,20 @@ def test_reference_arm_prints_the_contract_line():
         sys.path.remove(ROOT)
     for k, v in want.items():
         assert d["config"][k] == v, k
+
+
+def test_algorithmic_work_figures():
+    """The FLOP and byte counts bench.py divides by: 4*H*D*Nq*Nk for attention (QK^T + PV, unpadded,
+    nothing masked); K, V BF16 read plus INT8 codes and fp32 scales written for a commit."""
+    sys.path.insert(0, ROOT)
+    try:
+        import bench
+        import synth
+        w = synth.WORKLOADS[bench.WORKLOAD]
+        F, nq, nc, nk, flop = bench.workload_shape(w)
+        assert (F, nq, nc, nk) == (880, 3 * 880 + 256, 18 * 880, 18 * 880 + 3 * 880 + 256)
+        assert flop == 4 * 16 * 128 * 2896 * 18736 == 444_493_463_552
+        # 3 frames x 880 tokens x 16 heads x (K, V) x (256 B read + 128 B codes + 4 B scale written)
+        assert bench.commit_bytes(w) == 3 * 880 * 16 * 2 * (256 + 128 + 4) == 32_788_480
+    finally:
+        sys.path.remove(ROOT)
