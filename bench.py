@@ -221,15 +221,25 @@ def run_reference(args, rank, world):
     nthreads = oracle.default_threads()
     orc, q, k, v = oracle_setup(w)
     _, nq, _, nk, flop_step = workload_shape(w)
-    # one step = one query row of every head (bounded so K + W steps end in minutes)
+    # Each oracle call first rebuilds the key set of every head (dequantised
+    # cache + rotated current keys), then computes its rows. Measure that fixed
+    # cost and the cost per row, then size each step's row sample so the whole
+    # run (warm-up + timed steps) stays near the budget while the fixed cost is
+    # a small part of every step, as in the cpu_baseline leg.
     budget_s = 150.0
     rng = np.random.default_rng(1)
     t0 = time.perf_counter()
     oracle_rate(orc, q, k, v, w, np.array([0]), nthreads)
-    per_row = time.perf_counter() - t0
-    rows_per_step = int(np.clip(budget_s / max(per_row, 1e-4) / max(args.steps + args.warmup, 1), 1, 64))
+    t1 = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    oracle_rate(orc, q, k, v, w, np.sort(rng.choice(nq, 65, replace=False)), nthreads)
+    t65 = time.perf_counter() - t0
+    per_row = max((t65 - t1) / 64.0, 1e-6)
+    setup = max(t1 - per_row, 0.0)
+    step_s = budget_s / max(args.steps + args.warmup, 1)
+    rows_per_step = int(np.clip((step_s - setup) / per_row, 16, nq))
     for _ in range(args.warmup):
-        oracle_rate(orc, q, k, v, w, rng.choice(nq, rows_per_step, replace=False), nthreads)
+        oracle_rate(orc, q, k, v, w, np.sort(rng.choice(nq, rows_per_step, replace=False)), nthreads)
     tot_flop = 0.0
     tot_t = 0.0
     for _ in range(args.steps):
@@ -244,8 +254,10 @@ def run_reference(args, rank, world):
             "config": dict(workload_config(w), parallelism="host oracle, rank 0 only",
                            l2="n/a (host cores)"),
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": nthreads, "kind": "oracle",
-                             "sample": f"{rows_per_step} query rows x {w['heads']} heads per step; ms_per_step "
-                                       f"extrapolates to all {nq} rows"},
+                             "sample": f"{rows_per_step} query rows x {w['heads']} heads per step (one oracle call, "
+                                       f"which first rebuilds the {nk}-key set per head: {setup:.2f} s of the "
+                                       f"{setup + rows_per_step * per_row:.1f} s step); ms_per_step extrapolates "
+                                       f"the measured rate to all {nq} rows"},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -709,8 +721,12 @@ def main():
     attn_avg_ms = attn_total / K
     flop_rank = flop_step * nh / H  # attention FLOPs of this rank's heads
     achieved = flop_rank / (attn_avg_ms * 1e-3) / 1e12
-    peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
-    peak_burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    # the timed region is tens of milliseconds at full clock, a burst: the
+    # denominator is the burst BF16 GEMM peak; the sustained figure (a
+    # seconds-long GEMM loop under the power cap, at a lower clock) is kept
+    # as a secondary fraction
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    peak_sust = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     cm = statistics.mean(commit_ms)
     line = {
         "metric": "seg_attn_tflops",
@@ -735,8 +751,8 @@ def main():
         "commit_gbs": commit_bytes(w) * nh / H / (cm * 1e-3) / 1e9,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": traffic_from_profile("attn_kernel<bf16>"),
-                     "peak_kind": f"bf16 dense, sustained, {peak_src}",
-                     "frac_of_burst": achieved / peak_burst, "frac_of_nominal_2250": achieved / 2250.0,
+                     "peak_kind": f"bf16 dense GEMM, burst, {peak_src}",
+                     "frac_of_sustained": achieved / peak_sust, "frac_of_nominal_2250": achieved / 2250.0,
                      "kernel": "nomas_seg_attn call (INT8 window dequantised once + RoPE prep + BF16-cache "
                                "attn_kernel + split combine), CUDA events; the ncu launch list gives the split"},
         "e2e": {"value": jobs * flop_step * Ke / (e2e_total * 1e-3) / 1e12, "unit": "TFLOP/s",

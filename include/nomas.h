@@ -337,6 +337,22 @@ int nomas_seg_attn_static(const nomas_cache *c, const void *q, const void *k, co
  */
 int nomas_selftest_bounded_wait(void *workspace, void *stream);
 
+/*
+ * nomas_selftest_div127 -- check on the device, for every non-negative fp32
+ * bit pattern x (2^31 inputs), that the division the INT8 commit uses for its
+ * row scale (absmax / 127 by Markstein's method: a product with RN(1/127), an
+ * exact remainder by fma, one correction) returns the IEEE fp32 quotient
+ * RN(x / 127) bit for bit. The pages have no counterpart: this is a
+ * diagnostic of the library's commit arithmetic.
+ *   result  device pointer, 8-byte aligned, two uint32 words: the call sets
+ *           word 0 to the number of inputs whose results differ (NaN equals
+ *           NaN) and word 1 to the smallest such input pattern (0xFFFFFFFF
+ *           when there is none), once `stream` has passed the call.
+ * Returns NOMAS_OK once enqueued, NOMAS_ERR_ARG for a null or unaligned
+ * pointer, NOMAS_ERR_CUDA if a launch fails.
+ */
+int nomas_selftest_div127(void *result, void *stream);
+
 /* Human-readable name of a status code (static storage). */
 const char *nomas_status_string(int status);
 

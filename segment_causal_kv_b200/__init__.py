@@ -37,7 +37,7 @@ HEAD_DIM = 128
 EXPORTS = ("nomas_cache_reset", "nomas_kv_commit", "nomas_kv_commit_layers", "nomas_seg_attn_workspace_bytes",
            "nomas_seg_attn_workspace_min_bytes", "nomas_seg_attn",
            "nomas_device_status", "nomas_status_string", "nomas_seg_attn_static", "nomas_selftest_bounded_wait",
-           "nomas_kv_evicted_frames", "nomas_kv_archive_evicted", "nomas_camera_attn")
+           "nomas_kv_evicted_frames", "nomas_kv_archive_evicted", "nomas_camera_attn", "nomas_selftest_div127")
 NOMAS_STATIC_SCRATCH_BYTES = 64 << 20
 
 
@@ -100,6 +100,8 @@ def lib():
         L.nomas_seg_attn_static.restype = ctypes.c_int
         L.nomas_selftest_bounded_wait.argtypes = [P, P]
         L.nomas_selftest_bounded_wait.restype = ctypes.c_int
+        L.nomas_selftest_div127.argtypes = [P, P]
+        L.nomas_selftest_div127.restype = ctypes.c_int
         L.nomas_kv_evicted_frames.argtypes = [D, I32, ctypes.POINTER(I32), ctypes.POINTER(I64)]
         L.nomas_kv_evicted_frames.restype = ctypes.c_int
         L.nomas_kv_archive_evicted.argtypes = [D, I32, P, P, P, P, I32, ctypes.POINTER(I32), ctypes.POINTER(I64), P]
@@ -220,6 +222,11 @@ def nomas_selftest_bounded_wait(ws_ptr: int, stream: int | None) -> int:
     return lib().nomas_selftest_bounded_wait(ws_ptr, stream)
 
 
+def nomas_selftest_div127(result_ptr: int, stream: int | None) -> int:
+    """Enqueue the exhaustive check of the commit's division by 127 (two uint32 result words)."""
+    return lib().nomas_selftest_div127(result_ptr, stream)
+
+
 def nomas_device_status(ws_ptr: int, stream: int | None) -> int:
     return lib().nomas_device_status(ws_ptr, stream)
 
@@ -248,25 +255,30 @@ class KVCache:
 
     mode: "int8" (codes + fp32 per-(token, head) scales) or "bf16".
     window: history budget in latent frames (0 = full history).
+    alloc: optional allocator (shape, dtype, device) -> zero-filled tensor for the
+    cache and workspace buffers (default torch.zeros); the tests pass one that
+    surrounds every buffer with canary bands.
     """
 
     def __init__(self, mode: str, heads: int, grid_h: int, grid_w: int, window: int, capacity: int,
-                 theta: float = 256.0, device=None):
+                 theta: float = 256.0, device=None, alloc=None):
         torch = _torch()
         self.device = torch.device(device if device is not None else "cuda")
+        zeros = alloc or (lambda shape, dtype, dev: torch.zeros(shape, dtype=dtype, device=dev))
+        self._zeros = zeros
         self.mode = mode
         self.heads, self.grid_h, self.grid_w = heads, grid_h, grid_w
         self.window, self.capacity = window, capacity
         F = grid_h * grid_w
         if mode == "int8":
-            self.k = torch.zeros((heads, capacity * F, HEAD_DIM), dtype=torch.int8, device=self.device)
-            self.v = torch.zeros_like(self.k)
-            self.k_scale = torch.zeros((heads, capacity * F), dtype=torch.float32, device=self.device)
-            self.v_scale = torch.zeros_like(self.k_scale)
+            self.k = zeros((heads, capacity * F, HEAD_DIM), torch.int8, self.device)
+            self.v = zeros((heads, capacity * F, HEAD_DIM), torch.int8, self.device)
+            self.k_scale = zeros((heads, capacity * F), torch.float32, self.device)
+            self.v_scale = zeros((heads, capacity * F), torch.float32, self.device)
             m = NOMAS_CACHE_INT8
         elif mode == "bf16":
-            self.k = torch.zeros((heads, capacity * F, HEAD_DIM), dtype=torch.bfloat16, device=self.device)
-            self.v = torch.zeros_like(self.k)
+            self.k = zeros((heads, capacity * F, HEAD_DIM), torch.bfloat16, self.device)
+            self.v = zeros((heads, capacity * F, HEAD_DIM), torch.bfloat16, self.device)
             self.k_scale = self.v_scale = None
             m = NOMAS_CACHE_BF16
         else:
@@ -348,7 +360,7 @@ class KVCache:
         torch = _torch()
         need = self.workspace_bytes(n_video_frames, n_text)
         if self._ws is None or self._ws.numel() < need:
-            self._ws = torch.zeros(max(need, 256), dtype=torch.uint8, device=self.device)
+            self._ws = self._zeros((max(need, 256),), torch.uint8, self.device)
         return self._ws
 
     def seg_attn(self, q, k, v, n_video_frames: int, n_text: int, out=None, lse=None, workspace=None,

@@ -25,7 +25,7 @@ def built():
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(nomas_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(nomas_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_header_declares_the_binding_exports():
@@ -230,3 +230,8 @@ def test_camera_attn_argument_checks():
     assert call(q=A + 8) == nm.NOMAS_ERR_ALIGN
     assert call(vc=A + 2) == nm.NOMAS_ERR_ALIGN
     assert call(nf=1 << 20, tpf=1 << 10, h=16) == nm.NOMAS_ERR_ARG  # rows beyond 31 bits
+
+
+def test_div127_selftest_rejects_bad_pointers_before_any_cuda_call():
+    assert nm.nomas_selftest_div127(None, None) == nm.NOMAS_ERR_ARG
+    assert nm.nomas_selftest_div127(FAKE + 4, None) == nm.NOMAS_ERR_ARG

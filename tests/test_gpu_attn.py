@@ -9,7 +9,7 @@ import pytest
 
 import oracle
 import synth
-from harness import MAX_ABS, REL_L2, current_segment, errors, make_caches, sample_rows, to_dev, to_f64
+from harness import MAX_ABS, REL_L2, Guards, current_segment, errors, make_caches, sample_rows, to_dev, to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -19,22 +19,22 @@ def run_case(w, rows=None, check_lse=True, rel_l2=REL_L2, path="once"):
     dequantised once, then the BF16-cache kernel runs); "fused" = the minimum workspace
     (the INT8 kernel converts each tile in shared memory)."""
     torch = __import__("torch")
-    gpu, orc = make_caches(w)
+    g = Guards()
+    gpu, orc = make_caches(w, guards=g)
     q, k, v = current_segment(w)
     nq = q.shape[0]
-    lse = torch.full((w["heads"], nq), float("nan"), dtype=torch.float32, device="cuda")
-    out = torch.full((nq, w["heads"], 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse = g.alloc((w["heads"], nq), torch.float32, fill=float("nan"))
+    out = g.alloc((nq, w["heads"], 128), torch.bfloat16, fill=float("nan"))
     ws = None
     if path == "fused":
         need = gpu.workspace_min_bytes(w["cur_frames"], w["n_text"])
-        if w["mode"] == "int8" and gpu.valid_frames > 0:
-            assert need < gpu.workspace_bytes(w["cur_frames"], w["n_text"])
-        ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+        ws = g.alloc((need,), torch.uint8)
     gpu.seg_attn(to_dev(q), to_dev(k), to_dev(v), w["cur_frames"], w["n_text"], out=out, lse=lse, workspace=ws)
     torch.cuda.synchronize()
     assert gpu.device_status() == 0
     if ws is not None:
         assert int(ws[:4].view(torch.int32).item()) == 0
+    g.check()
     ref, ref_lse = orc.seg_attn(q, k, v, w["cur_frames"], w["n_text"], rows=rows)
     got = to_f64(out)
     got_lse = lse.cpu().numpy().astype(np.float64)
@@ -43,6 +43,7 @@ def run_case(w, rows=None, check_lse=True, rel_l2=REL_L2, path="once"):
         got_lse = got_lse[:, rows]
     assert np.isfinite(got).all()
     mx, rel = errors(got, ref)
+    print(f"[parity] {w.get('name', '')} {w['mode']} {path}: max-abs {mx:.3e} rel-L2 {rel:.3e}")
     assert mx <= MAX_ABS and rel <= rel_l2, (mx, rel)
     if check_lse:
         # the log-sum-exp carries the score error of BF16 operands, which grows with |score|
@@ -110,17 +111,25 @@ def test_wrapped_int8_ring(path):
 
 @pytest.mark.parametrize("path", INT8_PATHS)
 def test_peaky_softmax(path):
-    """Scores three times larger exercise the running-max rescaling of O.
-
-    The kernel's operands are BF16 (rotated Q and K, dequantised cache, P),
-    each rounded with relative error up to 2^-9. A score error grows with the
-    score's size, and a peaked softmax passes it on to the output almost
-    undamped: with q_std = 3 the expected relative L2 error is about three
-    times the N(0,1) figure (~2e-3 measured), so this stress case is held to
-    rel-L2 <= 1e-2 while keeping the max-abs bound of 2e-2.
-    """
+    """Scores three times larger (q_std = 3) make the softmax peaked: a few keys
+    carry most of each row's weight, so errors in the running max, the O
+    rescaling or the normalisation reach the output undamped. Held to the
+    same bar as every other case (max-abs 2e-2, rel-L2 5e-3)."""
     run_case(wl(heads=2, grid_h=8, grid_w=16, mode="int8", window=4, capacity=4, hist_commits=[2, 2],
-                cur_frames=2, n_text=30, seed=12, q_std=3.0), rel_l2=1e-2, path=path)
+                cur_frames=2, n_text=30, seed=12, q_std=3.0), path=path)
+
+
+@pytest.mark.parametrize("mode", ["bf16", "int8"])
+def test_rising_scores_force_rescales(mode):
+    """Scores that rise from frame to frame of the history (K of frame s scaled
+    by 1.25^s): a later KV tile's maximum exceeds the reference max the row
+    started from, so the reference moves and O is rescaled in tensor memory
+    partway through the row. Growth is kept moderate so that the scores stay
+    within the range where BF16 operands meet the parity bar."""
+    w = wl(heads=2, grid_h=8, grid_w=16, mode=mode, window=6 if mode == "int8" else 0,
+           capacity=6 if mode == "int8" else 8, hist_commits=[1] * 6, cur_frames=1, n_text=8, seed=17,
+           kv_ramp=1.25)
+    run_case(w)
 
 
 @pytest.mark.parametrize("path", INT8_PATHS)
@@ -162,13 +171,11 @@ def test_cache_is_read_only():
 
 
 @pytest.mark.parametrize("path", INT8_PATHS)
-def test_single_gpu_configuration_sampled_rows(path):
-    w = synth.WORKLOADS["single_gpu_int8_18f"]
-    F = w["grid_h"] * w["grid_w"]
-    nq = w["cur_frames"] * F + w["n_text"]
-    rows = sample_rows(nq, F, w["cur_frames"], per_head=48)
-    mx, rel = run_case(w, rows=rows, path=path)
-    print(f"single-GPU cfg ({path}): max-abs {mx:.3e} rel-L2 {rel:.3e}")
+def test_single_gpu_configuration_all_rows(path):
+    """The single-GPU configuration (16 heads, 18-frame INT8 history, 2896
+    queries x 18,736 keys), every output row against the oracle."""
+    w = dict(synth.WORKLOADS["single_gpu_int8_18f"], name="single_gpu_int8_18f")
+    run_case(w, path=path)
 
 
 def test_int8_paths_agree():

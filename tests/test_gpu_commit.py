@@ -155,3 +155,82 @@ def test_layered_commit_matches_per_layer_commits(mode, n_layers):
             o.commit(k, v, nf)
         for g, o in zip(gpus, orcs):
             assert_cache_equal(g, o)
+
+
+
+def _tie_row(scale_exp: int, rng) -> np.ndarray:
+    """A 128-element row whose absmax is 127 * 2^e (so the fp32 scale is exactly
+    2^e) and whose other elements sit exactly halfway between two codes
+    (x / scale = k + 1/2), or 1/64 beside a small half (k < 3, where 1/64 is
+    still a whole number of BF16 ulps). Dims 0-15 (the t block of
+    RoPE) are zero, so the row passes the commit's rotation unchanged at grid
+    cell (0, 0) of any frame. Returns the row as float64 (exact BF16 values)."""
+    s = 2.0 ** scale_exp
+    x = np.zeros(128, np.float64)
+    x[16] = 127 * s
+    x[17] = -127 * s
+    fixed = np.array([0.5, 1.5, 2.5, 3.5, 62.5, 63.5, 64.5, 125.5, 126.5])
+    fixed = np.concatenate([fixed, -fixed])
+    x[18:36] = fixed * s
+    k = rng.integers(0, 127, size=76)
+    sgn = np.where(rng.integers(0, 2, size=76) == 1, 1.0, -1.0)
+    x[36:112] = sgn * (k + 0.5) * s
+    off = np.where(rng.integers(0, 2, size=16) == 1, 1.0, -1.0) / 64.0
+    x[112:128] = (rng.integers(0, 3, size=16) + 0.5 + off) * s
+    return x
+
+
+def _bits(x: np.ndarray) -> np.ndarray:
+    b = synth.f32_to_bf16_bits(x.astype(np.float32))
+    assert np.array_equal(synth.bf16_bits_to_f32(b).astype(np.float64), x)  # exact in BF16
+    return b
+
+
+def test_commit_int8_round_half_even_ties():
+    """Hand-built exact ties x / scale = k + 1/2 in K and V rows: the codes are
+    round-half-to-even of the quotient (checked against the rule computed here
+    from the constructed values, and bit for bit against the oracle's commit).
+    K carries the ties at grid cell (0, 0) of each frame, whose h and w
+    rotations are the identity; V carries them at every token. The scales are
+    powers of two, so the kernel's reciprocal product is exact and every tie
+    lies exactly on the rounding boundary its packed fast path must hand to the
+    exact path."""
+    import segment_causal_kv_b200 as nm
+    H, gh, gw, W = 3, 4, 8, 4
+    F = gh * gw
+    geo = synth.Geometry(H, gh, gw)
+    rng = np.random.default_rng(33)
+    gpu = nm.KVCache("int8", H, gh, gw, W, W)
+    orc = oracle.OracleCache(oracle.MODE_INT8, H, gh, gw, W, W)
+    want = {}  # (tensor, head, slot row) -> (expected codes, expected scale)
+    frame0 = 0
+    for seg, nf in enumerate([2, 3]):  # the second segment wraps the 4-frame ring
+        k, v = synth.history_kv(geo, nf, 95, seg)
+        for f in range(nf):
+            slot = (frame0 + f) % W
+            for h in range(H):
+                xk = _tie_row(-4 - h, rng)
+                k[f * F, h] = _bits(xk)
+                want[("k", h, slot * F)] = (np.rint(xk / 2.0 ** (-4 - h)), 2.0 ** (-4 - h))
+                for t in range(f * F, (f + 1) * F):
+                    xv = _tie_row(-6 + h, rng)
+                    v[t, h] = _bits(xv)
+                    want[("v", h, slot * F + t - f * F)] = (np.rint(xv / 2.0 ** (-6 + h)), 2.0 ** (-6 + h))
+        gpu.commit(to_dev(k), to_dev(v), nf)
+        orc.commit(k, v, nf)
+        assert_cache_equal(gpu, orc)
+        frame0 += nf
+    codes = {"k": gpu.k.cpu().numpy(), "v": gpu.v.cpu().numpy()}
+    scales = {"k": gpu.k_scale.cpu().numpy(), "v": gpu.v_scale.cpu().numpy()}
+    # frames 1..4 are in the window; frame 0's slot was overwritten by frame 4
+    live = {(1 + i) % W for i in range(W)}
+    checked = 0
+    for (t, h, row), (c, sc) in want.items():
+        if row // F not in live:
+            continue
+        assert scales[t][h, row] == np.float32(sc)
+        assert np.array_equal(codes[t][h, row].astype(np.float64), c), (t, h, row)
+        checked += 1
+    assert checked == H * W * (1 + F)
+    # np.rint rounds half to even: the fixed ties landed on even codes
+    assert np.all(codes["k"][0, F, 18:36] % 2 == 0)
