@@ -7,9 +7,9 @@ One step = the whole hot path at steady state on one layer's cache:
   22x40 = 2640 video tokens + 256 text tokens, 16 heads x 128) over the
   18-frame INT8 history (15,840 cached tokens): Nk = 18,736 keys.
 The history stays at 18 frames, so every step does the same work.
-nomas_seg_attn gets the full workspace (nomas_seg_attn_workspace_bytes), so
-the INT8 window is dequantised once per call into a BF16 copy that the
-BF16-cache attention kernel reads.
+nomas_seg_attn gets the workspace of its fastest plan
+(nomas_seg_attn_workspace_bytes); the INT8 cache tiles are converted to BF16
+in shared memory inside the attention kernel.
 
 Metric: seg-attention TFLOP/s = 4*H*D*Nq*Nk FLOP per step / step time
 (QK^T + PV, unpadded, no softmax credit), and ms per layer-step.
@@ -750,21 +750,21 @@ def main():
         "commit_ms": cm,
         "commit_gbs": commit_bytes(w) * nh / H / (cm * 1e-3) / 1e9,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": traffic_from_profile("attn_kernel<bf16>"),
+                     "frac": achieved / peak, "traffic": traffic_from_profile("attn_kernel<int8>"),
                      "peak_kind": f"bf16 dense GEMM, burst, {peak_src}",
                      "frac_of_sustained": achieved / peak_sust, "frac_of_nominal_2250": achieved / 2250.0,
-                     "kernel": "nomas_seg_attn call (INT8 window dequantised once + RoPE prep + BF16-cache "
-                               "attn_kernel + split combine), CUDA events; the ncu launch list gives the split"},
+                     "kernel": "nomas_seg_attn call (RoPE prep + INT8-cache attn_kernel, which converts cache "
+                               "tiles in shared memory and merges its KV splits), CUDA events; the ncu launch "
+                               "list gives the split"},
         "e2e": {"value": jobs * flop_step * Ke / (e2e_total * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": Ke,
                 "ms_per_step": e2e_total / Ke,
                 "form": "pipelined: step i+1 upload and step i-1 readback overlap step i; L2 not flushed"},
         "e2e_serial": {"value": jobs * flop_step / (serial_avg * 1e-3) / 1e12, "unit": "TFLOP/s",
                        "ms_per_step": serial_avg, "form": "one step at a time, L2 flushed before each"},
-        # per step: commit, RoPE prep, attention, the INT8 window dequantisation and the
-        # split combine when used
-        "gpu_launches": K * (3 + _dequant_launches(cache, w["cur_frames"], w["n_text"])
-                             + _combine_launches(cache, w["cur_frames"], w["n_text"])),
+        # per step: the commit, the RoPE prep and the attention kernel (which merges
+        # its KV splits itself)
+        "gpu_launches": K * 3,
         "commit_traffic_profile": traffic_from_profile("commit_kernel<int8>"),
         "clocks": clocks,
     }
@@ -775,21 +775,6 @@ def main():
             line["cpu_baseline"] = {"value": None, "error": str(e)}
     print(json.dumps(line), flush=True)
     return 0
-
-
-def _combine_launches(cache, n_video_frames: int, n_text: int) -> int:
-    """1 when the shape uses KV splits (the combine kernel runs), else 0: the
-    minimum workspace holds split partials beyond the header and rotated Q, K."""
-    ws = cache.workspace_min_bytes(n_video_frames, n_text)
-    h, F = cache.heads, cache.tokens_per_frame
-    nq = n_video_frames * F + n_text
-    qk = 2 * ((h * nq * HEAD_DIM * 2 + 255) // 256 * 256)
-    return 1 if ws > 256 + qk + 256 else 0
-
-
-def _dequant_launches(cache, n_video_frames: int, n_text: int) -> int:
-    """1 when the call dequantises an INT8 window once (full workspace), else 0."""
-    return 1 if cache.workspace_bytes(n_video_frames, n_text) > cache.workspace_min_bytes(n_video_frames, n_text) else 0
 
 
 if __name__ == "__main__":

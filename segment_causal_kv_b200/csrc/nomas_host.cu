@@ -149,22 +149,20 @@ bool make_tmap(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint6
 struct Plan {
     int64_t tpf, nv, nq, nc;
     int tiles_c, tiles_q, pairs, splits, tiles_per_split;
-    size_t off_qt, off_kt, off_po, off_pml;
-    size_t total_min; // the fused kernel's workspace (the smallest accepted)
-    size_t off_kd, off_vd;
-    size_t total;     // with the BF16 copy of an INT8 window (dequantise once)
+    size_t off_qt, off_kt, off_po, off_pml, off_cnt;
+    size_t total; // workspace bytes of this plan
 };
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Split count minimising a makespan model: waves x (tiles per split + fixed
-// per-CTA cost), for a 148-SM part with one CTA per SM.
-void choose_splits(int units, int tiles, int& splits, int& tps) {
+// per-CTA cost), for a 148-SM part with one CTA per SM; at most max_splits.
+void choose_splits(int units, int tiles, int max_splits, int& splits, int& tps) {
     double best = 1e300;
     splits = 1;
     tps = tiles > 0 ? tiles : 1;
     if (tiles <= 0) return;
-    for (int s = 1; s <= 32; ++s) {
+    for (int s = 1; s <= max_splits; ++s) {
         const int t = (tiles + s - 1) / s;
         const int s_eff = (tiles + t - 1) / t;
         if (s > 1 && t < 4) break;
@@ -179,11 +177,10 @@ void choose_splits(int units, int tiles, int& splits, int& tps) {
     }
 }
 
-// The dequantise-once kernel indexes (tensor, row, 16-code part) in 32 bits,
-// with a few grid strides of headroom.
-bool dequant_once_fits(int heads, int64_t nc) { return static_cast<int64_t>(heads) * nc < (int64_t(1) << 27); }
-
-Plan make_plan(const nomas_cache* c, int32_t n_video_frames, int32_t n_text) {
+// Workspace layout of a plan: status header, rotated Q and K (head-major),
+// and with splits > 1 the split partials [splits][units][32][256] float4,
+// their (max, sum) pairs [splits][units][256] and one arrival counter per unit.
+Plan make_plan(const nomas_cache* c, int32_t n_video_frames, int32_t n_text, int max_splits) {
     Plan p{};
     p.tpf = static_cast<int64_t>(c->grid_h) * c->grid_w;
     p.nv = static_cast<int64_t>(n_video_frames) * p.tpf;
@@ -192,22 +189,32 @@ Plan make_plan(const nomas_cache* c, int32_t n_video_frames, int32_t n_text) {
     p.tiles_c = static_cast<int>((p.nc + kBM - 1) / kBM);
     p.tiles_q = static_cast<int>((p.nq + kBM - 1) / kBM);
     p.pairs = (p.tiles_q + 1) / 2;
-    choose_splits(c->heads * p.pairs, p.tiles_c + p.tiles_q, p.splits, p.tiles_per_split);
+    const int units = c->heads * p.pairs;
+    choose_splits(units, p.tiles_c + p.tiles_q, max_splits, p.splits, p.tiles_per_split);
     const size_t qk_bytes = static_cast<size_t>(c->heads) * p.nq * kD * 2;
-    const size_t prow = static_cast<size_t>(p.splits) * c->heads * p.pairs * 2 * kBM;
+    const size_t prow = static_cast<size_t>(p.splits) * units * 2 * kBM;
+    const bool sp = p.splits > 1;
     p.off_qt = kWsHeader;
     p.off_kt = round_up(p.off_qt + qk_bytes, 256);
     p.off_po = round_up(p.off_kt + qk_bytes, 256);
-    p.off_pml = p.off_po + (p.splits > 1 ? prow * kD * sizeof(float) : 0);
-    p.total_min = round_up(p.off_pml + (p.splits > 1 ? prow * sizeof(float2) : 0), 256);
-    p.off_kd = p.off_vd = p.total = p.total_min;
-    if (c->mode == NOMAS_CACHE_INT8 && p.nc > 0 && dequant_once_fits(c->heads, p.nc)) {
-        const size_t copy = round_up(static_cast<size_t>(c->heads) * p.nc * kD * 2, 256);
-        p.off_kd = p.total_min;
-        p.off_vd = p.off_kd + copy;
-        p.total = p.off_vd + copy;
-    }
+    p.off_pml = p.off_po + (sp ? prow * kD * sizeof(float) : 0);
+    p.off_cnt = round_up(p.off_pml + (sp ? prow * sizeof(float2) : 0), 256);
+    p.total = round_up(p.off_cnt + (sp ? static_cast<size_t>(units) * sizeof(unsigned) : 0), 256);
     return p;
+}
+
+constexpr int kMaxSplits = 32;
+
+// The fastest plan whose workspace fits in `bytes` (fewer splits need less:
+// splits = 1 keeps no partials). Returns false when not even that fits.
+bool fit_plan(const nomas_cache* c, int32_t n_video_frames, int32_t n_text, size_t bytes, Plan& out) {
+    int cap = kMaxSplits;
+    while (true) {
+        out = make_plan(c, n_video_frames, n_text, cap);
+        if (out.total <= bytes) return true;
+        if (out.splits <= 1) return false;
+        cap = out.splits - 1;
+    }
 }
 
 } // namespace
@@ -429,12 +436,12 @@ int nomas_kv_archive_evicted(const nomas_cache* c, int32_t n_frames, void* host_
 
 size_t nomas_seg_attn_workspace_bytes(const nomas_cache* c, int32_t n_video_frames, int32_t n_text) {
     if (validate_state(c) != NOMAS_OK || n_video_frames < 0 || n_text < 0) return 0;
-    return make_plan(c, n_video_frames, n_text).total;
+    return make_plan(c, n_video_frames, n_text, kMaxSplits).total;
 }
 
 size_t nomas_seg_attn_workspace_min_bytes(const nomas_cache* c, int32_t n_video_frames, int32_t n_text) {
     if (validate_state(c) != NOMAS_OK || n_video_frames < 0 || n_text < 0) return 0;
-    return make_plan(c, n_video_frames, n_text).total_min;
+    return make_plan(c, n_video_frames, n_text, 1).total;
 }
 
 int nomas_seg_attn(const nomas_cache* c, const void* q, const void* k, const void* v, int64_t token_stride,
@@ -443,14 +450,14 @@ int nomas_seg_attn(const nomas_cache* c, const void* q, const void* k, const voi
     int rc = validate_state(c);
     if (rc != NOMAS_OK) return rc;
     if (n_video_frames < 0 || n_text < 0) return NOMAS_ERR_ARG;
-    const Plan p = make_plan(c, n_video_frames, n_text);
+    Plan p = make_plan(c, n_video_frames, n_text, 1);
     if (p.nq == 0) return NOMAS_OK;
     if (p.nq > (int64_t(1) << 30) || p.nq * c->heads >= (int64_t(1) << 31)) return NOMAS_ERR_ARG;
     if (!q || !k || !v || !out) return NOMAS_ERR_ARG;
     if (token_stride < static_cast<int64_t>(c->heads) * kD || token_stride % 8 != 0) return NOMAS_ERR_ARG;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16)) return NOMAS_ERR_ALIGN;
     if (lse && !aligned(lse, 4)) return NOMAS_ERR_ALIGN;
-    if (!workspace || workspace_bytes < p.total_min) return NOMAS_ERR_WORKSPACE;
+    if (!workspace || !fit_plan(c, n_video_frames, n_text, workspace_bytes, p)) return NOMAS_ERR_WORKSPACE;
     if (!aligned(workspace, 256)) return NOMAS_ERR_ALIGN;
     if ((rc = check_device()) != NOMAS_OK) return rc;
 
@@ -458,8 +465,11 @@ int nomas_seg_attn(const nomas_cache* c, const void* q, const void* k, const voi
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     uint16_t* qt = reinterpret_cast<uint16_t*>(ws + p.off_qt);
     uint16_t* kt = reinterpret_cast<uint16_t*>(ws + p.off_kt);
+    unsigned* counters = reinterpret_cast<unsigned*>(ws + p.off_cnt);
+    const int units = c->heads * p.pairs;
 
-    // 1) RoPE + relayout of the current Q and K (video frames in chunks)
+    // 1) RoPE + relayout of the current Q and K (video frames in chunks); the
+    //    first launch also zeroes the split-KV arrival counters
     RopeTab tab;
     fill_hw(tab, c->rope_theta, c->grid_h, c->grid_w);
     {
@@ -485,6 +495,8 @@ int nomas_seg_attn(const nomas_cache* c, const void* q, const void* k, const voi
             a.div_heads = make_fastdiv(static_cast<uint32_t>(c->heads));
             a.div_tpf = make_fastdiv(static_cast<uint32_t>(p.tpf));
             a.div_gw = make_fastdiv(static_cast<uint32_t>(c->grid_w));
+            a.counters = counters;
+            a.n_counters = (f0 == 0 && p.splits > 1) ? units : 0;
             if (nf > 0) fill_t(tab, c->rope_theta, c->frames_committed + f0, nf);
             if (a.tok1 > a.tok0 && launch_prep(a, tab, s) != cudaSuccess) return NOMAS_ERR_CUDA;
             f0 += nf;
@@ -492,49 +504,25 @@ int nomas_seg_attn(const nomas_cache* c, const void* q, const void* k, const voi
         } while (true);
     }
 
-    // 2) an INT8 window with room for its BF16 copy is dequantised once here and
-    //    read by the BF16-cache kernel; otherwise the fused kernel converts it
-    //    tile by tile in shared memory (once per CTA that reads the tile)
-    const bool int8 = c->mode == NOMAS_CACHE_INT8;
-    const bool dequant_once = int8 && p.total > p.total_min && workspace_bytes >= p.total;
-    uint16_t* kd = reinterpret_cast<uint16_t*>(ws + p.off_kd);
-    uint16_t* vd = reinterpret_cast<uint16_t*>(ws + p.off_vd);
-    if (dequant_once) {
-        DequantArgs d{};
-        d.kc = static_cast<const int8_t*>(c->k);
-        d.vc = static_cast<const int8_t*>(c->v);
-        d.ks = c->k_scale;
-        d.vs = c->v_scale;
-        d.kd = kd;
-        d.vd = vd;
-        d.cap_tok = static_cast<int64_t>(c->capacity_frames) * p.tpf;
-        d.nc = static_cast<int32_t>(p.nc);
-        d.heads = c->heads;
-        d.div_nc = make_fastdiv(static_cast<uint32_t>(p.nc));
-        if (launch_dequant_window(d, s) != cudaSuccess) return NOMAS_ERR_CUDA;
-    }
-
-    // 3) tensor maps
+    // 2) tensor maps
     CUtensorMap tm_q, tm_kcur, tm_vcur, tm_kc, tm_vc;
     const uint64_t row_bytes = kD * 2;
     bool ok = make_tmap(&tm_q, qt, kD, p.nq, c->heads, row_bytes, p.nq * row_bytes, kBM, 1) &&
               make_tmap(&tm_kcur, kt, kD, p.nq, c->heads, row_bytes, p.nq * row_bytes, kBM, 1) &&
               make_tmap(&tm_vcur, v, kD, c->heads, p.nq, row_bytes, token_stride * 2, 1, kBM);
     const int64_t cap_tok = static_cast<int64_t>(c->capacity_frames) * p.tpf;
-    if (c->mode == NOMAS_CACHE_BF16) {
+    const bool int8 = c->mode == NOMAS_CACHE_INT8;
+    if (!int8) {
         const uint64_t nc_ext = p.nc > 0 ? p.nc : 1;
         ok = ok && make_tmap(&tm_kc, c->k, kD, nc_ext, c->heads, row_bytes, cap_tok * row_bytes, kBM, 1) &&
              make_tmap(&tm_vc, c->v, kD, nc_ext, c->heads, row_bytes, cap_tok * row_bytes, kBM, 1);
-    } else if (dequant_once) {
-        ok = ok && make_tmap(&tm_kc, kd, kD, p.nc, c->heads, row_bytes, p.nc * row_bytes, kBM, 1) &&
-             make_tmap(&tm_vc, vd, kD, p.nc, c->heads, row_bytes, p.nc * row_bytes, kBM, 1);
     } else {
-        tm_kc = tm_q;
+        tm_kc = tm_q; // unused: the INT8 kernel converts cache tiles itself
         tm_vc = tm_q;
     }
     if (!ok) return NOMAS_ERR_CUDA;
 
-    // 4) attention (+ combine of KV splits)
+    // 3) attention; with splits > 1 the last CTA of each unit merges the splits
     AttnArgs a{};
     a.heads = c->heads;
     a.nq = static_cast<int32_t>(p.nq);
@@ -551,24 +539,12 @@ int nomas_seg_attn(const nomas_cache* c, const void* q, const void* k, const voi
     a.vsc = c->v_scale;
     a.out = static_cast<uint16_t*>(out);
     a.lse = lse;
-    a.part_o = reinterpret_cast<float*>(ws + p.off_po);
+    a.part_o = reinterpret_cast<float4*>(ws + p.off_po);
     a.part_ml = reinterpret_cast<float2*>(ws + p.off_pml);
+    a.counters = counters;
     a.err = reinterpret_cast<unsigned*>(ws);
     a.scale_log2 = static_cast<float>(1.4426950408889634 / sqrt(static_cast<double>(kD)));
-    if (launch_attn(a, int8 && !dequant_once, tm_q, tm_kcur, tm_vcur, tm_kc, tm_vc, s) != cudaSuccess)
-        return NOMAS_ERR_CUDA;
-    if (p.splits > 1) {
-        CombineArgs cb{};
-        cb.heads = c->heads;
-        cb.nq = static_cast<int32_t>(p.nq);
-        cb.pairs = p.pairs;
-        cb.splits = p.splits;
-        cb.part_o = a.part_o;
-        cb.part_ml = a.part_ml;
-        cb.out = a.out;
-        cb.lse = lse;
-        if (launch_combine(cb, s) != cudaSuccess) return NOMAS_ERR_CUDA;
-    }
+    if (launch_attn(a, int8, tm_q, tm_kcur, tm_vcur, tm_kc, tm_vc, s) != cudaSuccess) return NOMAS_ERR_CUDA;
     return NOMAS_OK;
 }
 

@@ -90,6 +90,8 @@ struct PrepArgs {
     int32_t tok0, tok1;     // token range handled by this launch
     int32_t frame0;         // segment-local frame of table row t[0]
     FastDiv div_heads, div_tpf, div_gw;
+    unsigned* counters;     // split-KV arrival counters of the attention call, zeroed here
+    int32_t n_counters;     // (by the launch with tok0 == 0 only)
 };
 
 struct AttnArgs {
@@ -108,35 +110,11 @@ struct AttnArgs {
     const float* vsc;
     uint16_t* out;          // [nq][heads][128] BF16
     float* lse;             // [heads][nq] or null
-    float* part_o;          // [splits][heads][pairs*256][128] fp32 (splits > 1)
-    float2* part_ml;        // [splits][heads][pairs*256] (running max in log2 units, sum)
+    float4* part_o;         // splits > 1: [splits][units][32][256] unnormalised O, 4 dims per float4
+    float2* part_ml;        // splits > 1: [splits][units][256] (reference max in log2 units, sum)
+    unsigned* counters;     // splits > 1: [units] arrivals; the last CTA of a unit merges the splits
     unsigned* err;          // workspace status word
     float scale_log2;       // log2(e) / sqrt(128)
-};
-
-struct CombineArgs {
-    int32_t heads, nq, pairs, splits;
-    const float* part_o;
-    const float2* part_ml;
-    uint16_t* out;
-    float* lse;
-};
-
-// Dequantisation of an INT8 cache's visible window into a BF16 copy, once per
-// attention call: rows [0, nc) of every head of K and V, codes * scale rounded
-// to BF16 (the same values the fused kernel converts in shared memory), written
-// head-major [heads][nc][128].
-struct DequantArgs {
-    const int8_t* kc;
-    const int8_t* vc;
-    const float* ks;
-    const float* vs;
-    uint16_t* kd;
-    uint16_t* vd;
-    int64_t cap_tok; // token capacity of one head's slab in the cache
-    int32_t nc;      // visible tokens per head
-    int32_t heads;
-    FastDiv div_nc;
 };
 
 // Per-latent-frame camera cross-attention: rows are (video token, head) pairs,
@@ -179,8 +157,6 @@ cudaError_t launch_prep(const PrepArgs& a, const RopeTab& tab, cudaStream_t s);
 cudaError_t launch_attn(const AttnArgs& a, bool int8_cache, const CUtensorMap& tm_q, const CUtensorMap& tm_kcur,
                         const CUtensorMap& tm_vcur, const CUtensorMap& tm_kc, const CUtensorMap& tm_vc,
                         cudaStream_t s);
-cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s);
-cudaError_t launch_dequant_window(const DequantArgs& a, cudaStream_t s);
 cudaError_t launch_camera_attn(const CamArgs& a, cudaStream_t s);
 
 } // namespace nomas

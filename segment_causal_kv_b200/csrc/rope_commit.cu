@@ -278,9 +278,11 @@ __global__ void __launch_bounds__(kThreads) commit_kernel(const __grid_constant_
 
 __global__ void __launch_bounds__(kThreads) prep_kernel(const __grid_constant__ PrepArgs a,
                                                         const __grid_constant__ RopeTab tab) {
-    // the next kernel of the call (the window dequantisation, or the attention
-    // kernel, which waits for this one) may start launching right away
+    // the attention kernel of the call (which waits for this one before it
+    // reads anything) may start launching right away
     grid_dep_launch();
+    if (blockIdx.x == 0)
+        for (int i = threadIdx.x; i < a.n_counters; i += blockDim.x) a.counters[i] = 0u;
     __shared__ __align__(16) float2 s_t[kMaxFramesPerLaunch * kTPairs];
     __shared__ __align__(16) float2 s_hw[NOMAS_MAX_GRID_HW * kHWPairs];
     const int vid_lo = a.tok0 < a.nv ? a.tok0 : a.nv;

@@ -5,9 +5,9 @@
 // and each query token of the current segment, softmax attention over the
 // visible cached tokens of earlier segments followed by every token of the
 // current segment (no mask inside a segment; causality across segments is
-// structural: later segments are never in the cache). INT8 caches are
-// dequantised to BF16 in shared memory (model card, "Single-GPU Low-Memory
-// Inference": INT8 KV storage, BF16 attention computation).
+// structural: later segments are never in the cache). An INT8 cache is
+// converted to BF16 in shared memory tile by tile (model card, "Single-GPU
+// Low-Memory Inference": INT8 KV storage, BF16 attention computation).
 //
 // Structure of one CTA (one "unit" = two 128-row Q tiles of one head, and a
 // contiguous range of 128-key KV tiles: cache tiles first, then the current
@@ -17,22 +17,26 @@
 //   warp 1      TMEM allocator + tcgen05.mma issuer
 //   warps 4-7   softmax warpgroup for Q tile 0 (one thread per query row)
 //   warps 8-11  softmax warpgroup for Q tile 1
-//   warps 12-15 INT8 caches only: the one filler of the K/V ring -- cache
-//               tiles are dequantised (codes + scales from global memory ->
-//               BF16 in the 128B-swizzled stage layout), current-segment tiles
-//               are loaded by TMA. One filler in tile order keeps every parity
-//               wait on the ring exact.
+//   warps 12-15 INT8 caches only: the one filler of the K/V ring. Cache K
+//               tiles hold the INT8 codes themselves as BF16 (exact for
+//               |code| <= 127) and the per-key K scale goes to the softmax as
+//               a per-column coefficient; cache V tiles hold code * scale
+//               rounded to BF16. Current-segment tiles are loaded by TMA. One
+//               filler in tile order keeps every parity wait on the ring exact.
 // TMEM (512 columns): S0 | S1 | O0 | O1, 128 fp32 columns each; the BF16
 // probabilities P overwrite the first 64 columns of their S block and feed
 // the P.V product straight from TMEM (A operand in tensor memory).
 // MMA order per KV tile j: PV0(j-1) S0(j) | PV1(j-1) S1(j) -- while one
 // softmax warpgroup exponentiates, the tensor core works for the other. The
 // issuer waits for V(j-1) before PV0(j-1) and for K(j) only before S0(j).
-// Online softmax in base 2 with lazy rescaling: the running reference max is
-// raised only when a tile's max exceeds it by more than 8 (so P <= 256), and
-// only then is O rescaled in TMEM.
+// Softmax: a thread reads its whole 128-column S row from TMEM into registers
+// once, takes the row maximum there and exponentiates from registers. Online
+// softmax in base 2 with lazy rescaling: the running reference max is raised
+// only when a tile's max exceeds it by more than 8 (so P <= 256), and only
+// then is O rescaled in TMEM.
 // Split-KV: with splits > 1 each CTA leaves (O unnormalised, max, sum) in the
-// workspace and combine_kernel merges them.
+// workspace and counts itself in per unit; the last CTA of a unit to arrive
+// merges the splits and writes the output (the partials are still in L2).
 #include "nomas_internal.h"
 #include "nomas_ptx.cuh"
 
@@ -45,15 +49,18 @@ namespace {
 constexpr int BM = 128;
 constexpr int BN = 128;
 constexpr int kStages = 2;
-constexpr uint32_t kTileBytes = BM * kD * 2; // one BF16 128x128 tile
+constexpr int kCoefSlots = 4;                 // ring of per-tile K coefficients (INT8 caches)
+constexpr uint32_t kTileBytes = BM * kD * 2;  // one BF16 128x128 tile
 constexpr uint32_t kHalfBytes = kTileBytes / 2;
-constexpr float kRescaleThreshold = 8.0f; // P <= 2^8 between rescales
+constexpr float kRescaleThreshold = 8.0f;     // P <= 2^8 between rescales
 
 // shared memory map (offsets from a 1024-byte aligned base)
 constexpr uint32_t kOffQ = 0;                                // 2 tiles
 constexpr uint32_t kOffK = kOffQ + 2 * kTileBytes;           // kStages tiles
 constexpr uint32_t kOffV = kOffK + kStages * kTileBytes;     // kStages tiles
-constexpr uint32_t kOffBar = kOffV + kStages * kTileBytes;   // barriers
+constexpr uint32_t kOffCoef = kOffV + kStages * kTileBytes;  // kCoefSlots x 128 fp32
+constexpr uint32_t kOffBound = kOffCoef + kCoefSlots * BN * 4; // kCoefSlots x 4 warps x (max, min)
+constexpr uint32_t kOffBar = kOffBound + kCoefSlots * 4 * 8; // barriers
 constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;        // + alignment slack
 
 // barrier slots (8 bytes each)
@@ -67,12 +74,26 @@ enum {
     B_PFULL = B_SFULL + 2,
     B_OFULL = B_PFULL + 2,
     B_DRAIN = B_OFULL + 2,
-    B_COUNT
+    B_CFULL = B_DRAIN + 1,          // + coefficient slot: the filler wrote a tile's K coefficients
+    B_CEMPTY = B_CFULL + kCoefSlots, // + coefficient slot: every softmax warp is done with them
+    B_COUNT = B_CEMPTY + kCoefSlots
 };
 constexpr uint32_t kOffTmemSlot = B_COUNT * 8;
 constexpr uint32_t kOffAbort = kOffTmemSlot + 8;
 constexpr uint32_t kOffDqGo = kOffAbort + 4;
-static_assert(kOffDqGo + 4 <= 256, "barrier area overflow");
+constexpr uint32_t kOffLast = kOffDqGo + 4;
+static_assert(kOffLast + 4 <= 256, "barrier area overflow");
+static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+
+// Register budgets per warpgroup (setmaxnreg). The CTA is launched with the
+// registers the compiler reports for the kernel (BF16: 384 threads x 168 =
+// 64,512; INT8: 512 x 128 = 65,536); the budgets add up to exactly that:
+// BF16 128 x 72 + 256 x 216; INT8 128 x 64 + 256 x 176 + 128 x 96.
+template <bool kInt8> struct Regs;
+template <> struct Regs<false> { static constexpr uint32_t kCtl = 72, kSoftmax = 216, kFiller = 0; };
+template <> struct Regs<true> { static constexpr uint32_t kCtl = 64, kSoftmax = 176, kFiller = 96; };
+static_assert(128 * 72 + 256 * 216 == 384 * 168, "BF16 register split");
+static_assert(128 * 64 + 256 * 176 + 128 * 96 == 512 * 128, "INT8 register split");
 
 // mbar_wait run by every lane of a converged warp; lane 0's outcome is
 // broadcast so the warp leaves the wait converged.
@@ -124,13 +145,15 @@ __host__ __device__ constexpr uint64_t kstep_kmajor(int kk) {
 }
 __host__ __device__ constexpr uint64_t kstep_mnmajor(int kk) { return static_cast<uint64_t>((kk * 2048) >> 4); }
 
-// 8 INT8 codes -> 8 BF16 values code * scale. A code c is read exactly as the
-// float 2^23 + (c + 128) (the byte of c ^ 0x80 placed under the exponent of 2^23),
-// minus 2^23 + 128, then scaled in fp32 and rounded once to BF16.
-__device__ __forceinline__ uint4 dequant8(uint2 w, float scale) {
+// 8 INT8 codes -> 8 BF16 values. A code c is read exactly as the float
+// 2^23 + (c + 128) (the byte of c ^ 0x80 placed under the exponent of 2^23),
+// minus 2^23 + 128. kScale: times the row scale in fp32, then rounded once to
+// BF16; otherwise the integer itself, which BF16 holds exactly (at most 7
+// significant bits), so its fp32 pattern's upper half is the BF16 pattern.
+template <bool kScale>
+__device__ __forceinline__ uint4 codes_to_bf16(uint2 w, float scale) {
     const uint32_t w0 = w.x ^ 0x80808080u, w1 = w.y ^ 0x80808080u;
     const float2 bias = make_float2(-8388736.0f, -8388736.0f);
-    const float2 sc = make_float2(scale, scale);
     uint32_t out[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
@@ -138,8 +161,13 @@ __device__ __forceinline__ uint4 dequant8(uint2 w, float scale) {
         const uint32_t b = (q & 1) * 2;
         float2 f = make_float2(__uint_as_float(__byte_perm(src, 0x4B000000u, 0x7540u + b)),
                                __uint_as_float(__byte_perm(src, 0x4B000000u, 0x7541u + b)));
-        f = __fmul2_rn(__fadd2_rn(f, bias), sc);
-        out[q] = pack_bf16x2(f.x, f.y);
+        f = __fadd2_rn(f, bias);
+        if (kScale) {
+            f = __fmul2_rn(f, make_float2(scale, scale));
+            out[q] = pack_bf16x2(f.x, f.y);
+        } else {
+            out[q] = __byte_perm(__float_as_uint(f.x), __float_as_uint(f.y), 0x7632u);
+        }
     }
     return make_uint4(out[0], out[1], out[2], out[3]);
 }
@@ -160,34 +188,25 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
     return r;
 }
 
-// Maximum of one 128-key S row over its valid columns (kMask: columns >= vc
-// ignored). Eight independent accumulators keep the reduction off a single
-// dependency chain.
-template <bool kMask>
-__device__ __forceinline__ float row_max(uint32_t t_s, int vc) {
-    float mx = -INFINITY;
+// Maximum of 64 raw scores held in registers; eight independent accumulators
+// keep the reduction off a single dependency chain.
+__device__ __forceinline__ float max64(const uint32_t* s, float init) {
+    float m[8];
 #pragma unroll
-    for (int c = 0; c < 2; ++c) {
-        uint32_t s[64];
-        tmem_ld64(t_s + c * 64, s);
-        float m[8];
+    for (int k = 0; k < 8; ++k) m[k] = init;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) m[k] = mx;
+    for (int e = 0; e < 64; e += 2)
+        m[(e >> 1) & 7] = max3(m[(e >> 1) & 7], __uint_as_float(s[e]), __uint_as_float(s[e + 1]));
+    return max3(max3(m[0], m[1], m[2]), max3(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
+}
+
+// Columns [c0, c0 + 64) at or beyond vc of a ragged tile: score -inf, so they
+// are ignored by the maximum and their probability is 2^-inf = 0 (or 2^-125 on
+// the FMA-pipe path, against V rows that are zero: both the TMA boxes and the
+// INT8 filler fill keys past the end with zeros).
+__device__ __forceinline__ void mask64(uint32_t* s, int c0, int vc) {
 #pragma unroll
-        for (int e = 0; e < 64; e += 2) {
-            float x0 = __uint_as_float(s[e]), x1 = __uint_as_float(s[e + 1]);
-            if (kMask) {
-                x0 = (c * 64 + e < vc) ? x0 : -INFINITY;
-                x1 = (c * 64 + e + 1 < vc) ? x1 : -INFINITY;
-            }
-            m[(e >> 1) & 7] = max3(m[(e >> 1) & 7], x0, x1);
-        }
-        mx = max3(max3(m[0], m[1], m[2]), max3(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
-        // keep this chunk's reduction ahead of the next TMEM load, so its 64
-        // registers are dead before the next 64 arrive
-        asm volatile("" : "+f"(mx));
-    }
-    return mx;
+    for (int e = 0; e < 64; ++e) s[e] = (c0 + e < vc) ? s[e] : 0xFF800000u;
 }
 
 // 2^x of two values on the FMA pipe, so that part of a row's exponentials
@@ -196,9 +215,9 @@ __device__ __forceinline__ float row_max(uint32_t t_s, int vc) {
 // (the 1.5 * 2^23 shift puts n in the low mantissa bits of t) and f in
 // [-1/2, 1/2]; 2^f by a cubic whose coefficients minimise the maximum relative
 // error on that interval (7.5e-5, well under the 2^-9 of the BF16 rounding of P
-// that follows; fitted by exp2_poly_fit.py beside this file); 2^n by adding n
-// to the exponent field (the shift by 23 keeps exactly the low 9 bits of t,
-// i.e. n modulo 2^9). x is clamped below at -125 so the result stays normal
+// that follows; fitted by tests/tools/exp2_poly_fit.py); 2^n by adding n to
+// the exponent field (the shift by 23 keeps exactly the low 9 bits of t, i.e.
+// n modulo 2^9). x is clamped below at -125 so the result stays normal
 // (2^-125 in place of a smaller P, far under the BF16 resolution of the row).
 constexpr float kExp2C0 = 0.9999280571937561f;
 constexpr float kExp2C1 = 0.6932608485221863f;
@@ -217,85 +236,41 @@ __device__ __forceinline__ float2 exp2_fma2(float2 x) {
                        __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
 }
 
-// Of every 8 column pairs of a full tile, kPoly take exp2_fma2 and the rest
-// the MUFU ex2. With an INT8 cache the dequantising warps share the FMA pipe
-// and issue slots of every SM sub-partition, so that kernel keeps all of them
-// on the MUFU.
+// Of every 8 column pairs, kPoly take exp2_fma2 and the rest the MUFU ex2.
+// With an INT8 cache the converting warps share the FMA pipe and the issue
+// slots of every SM sub-partition, so fewer go to the FMA pipe there.
 constexpr int kExp2PolyPairsBf16 = 3;
-constexpr int kExp2PolyPairsInt8 = 0;
+constexpr int kExp2PolyPairsInt8 = 2;
 
-// One 32-column chunk of an unmasked S row -> 16 packed BF16 P columns.
-template <int kPoly>
-__device__ __forceinline__ void exp_chunk(const uint32_t (&s)[32], float2 sl2x2, float2 negm, float2 (&acc)[4],
-                                          uint32_t (&p)[16]) {
-#pragma unroll
-    for (int e = 0; e < 16; ++e) {
-        const float2 x = __ffma2_rn(make_float2(__uint_as_float(s[2 * e]), __uint_as_float(s[2 * e + 1])), sl2x2, negm);
-        float2 y;
-        if ((e & 7) < kPoly)
-            y = exp2_fma2(x);
-        else
-            y = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-        acc[e & 3] = __fadd2_rn(acc[e & 3], y);
-        p[e] = pack_bf16x2(y.x, y.y);
-    }
-}
-
-// P = 2^(s * scale_log2 - m) of one full 128-key S row, written as packed BF16
-// pairs over the first 64 columns of the row's S block; returns the fp32 row
-// sum (four independent packed accumulators). The TMEM loads are software
-// pipelined: chunk c + 1 is in flight while chunk c is exponentiated. P chunk c
-// lands on columns [16c, 16c + 16), all of which were read with chunks <= c.
-template <int kPoly>
-__device__ __forceinline__ float row_exp_store_full(uint32_t t_s, float sl2, float m) {
-    const float2 sl2x2 = make_float2(sl2, sl2);
+// P = 2^(s * c - m) of one 128-key S row held in registers, written as packed
+// BF16 pairs over the first 64 columns of the row's S block (all of S is in
+// registers by then); returns the fp32 row sum. c is the scalar scale_log2, or
+// with kCoef the per-column coefficients of the tile (scale_log2 times the
+// key's K scale) read from shared memory four at a time.
+template <int kPoly, bool kCoef>
+__device__ __forceinline__ float exp_row(const uint32_t (&s)[128], const float4* coef, float sl2, float m,
+                                         uint32_t t_s) {
     const float2 negm = make_float2(-m, -m);
     float2 acc[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) acc[k] = make_float2(0.0f, 0.0f);
-    uint32_t sa[32], sb[32], p[16];
-    tmem_ld32_issue(t_s, sa);
-    tmem_ld32_wait(sa);
-    tmem_ld32_issue(t_s + 32, sb);
-    exp_chunk<kPoly>(sa, sl2x2, negm, acc, p);
-    tmem_st16(t_s, p);
-    tmem_ld32_wait(sb);
-    tmem_ld32_issue(t_s + 64, sa);
-    exp_chunk<kPoly>(sb, sl2x2, negm, acc, p);
-    tmem_st16(t_s + 16, p);
-    tmem_ld32_wait(sa);
-    tmem_ld32_issue(t_s + 96, sb);
-    exp_chunk<kPoly>(sa, sl2x2, negm, acc, p);
-    tmem_st16(t_s + 32, p);
-    tmem_ld32_wait(sb);
-    exp_chunk<kPoly>(sb, sl2x2, negm, acc, p);
-    tmem_st16(t_s + 48, p);
-    const float2 t = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
-    return t.x + t.y;
-}
-
-// Masked form for a ragged last tile (columns >= vc get P = 0): MUFU only,
-// one 32-column chunk at a time.
-__device__ __forceinline__ float row_exp_store_masked_impl(uint32_t t_s, float sl2, float m, int vc) {
-    const float2 sl2x2 = make_float2(sl2, sl2);
-    const float2 negm = make_float2(-m, -m);
-    float2 acc[4];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) acc[k] = make_float2(0.0f, 0.0f);
-#pragma unroll 1
     for (int c = 0; c < 4; ++c) {
-        uint32_t s[32];
-        tmem_ld32(t_s + c * 32, s);
         uint32_t p[16];
+        float4 c4 = make_float4(sl2, sl2, sl2, sl2);
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-            float2 x = __ffma2_rn(make_float2(__uint_as_float(s[2 * e]), __uint_as_float(s[2 * e + 1])), sl2x2, negm);
             const int col = c * 32 + 2 * e;
-            x.x = col < vc ? x.x : -INFINITY;
-            x.y = col + 1 < vc ? x.y : -INFINITY;
-            const float p0 = ex2_approx(x.x), p1 = ex2_approx(x.y);
-            acc[e & 3] = __fadd2_rn(acc[e & 3], make_float2(p0, p1));
-            p[e] = pack_bf16x2(p0, p1);
+            if (kCoef && (e & 1) == 0) c4 = coef[col >> 2];
+            const float2 cc = (e & 1) ? make_float2(c4.z, c4.w) : make_float2(c4.x, c4.y);
+            const float2 x = __ffma2_rn(make_float2(__uint_as_float(s[col]), __uint_as_float(s[col + 1])), cc, negm);
+            float2 y;
+            if ((e & 7) < kPoly)
+                y = exp2_fma2(x);
+            else
+                y = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+            acc[e & 3] = __fadd2_rn(acc[e & 3], y);
+            p[e] = pack_bf16x2(y.x, y.y);
         }
         tmem_st16(t_s + c * 16, p);
     }
@@ -303,15 +278,22 @@ __device__ __forceinline__ float row_exp_store_masked_impl(uint32_t t_s, float s
     return t.x + t.y;
 }
 
-// Cold paths kept out of line, so they do not add to the register pressure of
-// the per-tile loop: tail tiles (masked), O rescaling, the epilogues.
-__device__ __noinline__ float row_max_masked(uint32_t t_s, int vc) { return row_max<true>(t_s, vc); }
-__device__ __noinline__ float row_exp_store_masked(uint32_t t_s, float sl2, float m, int vc) {
-    return row_exp_store_masked_impl(t_s, sl2, m, vc);
+// Exact maximum of s_j * c_j over a row (used when the cheap bound of a tile
+// is too loose to serve as the reference: keys of very different scales).
+__device__ __forceinline__ float max_scaled(const uint32_t (&s)[128], const float4* coef) {
+    float m0 = -INFINITY, m1 = -INFINITY;
+#pragma unroll
+    for (int k = 0; k < 32; ++k) {
+        const float4 c = coef[k];
+        m0 = max3(m0, __uint_as_float(s[4 * k]) * c.x, __uint_as_float(s[4 * k + 1]) * c.y);
+        m1 = max3(m1, __uint_as_float(s[4 * k + 2]) * c.z, __uint_as_float(s[4 * k + 3]) * c.w);
+    }
+    return fmaxf(m0, m1);
 }
 
-// O *= alpha for one row (one thread), in TMEM.
-__device__ __noinline__ void rescale_o(uint32_t t_o, float alpha) {
+// O *= alpha for one row (one thread), in TMEM. Inline: it runs while the
+// thread's S row is held in registers, which a call would have to preserve.
+__device__ __forceinline__ void rescale_o(uint32_t t_o, float alpha) {
 #pragma unroll 1
     for (int c = 0; c < 4; ++c) {
         uint32_t o[32];
@@ -322,6 +304,9 @@ __device__ __noinline__ void rescale_o(uint32_t t_o, float alpha) {
         tmem_st_wait();
     }
 }
+
+// Cold paths kept out of line, so they do not add to the register pressure of
+// the per-tile loop: the epilogues.
 
 // Final output row: O / l -> BF16 (all lanes load from TMEM; only valid rows store).
 __device__ __noinline__ void store_out_row(uint32_t t_o, float inv_l, uint16_t* dst, bool row_ok) {
@@ -343,18 +328,54 @@ __device__ __noinline__ void store_out_row(uint32_t t_o, float inv_l, uint16_t* 
     }
 }
 
-// Partial row: unnormalised fp32 O.
-__device__ __noinline__ void store_partial_row(uint32_t t_o, float* dst, bool row_ok) {
+// Partial row of one split: unnormalised fp32 O, 4 dims per float4, laid out
+// [32 chunks][256 rows] so that consecutive rows (threads) touch consecutive
+// 16-byte words.
+__device__ __noinline__ void store_partial_row(uint32_t t_o, float4* dst) {
 #pragma unroll 1
     for (int c = 0; c < 4; ++c) {
         uint32_t o[32];
         tmem_ld32(t_o + c * 32, o);
-        if (row_ok) {
-            uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) d4[e] = make_uint4(o[4 * e], o[4 * e + 1], o[4 * e + 2], o[4 * e + 3]);
-        }
+        for (int e = 0; e < 8; ++e)
+            dst[(c * 8 + e) * 256] = make_float4(__uint_as_float(o[4 * e]), __uint_as_float(o[4 * e + 1]),
+                                                 __uint_as_float(o[4 * e + 2]), __uint_as_float(o[4 * e + 3]));
     }
+}
+
+// Merge of the splits of one row (run by the last CTA of a unit to arrive):
+// O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s with M = max_s m_s.
+__device__ __noinline__ void merge_row(const AttnArgs& a, int unit, int row, uint16_t* dst, float* lse_dst) {
+    const int units = a.heads * a.pairs;
+    float mmax = -INFINITY;
+    for (int s = 0; s < a.splits; ++s)
+        mmax = fmaxf(mmax, __ldcg(&a.part_ml[(static_cast<int64_t>(s) * units + unit) * 256 + row]).x);
+    float L = 0.0f;
+    float wgt[8];
+    for (int s = 0; s < a.splits; ++s) {
+        const float2 ml = __ldcg(&a.part_ml[(static_cast<int64_t>(s) * units + unit) * 256 + row]);
+        const float g = exp2f(ml.x - mmax);
+        if (s < 8) wgt[s] = g;
+        L += ml.y * g;
+    }
+    const float inv = 1.0f / L;
+#pragma unroll 1
+    for (int c = 0; c < 32; c += 2) {
+        float4 acc0 = make_float4(0.f, 0.f, 0.f, 0.f), acc1 = acc0;
+        for (int s = 0; s < a.splits; ++s) {
+            const float g = s < 8 ? wgt[s]
+                                  : exp2f(__ldcg(&a.part_ml[(static_cast<int64_t>(s) * units + unit) * 256 + row]).x -
+                                          mmax);
+            const float4* base = a.part_o + (static_cast<int64_t>(s) * units + unit) * 32 * 256 + row;
+            const float4 o0 = __ldcg(base + c * 256), o1 = __ldcg(base + (c + 1) * 256);
+            acc0.x += o0.x * g; acc0.y += o0.y * g; acc0.z += o0.z * g; acc0.w += o0.w * g;
+            acc1.x += o1.x * g; acc1.y += o1.y * g; acc1.z += o1.z * g; acc1.w += o1.w * g;
+        }
+        reinterpret_cast<uint4*>(dst)[c >> 1] =
+            make_uint4(pack_bf16x2(acc0.x * inv, acc0.y * inv), pack_bf16x2(acc0.z * inv, acc0.w * inv),
+                       pack_bf16x2(acc1.x * inv, acc1.y * inv), pack_bf16x2(acc1.z * inv, acc1.w * inv));
+    }
+    if (lse_dst) *lse_dst = (mmax + log2f(L)) * 0.69314718055994531f;
 }
 
 // Arm a K (or V) stage for tile t and issue its two TMA boxes.
@@ -410,6 +431,7 @@ __global__ void __launch_bounds__(kInt8 ? 512 : 384, 1)
     volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + kOffBar + kOffTmemSlot);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffBar + kOffAbort);
     volatile int* dq_go = reinterpret_cast<volatile int*>(smem + kOffBar + kOffDqGo);
+    volatile int* last_flag = reinterpret_cast<volatile int*>(smem + kOffBar + kOffLast);
     const WaitCtl ctl{abort_flag, a.err};
 
     const int warp = threadIdx.x >> 5;
@@ -422,11 +444,14 @@ __global__ void __launch_bounds__(kInt8 ? 512 : 384, 1)
     const int pair = unit % a.pairs;
     const int qt0 = 2 * pair;
     const bool has_q1 = (qt0 + 1) < a.tiles_q;
+    const int nq_tiles = has_q1 ? 2 : 1;
     const int t_total = a.tiles_c + a.tiles_q;
     const int t_begin = split * a.tiles_per_split;
     int t_end = t_begin + a.tiles_per_split;
     if (t_end > t_total) t_end = t_total;
     const int n = t_end - t_begin; // >= 1 by construction of the split count
+    // cache tiles of this CTA come first: i < nci (INT8 caches: converted by the filler)
+    const int nci = kInt8 ? max(0, min(t_end, a.tiles_c) - t_begin) : 0;
 
     // ---- setup
     if (threadIdx.x == 0) {
@@ -443,6 +468,10 @@ __global__ void __launch_bounds__(kInt8 ? 512 : 384, 1)
             mbar_init(bar(B_OFULL + w), 1);
         }
         mbar_init(bar(B_DRAIN), 1);
+        for (int c = 0; c < kCoefSlots; ++c) {
+            mbar_init(bar(B_CFULL + c), 1);
+            mbar_init(bar(B_CEMPTY + c), 4 * nq_tiles); // one arrival per active softmax warp
+        }
         *abort_flag = 0;
         fence_barrier_init();
         fence_proxy_async_smem();
@@ -459,7 +488,14 @@ __global__ void __launch_bounds__(kInt8 ? 512 : 384, 1)
     // are set up while it finishes; nothing it wrote is read before this point
     grid_dep_wait();
 
-    if (warp == 0) {
+    // Roles by warpgroup. Each warpgroup first sets its register budget (one
+    // setmaxnreg for its four warps, at the top of its own branch, so that
+    // the compiler allocates each role's code under that role's budget): the
+    // control warpgroup and the filler give registers back, the softmax
+    // warpgroups take them.
+    if (warp < 4) {
+        regs_dec<Regs<kInt8>::kCtl>();
+        if (warp == 0) {
         // ================================================================ producer
         if (lane == 0) {
             tma_prefetch_desc(&tm_q);
@@ -469,13 +505,13 @@ __global__ void __launch_bounds__(kInt8 ? 512 : 384, 1)
                 tma_prefetch_desc(&tm_kc);
                 tma_prefetch_desc(&tm_vc);
             }
-            mbar_arrive_expect_tx(bar(B_QFULL), (has_q1 ? 2u : 1u) * kTileBytes);
-            for (int w = 0; w < (has_q1 ? 2 : 1); ++w) {
+            mbar_arrive_expect_tx(bar(B_QFULL), static_cast<uint32_t>(nq_tiles) * kTileBytes);
+            for (int w = 0; w < nq_tiles; ++w) {
                 const uint32_t dst = sbase + kOffQ + w * kTileBytes;
                 tma_load_3d(dst, &tm_q, 0, (qt0 + w) * BM, head, bar(B_QFULL));
                 tma_load_3d(dst + kHalfBytes, &tm_q, 64, (qt0 + w) * BM, head, bar(B_QFULL));
             }
-            // An INT8 cache has one filler for every stage, the dequantiser warpgroup
+            // An INT8 cache has one filler for every stage, the converting warpgroup
             // (codes for cache tiles, TMA for current-segment tiles): with a single
             // filler in tile order every parity wait on the stage ring is exact.
             if (!kInt8) {
@@ -495,122 +531,151 @@ __global__ void __launch_bounds__(kInt8 ? 512 : 384, 1)
                 drain_armed(k_armed, v_armed, bar(B_KFULL), bar(B_VFULL));
             }
         }
-    } else if (warp == 1) {
+        } else if (warp == 1) {
         // ================================================================ MMA issuer
-        // BF16 caches: the whole warp runs the loop (warp-uniform waits and
-        // conditions) and one elected lane issues each MMA and commit; MMAs issued
-        // by a single lane in a divergent branch run at little more than half the
-        // tensor-core rate whenever a branch separates two groups of them. With
-        // an INT8 cache the filler warps are the bottleneck and the warp-wide
-        // polling only takes issue slots from them, so lane 0 issues alone.
-        constexpr bool kWarpIssue = !kInt8;
-        if (kWarpIssue || lane == 0) {
-            using I = Issuer<kWarpIssue>;
-            constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, BN, false, false);
-            constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, kD, false, true);
-            const uint32_t q_tile[2] = {sbase + kOffQ, sbase + kOffQ + kTileBytes};
-            // TMEM columns: S of Q tile w at 128 w, O of Q tile w at 256 + 128 w
-            auto tm_s = [&](int w) { return tmem + 128u * static_cast<uint32_t>(w); };
-            auto tm_o = [&](int w) { return tmem + 256u + 128u * static_cast<uint32_t>(w); };
-            const int nq_tiles = has_q1 ? 2 : 1;
-            bool ok = I::wait(bar(B_QFULL), 0, ctl);
+        // The whole warp runs the loop (warp-uniform waits and conditions) and
+        // one elected lane issues each MMA and commit; MMAs issued by a single
+        // lane in a divergent branch run at little more than half the
+        // tensor-core rate whenever a branch separates two groups of them.
+        using I = Issuer<true>;
+        constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, BN, false, false);
+        constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, kD, false, true);
+        // TMEM columns: S of Q tile w at 128 w, O of Q tile w at 256 + 128 w
+        auto tm_s = [&](int w) { return tmem + 128u * static_cast<uint32_t>(w); };
+        auto tm_o = [&](int w) { return tmem + 256u + 128u * static_cast<uint32_t>(w); };
+        bool ok = I::wait(bar(B_QFULL), 0, ctl);
+        tc_fence_after();
+        // k-step-0 descriptors of the Q tiles and of the K and V stages (scalars:
+        // selected, not indexed, so they stay in registers)
+        static_assert(kStages == 2, "the stage descriptors below assume two stages");
+        const uint64_t q_desc0 = desc_kmajor(sbase + kOffQ, 0), q_desc1 = desc_kmajor(sbase + kOffQ + kTileBytes, 0);
+        const uint64_t k_desc0 = desc_kmajor(sbase + kOffK, 0), k_desc1 = desc_kmajor(sbase + kOffK + kTileBytes, 0);
+        const uint64_t v_desc0 = desc_mnmajor(sbase + kOffV, 0);
+        const uint64_t v_desc1 = desc_mnmajor(sbase + kOffV + kTileBytes, 0);
+        auto issue_s = [&](int w, int st) {
+            const uint64_t qd = w ? q_desc1 : q_desc0, kd = st ? k_desc1 : k_desc0;
+#pragma unroll
+            for (int kk = 0; kk < kD / 16; ++kk)
+                I::ss(tm_s(w), qd + kstep_kmajor(kk), kd + kstep_kmajor(kk), idesc_qk, kk > 0 ? 1u : 0u);
+        };
+        auto issue_pv = [&](int w, int st, bool first_tile) {
+            const uint64_t vd = st ? v_desc1 : v_desc0;
+#pragma unroll
+            for (int kk = 0; kk < BN / 16; ++kk)
+                I::ts(tm_o(w), tm_s(w) + kk * 8, vd + kstep_mnmajor(kk), idesc_pv, (first_tile && kk == 0) ? 0u : 1u);
+        };
+        if (ok) ok = I::wait(bar(B_KFULL + 0), 0, ctl);
+        if (ok) {
             tc_fence_after();
-            // k-step-0 descriptors of the Q tiles and of the K and V stages (scalars:
-            // selected, not indexed, so they stay in registers)
-            static_assert(kStages == 2, "the stage descriptors below assume two stages");
-            const uint64_t q_desc0 = desc_kmajor(q_tile[0], 0), q_desc1 = desc_kmajor(q_tile[1], 0);
-            const uint64_t k_desc0 = desc_kmajor(sbase + kOffK, 0), k_desc1 = desc_kmajor(sbase + kOffK + kTileBytes, 0);
-            const uint64_t v_desc0 = desc_mnmajor(sbase + kOffV, 0);
-            const uint64_t v_desc1 = desc_mnmajor(sbase + kOffV + kTileBytes, 0);
-            auto issue_s = [&](int w, int st) {
-                const uint64_t qd = w ? q_desc1 : q_desc0, kd = st ? k_desc1 : k_desc0;
-#pragma unroll
-                for (int kk = 0; kk < kD / 16; ++kk)
-                    I::ss(tm_s(w), qd + kstep_kmajor(kk), kd + kstep_kmajor(kk), idesc_qk, kk > 0 ? 1u : 0u);
-            };
-            auto issue_pv = [&](int w, int st, bool first_tile) {
-                const uint64_t vd = st ? v_desc1 : v_desc0;
-#pragma unroll
-                for (int kk = 0; kk < BN / 16; ++kk)
-                    I::ts(tm_o(w), tm_s(w) + kk * 8, vd + kstep_mnmajor(kk), idesc_pv,
-                           (first_tile && kk == 0) ? 0u : 1u);
-            };
-            if (ok) ok = I::wait(bar(B_KFULL + 0), 0, ctl);
-            if (ok) {
+            for (int w = 0; w < nq_tiles; ++w) {
+                issue_s(w, 0);
+                I::commit(bar(B_SFULL + w));
+            }
+            // K of tile 0 is free once these S MMAs finish (a fill of tile 2 waits for it)
+            if (kStages < n) I::commit(bar(B_KEMPTY + 0));
+        }
+        for (int i = 0; ok && i < n; ++i) {
+            const int st = i % kStages;
+            const uint32_t ph = (i / kStages) & 1;
+            const int st1 = (i + 1) % kStages;
+            const uint32_t ph1 = ((i + 1) / kStages) & 1;
+            const bool last = (i + 1 == n);
+            if (!(ok = I::wait(bar(B_VFULL + st), ph, ctl))) break;
+            for (int w = 0; w < nq_tiles; ++w) {
+                if (!(ok = I::wait(bar(B_PFULL + w), i & 1, ctl))) break;
                 tc_fence_after();
-                for (int w = 0; w < nq_tiles; ++w) {
-                    issue_s(w, 0);
-                    I::commit(bar(B_SFULL + w));
-                }
-                // K of tile 0 is free once these S MMAs finish (a fill of tile 2 waits for it)
-                if (kStages < n) I::commit(bar(B_KEMPTY + 0));
-            }
-            for (int i = 0; ok && i < n; ++i) {
-                const int st = i % kStages;
-                const uint32_t ph = (i / kStages) & 1;
-                const int st1 = (i + 1) % kStages;
-                const uint32_t ph1 = ((i + 1) / kStages) & 1;
-                const bool last = (i + 1 == n);
-                if (!(ok = I::wait(bar(B_VFULL + st), ph, ctl))) break;
-                for (int w = 0; w < nq_tiles; ++w) {
-                    if (!(ok = I::wait(bar(B_PFULL + w), i & 1, ctl))) break;
-                    tc_fence_after();
-                    issue_pv(w, st, i == 0);
-                    // each release is committed only when a later fill waits for it,
-                    // so no arrival is left pending at exit
-                    if (w == nq_tiles - 1 && i + kStages < n) I::commit(bar(B_VEMPTY + st));
-                    if (!last) {
-                        // K of tile i + 1 is needed from here on only: P.V of Q tile 0
-                        // never waits for it
-                        if (w == 0) {
-                            if (!(ok = I::wait(bar(B_KFULL + st1), ph1, ctl))) break;
-                            tc_fence_after();
-                        }
-                        issue_s(w, st1);
-                        I::commit(bar(B_SFULL + w));
-                        if (w == nq_tiles - 1 && i + 1 + kStages < n) I::commit(bar(B_KEMPTY + st1));
-                    } else {
-                        I::commit(bar(B_OFULL + w));
+                issue_pv(w, st, i == 0);
+                // each release is committed only when a later fill waits for it,
+                // so no arrival is left pending at exit
+                if (w == nq_tiles - 1 && i + kStages < n) I::commit(bar(B_VEMPTY + st));
+                if (!last) {
+                    // K of tile i + 1 is needed from here on only: P.V of Q tile 0
+                    // never waits for it
+                    if (w == 0) {
+                        if (!(ok = I::wait(bar(B_KFULL + st1), ph1, ctl))) break;
+                        tc_fence_after();
                     }
+                    issue_s(w, st1);
+                    I::commit(bar(B_SFULL + w));
+                    if (w == nq_tiles - 1 && i + 1 + kStages < n) I::commit(bar(B_KEMPTY + st1));
+                } else {
+                    I::commit(bar(B_OFULL + w));
                 }
-            }
-            // drain: every MMA issued above has completed before teardown
-            I::commit(bar(B_DRAIN));
-            const uint64_t t0 = global_timer_ns();
-            while (!mbar_try_wait(bar(B_DRAIN), 0)) {
-                if (global_timer_ns() - t0 > NOMAS_WAIT_NS) break;
             }
         }
-    } else if (warp >= 4 && warp < 12) {
+        // drain: every MMA issued above has completed before teardown
+        I::commit(bar(B_DRAIN));
+        const uint64_t t0 = global_timer_ns();
+        while (!mbar_try_wait(bar(B_DRAIN), 0)) {
+            if (global_timer_ns() - t0 > NOMAS_WAIT_NS) break;
+        }
+        }
+    } else if (warp < 12) {
+        regs_inc<Regs<kInt8>::kSoftmax>();
         // ================================================================ softmax
         const int w = (warp - 4) >> 2;
         const int quad = warp & 3;
         const int r = quad * 32 + lane; // row inside the Q tile
-        if (w == 0 || has_q1) {
-            const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-            const uint32_t t_s = tmem + lane_off + w * 128;
-            const uint32_t t_o = tmem + lane_off + 256 + w * 128;
+        const bool active = (w == 0 || has_q1);
+        const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+        const uint32_t t_s = tmem + lane_off + w * 128;
+        const uint32_t t_o = tmem + lane_off + 256 + w * 128;
+        float m_ref = -INFINITY; // reference max, log2 units
+        float l = 0.0f;
+        bool ok = true;
+        if (active) {
             const float sl2 = a.scale_log2;
-            float m_ref = -INFINITY; // reference max, log2 units
-            float l = 0.0f;
-            bool ok = true;
             for (int i = 0; i < n; ++i) {
+                const int t = t_begin + i;
+                const bool coef = kInt8 && i < nci; // warp-uniform
+                const uint32_t slot = static_cast<uint32_t>(i % kCoefSlots);
                 if (!(ok = mbar_wait(bar(B_SFULL + w), i & 1, ctl))) break;
                 tc_fence_after();
-                const int vc = tile_valid(a, t_begin + i);
-                const bool full = (vc == BN);
-                // pass 1: tile max; the reference max moves only when it is exceeded
-                // by more than the threshold (then O is rescaled in TMEM)
-                const float mxl = (full ? row_max<false>(t_s, vc) : row_max_masked(t_s, vc)) * sl2;
-                const bool resc = mxl > m_ref + kRescaleThreshold;
-                const float m_new = resc ? mxl : m_ref;
-                const float alpha = resc ? ex2_approx(m_ref - m_new) : 1.0f; // 0 on the first tile
-                if (i > 0 && __any_sync(0xFFFFFFFFu, resc)) rescale_o(t_o, alpha);
+                const int vc = tile_valid(a, t);
+                // the whole S row into registers: the second half loads while the
+                // first half's maximum is taken
+                uint32_t s[128];
+                tmem_ld64_issue(t_s, s);
+                tmem_ld64_wait(s);
+                tmem_ld64_issue(t_s + 64, s + 64);
+                if (vc < BN) mask64(s, 0, vc);
+                float mx = max64(s, -INFINITY);
+                tmem_ld64_wait(s + 64);
+                if (vc < BN) mask64(s + 64, 64, vc);
+                mx = max64(s + 64, mx);
+                // bounds of the tile's scaled maximum: x_j = s_j * c_j with every c_j in
+                // [clo, chi], so max_j x_j lies in [lo, hi] below
+                float chi = sl2, clo = sl2;
+                const float4* cf = nullptr;
+                if (coef) {
+                    if (!(ok = mbar_wait(bar(B_CFULL + slot), (i / kCoefSlots) & 1, ctl))) break;
+                    const float4* bd = reinterpret_cast<const float4*>(smem + kOffBound + slot * 32);
+                    const float4 b0 = bd[0], b1 = bd[1];
+                    chi = fmaxf(fmaxf(b0.x, b0.z), fmaxf(b1.x, b1.z));
+                    clo = fminf(fminf(b0.y, b0.w), fminf(b1.y, b1.w));
+                    cf = reinterpret_cast<const float4*>(smem + kOffCoef + slot * (BN * 4));
+                }
+                const float hi = mx >= 0.0f ? mx * chi : mx * clo;
+                const float lo = mx >= 0.0f ? mx * clo : mx * chi;
+                // the reference moves only when the tile may exceed it by more than the
+                // threshold; it moves to the upper bound when the bound is within the
+                // threshold of the true maximum, else to the exact maximum
+                const bool up = hi > m_ref + kRescaleThreshold;
+                float m_new = m_ref;
+                if (up) m_new = (coef && hi - lo > kRescaleThreshold) ? max_scaled(s, cf) : hi;
+                const float alpha = up ? ex2_approx(m_ref - m_new) : 1.0f; // 0 on the first tile
+                if (i > 0 && __any_sync(0xFFFFFFFFu, up)) rescale_o(t_o, alpha);
                 l *= alpha;
                 m_ref = m_new;
-                // pass 2: P into TMEM, row sum in fp32
-                l += full ? row_exp_store_full<kInt8 ? kExp2PolyPairsInt8 : kExp2PolyPairsBf16>(t_s, sl2, m_ref)
-                          : row_exp_store_masked(t_s, sl2, m_ref, vc);
+                // P into TMEM, row sum in fp32
+                if (coef) {
+                    l += exp_row<kExp2PolyPairsInt8, true>(s, cf, sl2, m_ref, t_s);
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar(B_CEMPTY + slot));
+                } else {
+                    l += exp_row<kInt8 ? kExp2PolyPairsInt8 : kExp2PolyPairsBf16, false>(s, nullptr, sl2, m_ref,
+                                                                                        t_s);
+                }
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
@@ -618,42 +683,68 @@ __global__ void __launch_bounds__(kInt8 ? 512 : 384, 1)
             }
             // ---- epilogue
             if (ok) ok = mbar_wait(bar(B_OFULL + w), 0, ctl);
-            if (ok) {
+        }
+        const int qrow = (qt0 + w) * BM + r;
+        const bool row_ok = active && ok && qrow < a.nq;
+        if (a.splits == 1) {
+            if (active && ok) {
                 tc_fence_after();
-                const int qrow = (qt0 + w) * BM + r;
-                const bool row_ok = qrow < a.nq;
-                if (a.splits == 1) {
-                    store_out_row(t_o, 1.0f / l, a.out + (static_cast<int64_t>(qrow) * a.heads + head) * kD, row_ok);
-                    if (row_ok && a.lse)
-                        a.lse[static_cast<int64_t>(head) * a.nq + qrow] = (m_ref + log2f(l)) * 0.69314718055994531f;
-                } else {
-                    const int64_t prow = (static_cast<int64_t>(split) * a.heads + head) * (a.pairs * 2 * BM) +
-                                         static_cast<int64_t>(pair) * 2 * BM + w * BM + r;
-                    store_partial_row(t_o, a.part_o + prow * kD, row_ok);
-                    if (row_ok) a.part_ml[prow] = make_float2(m_ref, l);
-                }
+                store_out_row(t_o, 1.0f / l, a.out + (static_cast<int64_t>(qrow) * a.heads + head) * kD, row_ok);
+                if (row_ok && a.lse)
+                    a.lse[static_cast<int64_t>(head) * a.nq + qrow] = (m_ref + log2f(l)) * 0.69314718055994531f;
+            }
+        } else {
+            // partial of this split, then the unit's arrival count; the last CTA to
+            // arrive merges every split's partial of its rows
+            const int units = a.heads * a.pairs;
+            const int64_t pu = static_cast<int64_t>(split) * units + unit;
+            const int prow = w * BM + r;
+            if (active && ok) {
+                tc_fence_after();
+                store_partial_row(t_o, a.part_o + pu * 32 * 256 + prow);
+                a.part_ml[pu * 256 + prow] = make_float2(m_ref, l);
+            }
+            __threadfence();
+            named_bar_sync(2, 256);
+            if (threadIdx.x == 128) {
+                const unsigned old = atomicAdd(&a.counters[unit], 1u);
+                const bool is_last = old == static_cast<unsigned>(a.splits - 1);
+                if (is_last) a.counters[unit] = 0u; // every split has arrived: ready for the next call
+                *last_flag = is_last ? 1 : 0;
+            }
+            named_bar_sync(2, 256);
+            if (*last_flag) {
+                __threadfence();
+                if (row_ok)
+                    merge_row(a, unit, prow, a.out + (static_cast<int64_t>(qrow) * a.heads + head) * kD,
+                              a.lse ? a.lse + static_cast<int64_t>(head) * a.nq + qrow : nullptr);
             }
         }
-    } else if (kInt8 && warp >= 12) {
+    } else if constexpr (kInt8) {
+        regs_dec<Regs<kInt8>::kFiller>();
         // ================================================================ INT8 filler
         // Warp wq converts rows [32 wq, 32 wq + 32) of a cache tile; in step j a
         // warp covers rows 2j and 2j+1, 16 lanes per row, 8 codes per lane, so a
         // lane writes exactly one 16-byte BF16 chunk and each quarter-warp hits 8
-        // distinct chunk slots of the swizzled row (no bank conflicts). The next
-        // cache tile's codes are loaded into registers as soon as the current
-        // tile has been converted, so global latency overlaps the MMA pipeline.
+        // distinct chunk slots of the swizzled row (no bank conflicts). Filler
+        // thread f (0..127) also loads the K and V scales of key f of the tile.
+        // The next cache tile's codes are loaded into registers as soon as the
+        // current tile has been converted, so global latency overlaps the MMAs.
+        const int f = threadIdx.x - 384;
         const int wq = warp - 12;
         const int half = lane >> 4;
         const int l16 = lane & 15;
-        const bool elected = (wq == 0 && lane == 0);
+        const bool elected = (f == 0);
+        const float sl2 = a.scale_log2;
         const uint32_t chunk_off = (l16 >> 3) * kHalfBytes;
         uint2 kb[16], vb[16];
-        float ks_own = 0.0f, vs_own = 0.0f; // scales of row 2*l16 + half of this warp's block
+        float ks_own = 0.0f, vs_own = 0.0f; // scales of key f of the tile whose codes are in kb / vb
+        bool key_ok = false;
         // row (32 wq + 2j + half) of a tile: (row & 7) = (2j & 7) ^ half, so the swizzled
         // chunk slot is slot0 ^ (2j & 7) and the byte offset is a constant per j
         const uint32_t slot0 = static_cast<uint32_t>((l16 & 7) ^ half);
         const uint32_t row_off0 = chunk_off + static_cast<uint32_t>(wq * 32 + half) * 128u;
-        auto load_codes = [&](const int8_t* base, const float* scales, int t, uint2 (&buf)[16], float& sc_own) {
+        auto load_codes = [&](const int8_t* base, int t, uint2 (&buf)[16]) {
             const int key0 = t * BN + wq * 32 + half;
             const int64_t grow0 = static_cast<int64_t>(head) * a.cap_tok + key0;
             const uint2* p = reinterpret_cast<const uint2*>(base + grow0 * kD) + l16;
@@ -662,15 +753,27 @@ __global__ void __launch_bounds__(kInt8 ? 512 : 384, 1)
                 const bool in = key0 + 2 * j < a.nc;
                 buf[j] = in ? __ldg(p + j * 32) : make_uint2(0u, 0u); // 2 rows = 256 B = 32 uint2
             }
-            const int skey = t * BN + wq * 32 + 2 * l16 + half;
-            sc_own = skey < a.nc ? __ldg(scales + static_cast<int64_t>(head) * a.cap_tok + skey) : 0.0f;
         };
-        auto convert = [&](uint32_t tile, const uint2 (&buf)[16], float sc_own) {
+        auto load_scales = [&](int t) {
+            const int key = t * BN + f;
+            key_ok = key < a.nc;
+            const int64_t g = static_cast<int64_t>(head) * a.cap_tok + key;
+            ks_own = key_ok ? __ldg(a.ksc + g) : 0.0f;
+            vs_own = key_ok ? __ldg(a.vsc + g) : 0.0f;
+        };
+        auto convert_k = [&](uint32_t tile) {
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
-                const float sc = __shfl_sync(0xFFFFFFFFu, sc_own, half * 16 + j);
                 const uint32_t off = row_off0 + j * 256u + ((slot0 ^ static_cast<uint32_t>((2 * j) & 7)) << 4);
-                st_shared_v4(tile + off, dequant8(buf[j], sc));
+                st_shared_v4(tile + off, codes_to_bf16<false>(kb[j], 0.0f));
+            }
+        };
+        auto convert_v = [&](uint32_t tile) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const float sc = __shfl_sync(0xFFFFFFFFu, vs_own, 2 * j + half);
+                const uint32_t off = row_off0 + j * 256u + ((slot0 ^ static_cast<uint32_t>((2 * j) & 7)) << 4);
+                st_shared_v4(tile + off, codes_to_bf16<true>(vb[j], sc));
             }
         };
         // one elected thread waits; the group learns the outcome after a named
@@ -681,9 +784,10 @@ __global__ void __launch_bounds__(kInt8 ? 512 : 384, 1)
             return *dq_go != 0;
         };
         int k_armed[kStages] = {-1, -1}, v_armed[kStages] = {-1, -1};
-        if (t_begin < a.tiles_c) {
-            load_codes(a.kc8, a.ksc, t_begin, kb, ks_own);
-            load_codes(a.vc8, a.vsc, t_begin, vb, vs_own);
+        if (nci > 0) {
+            load_codes(a.kc8, t_begin, kb);
+            load_codes(a.vc8, t_begin, vb);
+            load_scales(t_begin);
         }
         for (int i = 0; i < n; ++i) {
             const int t = t_begin + i;
@@ -691,31 +795,53 @@ __global__ void __launch_bounds__(kInt8 ? 512 : 384, 1)
             const uint32_t free_ph = ((i / kStages) & 1) ^ 1;
             const uint32_t ktile = sbase + kOffK + st * kTileBytes;
             const uint32_t vtile = sbase + kOffV + st * kTileBytes;
-            const bool next_cached = (t + 1 < a.tiles_c && i + 1 < n);
+            const bool cached = i < nci;
+            const bool next_cached = i + 1 < nci;
             // ---- K (freed early: right after the S MMAs of tile i - 2)
             if (i >= kStages && !group_wait(bar(B_KEMPTY + st), free_ph)) break;
-            if (t >= a.tiles_c) {
+            if (!cached) {
                 if (elected) {
                     load_k_tile(a, t, head, ktile, bar(B_KFULL + st), &tm_kc, &tm_kcur);
                     k_armed[st] = (i / kStages) & 1;
                 }
             } else {
-                convert(ktile, kb, ks_own);
-                if (next_cached) load_codes(a.kc8, a.ksc, t + 1, kb, ks_own);
+                const uint32_t slot = static_cast<uint32_t>(i % kCoefSlots);
+                convert_k(ktile);
+                if (next_cached) load_codes(a.kc8, t + 1, kb);
+                // the tile's K coefficients (scale_log2 * K scale; keys past the end
+                // get scale_log2 so that a masked score -inf stays -inf) and their
+                // range per warp, into the coefficient ring
+                if (i >= kCoefSlots && !group_wait(bar(B_CEMPTY + slot), ((i / kCoefSlots) & 1) ^ 1)) break;
+                const float c = key_ok ? sl2 * ks_own : sl2;
+                float cmax = key_ok ? c : -INFINITY, cmin = key_ok ? c : INFINITY;
+#pragma unroll
+                for (int off = 16; off >= 1; off >>= 1) {
+                    cmax = fmaxf(cmax, __shfl_xor_sync(0xFFFFFFFFu, cmax, off));
+                    cmin = fminf(cmin, __shfl_xor_sync(0xFFFFFFFFu, cmin, off));
+                }
+                reinterpret_cast<float*>(smem + kOffCoef + slot * (BN * 4))[f] = c;
+                if (lane == 0)
+                    reinterpret_cast<float2*>(smem + kOffBound + slot * 32)[wq] = make_float2(cmax, cmin);
                 fence_proxy_async_smem();
                 named_bar_sync(1, 128);
-                if (elected) mbar_arrive(bar(B_KFULL + st));
+                if (elected) {
+                    mbar_arrive(bar(B_KFULL + st));
+                    mbar_arrive(bar(B_CFULL + slot));
+                }
             }
             // ---- V (freed after the P.V MMAs of tile i - 2)
             if (i >= kStages && !group_wait(bar(B_VEMPTY + st), free_ph)) break;
-            if (t >= a.tiles_c) {
+            if (!cached) {
                 if (elected) {
                     load_v_tile(a, t, head, vtile, bar(B_VFULL + st), &tm_vc, &tm_vcur);
                     v_armed[st] = (i / kStages) & 1;
                 }
             } else {
-                convert(vtile, vb, vs_own);
-                if (next_cached) load_codes(a.vc8, a.vsc, t + 1, vb, vs_own);
+                convert_v(vtile);
+                if (next_cached) {
+                    load_codes(a.vc8, t + 1, vb);
+                    load_scales(t + 1);
+                }
                 fence_proxy_async_smem();
                 named_bar_sync(1, 128);
                 if (elected) mbar_arrive(bar(B_VFULL + st));
@@ -731,78 +857,6 @@ __global__ void __launch_bounds__(kInt8 ? 512 : 384, 1)
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
-}
-
-__global__ void __launch_bounds__(256) combine_kernel(const __grid_constant__ CombineArgs a) {
-    grid_dep_wait(); // launched dependent on the attention kernel
-    // one warp per (head, query row); each lane owns 4 of the 128 dims
-    const int64_t gw = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-    const int lane = threadIdx.x & 31;
-    if (gw >= static_cast<int64_t>(a.heads) * a.nq) return;
-    const int head = static_cast<int>(gw / a.nq);
-    const int qrow = static_cast<int>(gw % a.nq);
-    const int64_t rows_per_head = static_cast<int64_t>(a.pairs) * 2 * BM;
-    float mmax = -INFINITY;
-    for (int s = 0; s < a.splits; ++s)
-        mmax = fmaxf(mmax, a.part_ml[(static_cast<int64_t>(s) * a.heads + head) * rows_per_head + qrow].x);
-    float L = 0.0f;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s = 0; s < a.splits; ++s) {
-        const int64_t prow = (static_cast<int64_t>(s) * a.heads + head) * rows_per_head + qrow;
-        const float2 ml = a.part_ml[prow];
-        const float wgt = exp2f(ml.x - mmax);
-        L += ml.y * wgt;
-        const float4 o = reinterpret_cast<const float4*>(a.part_o + prow * kD)[lane];
-        acc.x += o.x * wgt;
-        acc.y += o.y * wgt;
-        acc.z += o.z * wgt;
-        acc.w += o.w * wgt;
-    }
-    const float inv = 1.0f / L;
-    uint2 b;
-    b.x = pack_bf16x2(acc.x * inv, acc.y * inv);
-    b.y = pack_bf16x2(acc.z * inv, acc.w * inv);
-    reinterpret_cast<uint2*>(a.out + (static_cast<int64_t>(qrow) * a.heads + head) * kD)[lane] = b;
-    if (lane == 0 && a.lse) a.lse[static_cast<int64_t>(head) * a.nq + qrow] = (mmax + log2f(L)) * 0.69314718055994531f;
-}
-
-// One work item = 16 codes (16 bytes) of one row of K or V; 8 items per row,
-// consecutive threads on consecutive items, so loads (128 B per row) and
-// stores (256 B per row) are fully coalesced. Grid-stride over both tensors.
-__global__ void __launch_bounds__(512) dequant_window_kernel(const __grid_constant__ DequantArgs a) {
-    // Launched dependent on the RoPE prep kernel and overlapping it: it reads
-    // only the cache, which was complete before prep started. It lets the
-    // attention kernel launch early, and before it exits it waits for prep, so
-    // the attention kernel's wait on it covers prep too.
-    grid_dep_launch();
-    const uint32_t rows = static_cast<uint32_t>(a.heads) * static_cast<uint32_t>(a.nc); // per tensor, < 2^31
-    const uint32_t items = 2u * rows * 8u;                                              // < 2^32 by the host check
-    for (uint32_t it = blockIdx.x * blockDim.x + threadIdx.x; it < items; it += gridDim.x * blockDim.x) {
-        const uint32_t trow = it >> 3;
-        const uint32_t part = it & 7u;
-        const bool is_v = trow >= rows;
-        const uint32_t r = is_v ? trow - rows : trow;
-        const uint32_t head = fast_div(r, a.div_nc);
-        const uint32_t tok = r - head * static_cast<uint32_t>(a.nc);
-        const int64_t src_row = static_cast<int64_t>(head) * a.cap_tok + tok;
-        const uint4 w = __ldg(reinterpret_cast<const uint4*>((is_v ? a.vc : a.kc) + src_row * kD) + part);
-        const float sc = __ldg((is_v ? a.vs : a.ks) + src_row);
-        uint4* dst = reinterpret_cast<uint4*>((is_v ? a.vd : a.kd) + static_cast<int64_t>(r) * kD) + 2 * part;
-        dst[0] = dequant8(make_uint2(w.x, w.y), sc);
-        dst[1] = dequant8(make_uint2(w.z, w.w), sc);
-    }
-    grid_dep_wait();
-}
-
-} // namespace
-
-cudaError_t launch_dequant_window(const DequantArgs& a, cudaStream_t s) {
-    const uint64_t items = 2ull * static_cast<uint64_t>(a.heads) * static_cast<uint64_t>(a.nc) * 8ull;
-    if (items == 0) return cudaSuccess;
-    uint64_t blocks = (items + 511) / 512;
-    const uint64_t cap = 148ull * 4ull; // persistent: 4 blocks of 512 threads per SM
-    if (blocks > cap) blocks = cap;
-    return launch_dependent(dequant_window_kernel, dim3(static_cast<unsigned>(blocks)), dim3(512), 0, s, a);
 }
 
 // The dynamic shared-memory limit of a kernel is an attribute of the kernel in
@@ -822,6 +876,8 @@ cudaError_t ensure_smem_attr() {
     return e;
 }
 
+} // namespace
+
 cudaError_t launch_attn(const AttnArgs& a, bool int8_cache, const CUtensorMap& tm_q, const CUtensorMap& tm_kcur,
                         const CUtensorMap& tm_vcur, const CUtensorMap& tm_kc, const CUtensorMap& tm_vc,
                         cudaStream_t s) {
@@ -831,19 +887,11 @@ cudaError_t launch_attn(const AttnArgs& a, bool int8_cache, const CUtensorMap& t
         if (e != cudaSuccess) return e;
         return launch_dependent(attn_kernel<true>, dim3(grid), dim3(512), kSmemBytes, s, a, tm_q, tm_kcur, tm_vcur,
                                 tm_kc, tm_vc);
-    } else {
-        cudaError_t e = ensure_smem_attr<false>();
-        if (e != cudaSuccess) return e;
-        return launch_dependent(attn_kernel<false>, dim3(grid), dim3(384), kSmemBytes, s, a, tm_q, tm_kcur, tm_vcur,
-                                tm_kc, tm_vc);
     }
-    return cudaGetLastError();
-}
-
-cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s) {
-    const int64_t warps = static_cast<int64_t>(a.heads) * a.nq;
-    const int64_t blocks = (warps * 32 + 255) / 256;
-    return launch_dependent(combine_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, a);
+    cudaError_t e = ensure_smem_attr<false>();
+    if (e != cudaSuccess) return e;
+    return launch_dependent(attn_kernel<false>, dim3(grid), dim3(384), kSmemBytes, s, a, tm_q, tm_kcur, tm_vcur,
+                            tm_kc, tm_vc);
 }
 
 } // namespace nomas

@@ -136,7 +136,7 @@ def test_full_history_capacity_is_enforced_before_launch():
 def test_seg_attn_argument_checks():
     d = desc()
     assert nm.nomas_cache_reset(d) == nm.NOMAS_OK
-    need = nm.nomas_seg_attn_workspace_bytes(d, 3, 256)
+    need = nm.nomas_seg_attn_workspace_min_bytes(d, 3, 256)
     assert need > 2 * 16 * 2896 * 128 * 2  # holds at least rotated Q and K
     call = lambda **kw: nm.nomas_seg_attn(d, kw.get("q", FAKE), FAKE, FAKE, kw.get("ts", 2048), kw.get("nv", 3),
                                           kw.get("nt", 256), kw.get("out", FAKE), kw.get("lse", None),
@@ -162,22 +162,27 @@ def test_workspace_size_is_a_function_of_the_shape():
     assert nm.nomas_seg_attn_workspace_bytes(d, -1, 0) == 0
 
 
-def test_min_workspace_selects_the_fused_form_and_bounds_the_call():
+def test_workspace_plans_between_the_minimum_and_the_full_size():
     d = desc()
     assert nm.nomas_cache_reset(d) == nm.NOMAS_OK
     d.valid_frames = 18  # as after 18 committed frames (state is not part of the stamp)
     full = nm.nomas_seg_attn_workspace_bytes(d, 3, 256)
     low = nm.nomas_seg_attn_workspace_min_bytes(d, 3, 256)
-    # the full workspace adds the BF16 copy of the window: 2 x 16 heads x 15,840 tokens x 256 B
-    assert full - low >= 2 * 16 * 18 * 880 * 256
+    # the minimum is the one-split plan: the 256-byte status header and the rotated Q
+    # and K (16 heads x 2896 tokens x 256 B each, rounded up to 256 bytes)
+    qk = -(-16 * 2896 * 128 * 2 // 256) * 256
+    assert low == 256 + 2 * qk
+    # the full plan adds the KV-split partials: per split, 16 heads x 12 Q-tile pairs x
+    # 256 rows of 128 fp32 values and an fp32 (max, sum) pair, and one counter per unit
+    part = full - low
+    per_split = 16 * 12 * 256 * (128 * 4 + 8)
+    assert part >= 2 * per_split and part % 256 == 0
     call = lambda wsb: nm.nomas_seg_attn(d, FAKE, FAKE, FAKE, 2048, 3, 256, FAKE, None, FAKE, wsb, None)
     assert call(low - 1) == nm.NOMAS_ERR_WORKSPACE
-    # with low or more bytes validation passes; without a GPU the call then stops at the device check
-    assert call(low) in (nm.NOMAS_ERR_DEVICE, nm.NOMAS_ERR_CUDA)
-    bf = desc(mode=nm.NOMAS_CACHE_BF16, window=0, cap=20)
-    assert nm.nomas_cache_reset(bf) == nm.NOMAS_OK
-    bf.valid_frames = 18
-    assert nm.nomas_seg_attn_workspace_bytes(bf, 3, 256) == nm.nomas_seg_attn_workspace_min_bytes(bf, 3, 256)
+    # the minimum, the full size and any size in between (a plan with fewer splits)
+    # pass validation; without a GPU the call then stops at the device check
+    for wsb in (low, (low + full) // 2, full):
+        assert call(wsb) in (nm.NOMAS_ERR_DEVICE, nm.NOMAS_ERR_CUDA)
 
 
 def test_layered_commit_argument_checks():

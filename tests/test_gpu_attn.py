@@ -14,10 +14,10 @@ from harness import MAX_ABS, REL_L2, Guards, current_segment, errors, make_cache
 pytestmark = pytest.mark.gpu
 
 
-def run_case(w, rows=None, check_lse=True, rel_l2=REL_L2, path="once"):
-    """path: "once" = the workspace of nomas_seg_attn_workspace_bytes (an INT8 window is
-    dequantised once, then the BF16-cache kernel runs); "fused" = the minimum workspace
-    (the INT8 kernel converts each tile in shared memory)."""
+def run_case(w, rows=None, check_lse=True, rel_l2=REL_L2, path="full"):
+    """path: "full" = the workspace of nomas_seg_attn_workspace_bytes (the fastest plan,
+    KV splits merged inside the kernel when the shape has them); "min" = the minimum
+    workspace (one split: each CTA covers every KV tile of its unit)."""
     torch = __import__("torch")
     g = Guards()
     gpu, orc = make_caches(w, guards=g)
@@ -26,7 +26,7 @@ def run_case(w, rows=None, check_lse=True, rel_l2=REL_L2, path="once"):
     lse = g.alloc((w["heads"], nq), torch.float32, fill=float("nan"))
     out = g.alloc((nq, w["heads"], 128), torch.bfloat16, fill=float("nan"))
     ws = None
-    if path == "fused":
+    if path == "min":
         need = gpu.workspace_min_bytes(w["cur_frames"], w["n_text"])
         ws = g.alloc((need,), torch.uint8)
     gpu.seg_attn(to_dev(q), to_dev(k), to_dev(v), w["cur_frames"], w["n_text"], out=out, lse=lse, workspace=ws)
@@ -62,7 +62,7 @@ def test_tiny_workload():
     run_case(synth.WORKLOADS["tiny"])
 
 
-INT8_PATHS = ["once", "fused"]
+INT8_PATHS = ["full", "min"]
 
 
 @pytest.mark.parametrize("path", INT8_PATHS)
@@ -70,7 +70,7 @@ def test_tiny_int8(path):
     run_case(wl(mode="int8", window=4, capacity=4, hist_commits=[1, 2]), path=path)
 
 
-@pytest.mark.parametrize("mode,path", [("bf16", "once"), ("int8", "once"), ("int8", "fused")])
+@pytest.mark.parametrize("mode,path", [("bf16", "full"), ("int8", "full"), ("int8", "min")])
 def test_ragged_tiles_and_tails(mode, path):
     # 35 tokens/frame, 4 history frames = 140 keys (128 + 12); 5 frames + 37 text = 212 queries (128 + 84)
     run_case(wl(heads=3, grid_h=5, grid_w=7, mode=mode, window=4 if mode == "int8" else 0,
@@ -78,7 +78,7 @@ def test_ragged_tiles_and_tails(mode, path):
              path=path)
 
 
-@pytest.mark.parametrize("mode,path", [("bf16", "once"), ("int8", "once"), ("int8", "fused")])
+@pytest.mark.parametrize("mode,path", [("bf16", "full"), ("bf16", "min"), ("int8", "full"), ("int8", "min")])
 def test_multi_tile_with_kv_splits(mode, path):
     # 256 tokens/frame: 1536 cached keys (12 tiles), 868 queries (7 tiles): the split-KV + combine path
     run_case(wl(heads=4, grid_h=16, grid_w=16, mode=mode, window=6 if mode == "int8" else 0,
@@ -134,9 +134,9 @@ def test_rising_scores_force_rescales(mode):
 
 @pytest.mark.parametrize("path", INT8_PATHS)
 def test_int8_split_mixing_cache_and_current_tiles(path):
-    """160 Q-tile pairs x 38 KV tiles: three KV splits, the middle one runs five
-    cache tiles and then current-segment tiles (fused path: dequantised cache
-    tiles, then TMA-loaded current tiles)."""
+    """160 Q-tile pairs x 38 KV tiles: the KV splits of the full plan, one of
+    which runs its last cache tiles (converted in shared memory) and then
+    current-segment tiles (TMA-loaded); and the one-split plan."""
     w = wl(heads=16, grid_h=8, grid_w=16, mode="int8", window=18, capacity=18, hist_commits=[6, 6, 6],
            cur_frames=19, n_text=64, seed=15)
     F = 128
@@ -178,10 +178,11 @@ def test_single_gpu_configuration_all_rows(path):
     run_case(w, path=path)
 
 
-def test_int8_paths_agree():
-    """Both INT8 forms feed identical BF16 K/V values to the tensor cores; they
-    differ only in the softmax exponentials (part on the FMA pipe in the BF16
-    kernel), so their outputs agree far inside the oracle tolerance."""
+def test_int8_plans_agree():
+    """The full plan (KV splits merged in the kernel) and the one-split plan feed
+    identical K/V values to the tensor cores; they differ only in where the
+    running maximum of each split starts and in the fp32 merge, so their
+    outputs agree far inside the oracle tolerance."""
     torch = __import__("torch")
     w = wl(heads=4, grid_h=16, grid_w=16, mode="int8", window=6, capacity=6, hist_commits=[3, 3], cur_frames=3,
            n_text=100, seed=16)
