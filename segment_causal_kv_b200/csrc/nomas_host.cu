@@ -149,7 +149,8 @@ bool make_tmap(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint6
 struct Plan {
     int64_t tpf, nv, nq, nc;
     int tiles_c, tiles_q, pairs, splits, tiles_per_split;
-    size_t off_qt, off_kt, off_po, off_pml, off_cnt;
+    bool window;  // INT8 cache read through a BF16 copy of its visible window
+    size_t off_qt, off_kt, off_po, off_pml, off_cnt, off_kd, off_vd;
     size_t total; // workspace bytes of this plan
 };
 
@@ -177,10 +178,15 @@ void choose_splits(int units, int tiles, int max_splits, int& splits, int& tps) 
     }
 }
 
-// Workspace layout of a plan: status header, rotated Q and K (head-major),
-// and with splits > 1 the split partials [splits][units][32][256] float4,
-// their (max, sum) pairs [splits][units][256] and one arrival counter per unit.
-Plan make_plan(const nomas_cache* c, int32_t n_video_frames, int32_t n_text, int max_splits) {
+// The window copy's dequantisation kernel indexes (tensor, row, 16-code part)
+// in 32 bits, with a few grid strides of headroom.
+bool window_copy_fits(int heads, int64_t nc) { return static_cast<int64_t>(heads) * nc < (int64_t(1) << 27); }
+
+// Workspace layout of a plan: status header, rotated Q and K (head-major);
+// with splits > 1 the split partials [splits][units][32][256] float4, their
+// (max, sum) pairs [splits][units][256] and one arrival counter per unit; with
+// the window form the BF16 copy of the visible window, K then V [heads][nc][128].
+Plan make_plan(const nomas_cache* c, int32_t n_video_frames, int32_t n_text, int max_splits, bool window) {
     Plan p{};
     p.tpf = static_cast<int64_t>(c->grid_h) * c->grid_w;
     p.nv = static_cast<int64_t>(n_video_frames) * p.tpf;
@@ -189,6 +195,7 @@ Plan make_plan(const nomas_cache* c, int32_t n_video_frames, int32_t n_text, int
     p.tiles_c = static_cast<int>((p.nc + kBM - 1) / kBM);
     p.tiles_q = static_cast<int>((p.nq + kBM - 1) / kBM);
     p.pairs = (p.tiles_q + 1) / 2;
+    p.window = window;
     const int units = c->heads * p.pairs;
     choose_splits(units, p.tiles_c + p.tiles_q, max_splits, p.splits, p.tiles_per_split);
     const size_t qk_bytes = static_cast<size_t>(c->heads) * p.nq * kD * 2;
@@ -199,22 +206,38 @@ Plan make_plan(const nomas_cache* c, int32_t n_video_frames, int32_t n_text, int
     p.off_po = round_up(p.off_kt + qk_bytes, 256);
     p.off_pml = p.off_po + (sp ? prow * kD * sizeof(float) : 0);
     p.off_cnt = round_up(p.off_pml + (sp ? prow * sizeof(float2) : 0), 256);
-    p.total = round_up(p.off_cnt + (sp ? static_cast<size_t>(units) * sizeof(unsigned) : 0), 256);
+    p.off_kd = p.off_vd = p.total = round_up(p.off_cnt + (sp ? static_cast<size_t>(units) * sizeof(unsigned) : 0), 256);
+    if (window) {
+        const size_t copy = round_up(static_cast<size_t>(c->heads) * p.nc * kD * 2, 256);
+        p.off_vd = p.off_kd + copy;
+        p.total = p.off_vd + copy;
+    }
     return p;
 }
 
 constexpr int kMaxSplits = 32;
 
-// The fastest plan whose workspace fits in `bytes` (fewer splits need less:
-// splits = 1 keeps no partials). Returns false when not even that fits.
+// An INT8 cache with a visible history can use the window form.
+bool window_form(const nomas_cache* c) {
+    const int64_t nc = static_cast<int64_t>(c->valid_frames) * c->grid_h * c->grid_w;
+    return c->mode == NOMAS_CACHE_INT8 && nc > 0 && window_copy_fits(c->heads, nc);
+}
+
+// The fastest plan whose workspace fits in `bytes`: for an INT8 cache the
+// window form before the in-shared-memory form (it runs at about twice the
+// rate per KV tile), and within a form more splits before fewer (fewer need
+// less room: splits = 1 keeps no partials). False when nothing fits.
 bool fit_plan(const nomas_cache* c, int32_t n_video_frames, int32_t n_text, size_t bytes, Plan& out) {
-    int cap = kMaxSplits;
-    while (true) {
-        out = make_plan(c, n_video_frames, n_text, cap);
-        if (out.total <= bytes) return true;
-        if (out.splits <= 1) return false;
-        cap = out.splits - 1;
+    for (int form = window_form(c) ? 1 : 0; form >= 0; --form) {
+        int cap = kMaxSplits;
+        while (true) {
+            out = make_plan(c, n_video_frames, n_text, cap, form == 1);
+            if (out.total <= bytes) return true;
+            if (out.splits <= 1) break;
+            cap = out.splits - 1;
+        }
     }
+    return false;
 }
 
 } // namespace
@@ -436,12 +459,12 @@ int nomas_kv_archive_evicted(const nomas_cache* c, int32_t n_frames, void* host_
 
 size_t nomas_seg_attn_workspace_bytes(const nomas_cache* c, int32_t n_video_frames, int32_t n_text) {
     if (validate_state(c) != NOMAS_OK || n_video_frames < 0 || n_text < 0) return 0;
-    return make_plan(c, n_video_frames, n_text, kMaxSplits).total;
+    return make_plan(c, n_video_frames, n_text, kMaxSplits, window_form(c)).total;
 }
 
 size_t nomas_seg_attn_workspace_min_bytes(const nomas_cache* c, int32_t n_video_frames, int32_t n_text) {
     if (validate_state(c) != NOMAS_OK || n_video_frames < 0 || n_text < 0) return 0;
-    return make_plan(c, n_video_frames, n_text, 1).total;
+    return make_plan(c, n_video_frames, n_text, 1, false).total;
 }
 
 int nomas_seg_attn(const nomas_cache* c, const void* q, const void* k, const void* v, int64_t token_stride,
@@ -450,7 +473,7 @@ int nomas_seg_attn(const nomas_cache* c, const void* q, const void* k, const voi
     int rc = validate_state(c);
     if (rc != NOMAS_OK) return rc;
     if (n_video_frames < 0 || n_text < 0) return NOMAS_ERR_ARG;
-    Plan p = make_plan(c, n_video_frames, n_text, 1);
+    Plan p = make_plan(c, n_video_frames, n_text, 1, false);
     if (p.nq == 0) return NOMAS_OK;
     if (p.nq > (int64_t(1) << 30) || p.nq * c->heads >= (int64_t(1) << 31)) return NOMAS_ERR_ARG;
     if (!q || !k || !v || !out) return NOMAS_ERR_ARG;
@@ -504,20 +527,40 @@ int nomas_seg_attn(const nomas_cache* c, const void* q, const void* k, const voi
         } while (true);
     }
 
-    // 2) tensor maps
+    // 2) an INT8 window is dequantised once into its BF16 copy (window form)
+    const bool int8 = c->mode == NOMAS_CACHE_INT8;
+    const int64_t cap_tok = static_cast<int64_t>(c->capacity_frames) * p.tpf;
+    uint16_t* kd = reinterpret_cast<uint16_t*>(ws + p.off_kd);
+    uint16_t* vd = reinterpret_cast<uint16_t*>(ws + p.off_vd);
+    if (p.window) {
+        DequantArgs d{};
+        d.kc = static_cast<const int8_t*>(c->k);
+        d.vc = static_cast<const int8_t*>(c->v);
+        d.vs = c->v_scale;
+        d.kd = kd;
+        d.vd = vd;
+        d.cap_tok = cap_tok;
+        d.nc = static_cast<int32_t>(p.nc);
+        d.heads = c->heads;
+        d.div_nc = make_fastdiv(static_cast<uint32_t>(p.nc));
+        if (launch_dequant_window(d, s) != cudaSuccess) return NOMAS_ERR_CUDA;
+    }
+
+    // 3) tensor maps
     CUtensorMap tm_q, tm_kcur, tm_vcur, tm_kc, tm_vc;
     const uint64_t row_bytes = kD * 2;
     bool ok = make_tmap(&tm_q, qt, kD, p.nq, c->heads, row_bytes, p.nq * row_bytes, kBM, 1) &&
               make_tmap(&tm_kcur, kt, kD, p.nq, c->heads, row_bytes, p.nq * row_bytes, kBM, 1) &&
               make_tmap(&tm_vcur, v, kD, c->heads, p.nq, row_bytes, token_stride * 2, 1, kBM);
-    const int64_t cap_tok = static_cast<int64_t>(c->capacity_frames) * p.tpf;
-    const bool int8 = c->mode == NOMAS_CACHE_INT8;
     if (!int8) {
         const uint64_t nc_ext = p.nc > 0 ? p.nc : 1;
         ok = ok && make_tmap(&tm_kc, c->k, kD, nc_ext, c->heads, row_bytes, cap_tok * row_bytes, kBM, 1) &&
              make_tmap(&tm_vc, c->v, kD, nc_ext, c->heads, row_bytes, cap_tok * row_bytes, kBM, 1);
+    } else if (p.window) {
+        ok = ok && make_tmap(&tm_kc, kd, kD, p.nc, c->heads, row_bytes, p.nc * row_bytes, kBM, 1) &&
+             make_tmap(&tm_vc, vd, kD, p.nc, c->heads, row_bytes, p.nc * row_bytes, kBM, 1);
     } else {
-        tm_kc = tm_q; // unused: the INT8 kernel converts cache tiles itself
+        tm_kc = tm_q; // unused: the fused form converts cache tiles itself
         tm_vc = tm_q;
     }
     if (!ok) return NOMAS_ERR_CUDA;
@@ -544,7 +587,8 @@ int nomas_seg_attn(const nomas_cache* c, const void* q, const void* k, const voi
     a.counters = counters;
     a.err = reinterpret_cast<unsigned*>(ws);
     a.scale_log2 = static_cast<float>(1.4426950408889634 / sqrt(static_cast<double>(kD)));
-    if (launch_attn(a, int8, tm_q, tm_kcur, tm_vcur, tm_kc, tm_vc, s) != cudaSuccess) return NOMAS_ERR_CUDA;
+    const AttnForm form = !int8 ? AttnForm::kBf16Cache : p.window ? AttnForm::kInt8Window : AttnForm::kInt8Fused;
+    if (launch_attn(a, form, tm_q, tm_kcur, tm_vcur, tm_kc, tm_vc, s) != cudaSuccess) return NOMAS_ERR_CUDA;
     return NOMAS_OK;
 }
 

@@ -117,6 +117,27 @@ struct AttnArgs {
     float scale_log2;       // log2(e) / sqrt(128)
 };
 
+// Dequantisation of an INT8 cache's visible window into a BF16 copy, once per
+// attention call: rows [0, nc) of every head, written head-major
+// [heads][nc][128]. K rows are the codes themselves (exact in BF16; the K scale
+// is applied to the scores by the attention kernel), V rows code * scale
+// rounded to BF16 (the values the in-shared-memory conversion produces).
+struct DequantArgs {
+    const int8_t* kc;
+    const int8_t* vc;
+    const float* vs;
+    uint16_t* kd;
+    uint16_t* vd;
+    int64_t cap_tok; // token capacity of one head's slab in the cache
+    int32_t nc;      // visible tokens per head
+    int32_t heads;
+    FastDiv div_nc;
+};
+
+// Forms of the attention kernel: a BF16 cache; an INT8 cache read through its
+// dequantised window copy; an INT8 cache converted in shared memory.
+enum class AttnForm { kBf16Cache, kInt8Window, kInt8Fused };
+
 // Per-latent-frame camera cross-attention: rows are (video token, head) pairs,
 // row = token * heads + head; token i uses camera chunk (i / tpf) / chunk_frames.
 struct CamArgs {
@@ -154,9 +175,10 @@ cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, si
 // Kernel launchers (return cudaError_t of the launch).
 cudaError_t launch_commit(const CommitArgs& a, const CommitLayers& layers, const RopeTab& tab, cudaStream_t s);
 cudaError_t launch_prep(const PrepArgs& a, const RopeTab& tab, cudaStream_t s);
-cudaError_t launch_attn(const AttnArgs& a, bool int8_cache, const CUtensorMap& tm_q, const CUtensorMap& tm_kcur,
+cudaError_t launch_attn(const AttnArgs& a, AttnForm form, const CUtensorMap& tm_q, const CUtensorMap& tm_kcur,
                         const CUtensorMap& tm_vcur, const CUtensorMap& tm_kc, const CUtensorMap& tm_vc,
                         cudaStream_t s);
+cudaError_t launch_dequant_window(const DequantArgs& a, cudaStream_t s);
 cudaError_t launch_camera_attn(const CamArgs& a, cudaStream_t s);
 
 } // namespace nomas

@@ -6,34 +6,40 @@
 // visible cached tokens of earlier segments followed by every token of the
 // current segment (no mask inside a segment; causality across segments is
 // structural: later segments are never in the cache). An INT8 cache is
-// converted to BF16 in shared memory tile by tile (model card, "Single-GPU
-// Low-Memory Inference": INT8 KV storage, BF16 attention computation).
+// attended to in BF16 (model card, "Single-GPU Low-Memory Inference": INT8 KV
+// storage, BF16 attention computation): K as its integer codes, which BF16
+// holds exactly, with the per-key K scale applied to the scores in the
+// softmax; V as code * scale rounded to BF16.
+//
+// Three forms (template parameter kMode):
+//   kBf16   BF16 cache; every K/V tile arrives by TMA.
+//   kWindow INT8 cache whose visible window dequant_window_kernel has written
+//           to a BF16 copy once per call (K codes, V code * scale); tiles by
+//           TMA, the K scales of each cache tile go into a coefficient ring.
+//   kFused  INT8 cache converted in shared memory tile by tile by a filler
+//           warpgroup (no copy: for workspaces too small to hold one).
 //
 // Structure of one CTA (one "unit" = two 128-row Q tiles of one head, and a
 // contiguous range of 128-key KV tiles: cache tiles first, then the current
 // segment's tiles):
-//   warp 0      TMA producer: Q tiles once, then (BF16 caches) every K/V tile
-//               into a 2-stage ring
+//   warp 0      TMA producer: Q tiles once, then (kBf16, kWindow) every K/V
+//               tile into a 2-stage ring; kWindow: the K coefficients
 //   warp 1      TMEM allocator + tcgen05.mma issuer
 //   warps 4-7   softmax warpgroup for Q tile 0 (one thread per query row)
 //   warps 8-11  softmax warpgroup for Q tile 1
-//   warps 12-15 INT8 caches only: the one filler of the K/V ring. Cache K
-//               tiles hold the INT8 codes themselves as BF16 (exact for
-//               |code| <= 127) and the per-key K scale goes to the softmax as
-//               a per-column coefficient; cache V tiles hold code * scale
-//               rounded to BF16. Current-segment tiles are loaded by TMA. One
-//               filler in tile order keeps every parity wait on the ring exact.
+//   warps 12-15 kFused only: the one filler of the K/V ring. Cache tiles are
+//               converted from codes and scales; current-segment tiles are
+//               loaded by TMA. One filler in tile order keeps every parity
+//               wait on the ring exact.
 // TMEM (512 columns): S0 | S1 | O0 | O1, 128 fp32 columns each; the BF16
 // probabilities P overwrite the first 64 columns of their S block and feed
 // the P.V product straight from TMEM (A operand in tensor memory).
 // MMA order per KV tile j: PV0(j-1) S0(j) | PV1(j-1) S1(j) -- while one
 // softmax warpgroup exponentiates, the tensor core works for the other. The
 // issuer waits for V(j-1) before PV0(j-1) and for K(j) only before S0(j).
-// Softmax: a thread reads its whole 128-column S row from TMEM into registers
-// once, takes the row maximum there and exponentiates from registers. Online
-// softmax in base 2 with lazy rescaling: the running reference max is raised
-// only when a tile's max exceeds it by more than 8 (so P <= 256), and only
-// then is O rescaled in TMEM.
+// Online softmax in base 2 with lazy rescaling: the running reference max is
+// raised only when a tile's max may exceed it by more than 8 (so P <= 256),
+// and only then is O rescaled in TMEM.
 // Split-KV: with splits > 1 each CTA leaves (O unnormalised, max, sum) in the
 // workspace and counts itself in per unit; the last CTA of a unit to arrive
 // merges the splits and writes the output (the partials are still in L2).
@@ -85,15 +91,7 @@ constexpr uint32_t kOffLast = kOffDqGo + 4;
 static_assert(kOffLast + 4 <= 256, "barrier area overflow");
 static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 
-// Register budgets per warpgroup (setmaxnreg). The CTA is launched with the
-// registers the compiler reports for the kernel (BF16: 384 threads x 168 =
-// 64,512; INT8: 512 x 128 = 65,536); the budgets add up to exactly that:
-// BF16 128 x 72 + 256 x 216; INT8 128 x 64 + 256 x 176 + 128 x 96.
-template <bool kInt8> struct Regs;
-template <> struct Regs<false> { static constexpr uint32_t kCtl = 72, kSoftmax = 216, kFiller = 0; };
-template <> struct Regs<true> { static constexpr uint32_t kCtl = 64, kSoftmax = 176, kFiller = 96; };
-static_assert(128 * 72 + 256 * 216 == 384 * 168, "BF16 register split");
-static_assert(128 * 64 + 256 * 176 + 128 * 96 == 512 * 128, "INT8 register split");
+enum { kBf16 = 0, kWindow = 1, kFused = 2 };
 
 // mbar_wait run by every lane of a converged warp; lane 0's outcome is
 // broadcast so the warp leaves the wait converged.
@@ -188,25 +186,55 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
     return r;
 }
 
-// Maximum of 64 raw scores held in registers; eight independent accumulators
-// keep the reduction off a single dependency chain.
-__device__ __forceinline__ float max64(const uint32_t* s, float init) {
-    float m[8];
+// Maximum of one 128-key S row over its valid columns (kMask: columns >= vc
+// ignored), raw scores. Eight independent accumulators keep the reduction off
+// a single dependency chain.
+template <bool kMask>
+__device__ __forceinline__ float row_max(uint32_t t_s, int vc) {
+    float mx = -INFINITY;
 #pragma unroll
-    for (int k = 0; k < 8; ++k) m[k] = init;
+    for (int c = 0; c < 2; ++c) {
+        uint32_t s[64];
+        tmem_ld64(t_s + c * 64, s);
+        float m[8];
 #pragma unroll
-    for (int e = 0; e < 64; e += 2)
-        m[(e >> 1) & 7] = max3(m[(e >> 1) & 7], __uint_as_float(s[e]), __uint_as_float(s[e + 1]));
-    return max3(max3(m[0], m[1], m[2]), max3(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
+        for (int k = 0; k < 8; ++k) m[k] = mx;
+#pragma unroll
+        for (int e = 0; e < 64; e += 2) {
+            float x0 = __uint_as_float(s[e]), x1 = __uint_as_float(s[e + 1]);
+            if (kMask) {
+                x0 = (c * 64 + e < vc) ? x0 : -INFINITY;
+                x1 = (c * 64 + e + 1 < vc) ? x1 : -INFINITY;
+            }
+            m[(e >> 1) & 7] = max3(m[(e >> 1) & 7], x0, x1);
+        }
+        mx = max3(max3(m[0], m[1], m[2]), max3(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
+        // keep this chunk's reduction ahead of the next TMEM load, so its 64
+        // registers are dead before the next 64 arrive
+        asm volatile("" : "+f"(mx));
+    }
+    return mx;
 }
 
-// Columns [c0, c0 + 64) at or beyond vc of a ragged tile: score -inf, so they
-// are ignored by the maximum and their probability is 2^-inf = 0 (or 2^-125 on
-// the FMA-pipe path, against V rows that are zero: both the TMA boxes and the
-// INT8 filler fill keys past the end with zeros).
-__device__ __forceinline__ void mask64(uint32_t* s, int c0, int vc) {
+// Exact maximum of s_j * c_j over the valid columns of a row (used when the
+// cheap bound of a tile is too loose to serve as the reference: keys of very
+// different scales). Cold: run by a whole warp only when one of its rows needs it.
+__device__ __noinline__ float row_max_scaled(uint32_t t_s, const float4* coef, int vc) {
+    float mx = -INFINITY;
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+        uint32_t s[32];
+        tmem_ld32(t_s + c * 32, s);
 #pragma unroll
-    for (int e = 0; e < 64; ++e) s[e] = (c0 + e < vc) ? s[e] : 0xFF800000u;
+        for (int e = 0; e < 32; e += 4) {
+            const float4 k = coef[(c * 32 + e) >> 2];
+            const float v[4] = {__uint_as_float(s[e]) * k.x, __uint_as_float(s[e + 1]) * k.y,
+                                __uint_as_float(s[e + 2]) * k.z, __uint_as_float(s[e + 3]) * k.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) mx = (c * 32 + e + q < vc) ? fmaxf(mx, v[q]) : mx;
+        }
+    }
+    return mx;
 }
 
 // 2^x of two values on the FMA pipe, so that part of a row's exponentials
@@ -236,41 +264,96 @@ __device__ __forceinline__ float2 exp2_fma2(float2 x) {
                        __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
 }
 
-// Of every 8 column pairs, kPoly take exp2_fma2 and the rest the MUFU ex2.
-// With an INT8 cache the converting warps share the FMA pipe and the issue
-// slots of every SM sub-partition, so fewer go to the FMA pipe there.
-constexpr int kExp2PolyPairsBf16 = 3;
-constexpr int kExp2PolyPairsInt8 = 2;
+// Of every 8 column pairs of a full tile, kPoly take exp2_fma2 and the rest
+// the MUFU ex2. In the kFused form the converting warps share the FMA pipe
+// and issue slots of every SM sub-partition, so there all go to the MUFU.
+constexpr int kExp2PolyPairs = 3;
+constexpr int kExp2PolyPairsFused = 0;
 
-// P = 2^(s * c - m) of one 128-key S row held in registers, written as packed
-// BF16 pairs over the first 64 columns of the row's S block (all of S is in
-// registers by then); returns the fp32 row sum. c is the scalar scale_log2, or
-// with kCoef the per-column coefficients of the tile (scale_log2 times the
-// key's K scale) read from shared memory four at a time.
+
+// One 32-column chunk of an unmasked S row -> 16 packed BF16 P columns;
+// x = s * c - m with c the scalar scale_log2, or with kCoef the tile's
+// per-column coefficients (scale_log2 times the key's K scale), read from
+// shared memory four at a time.
 template <int kPoly, bool kCoef>
-__device__ __forceinline__ float exp_row(const uint32_t (&s)[128], const float4* coef, float sl2, float m,
-                                         uint32_t t_s) {
+__device__ __forceinline__ void exp_chunk(const uint32_t (&s)[32], const float4* coef, float2 sl2x2, float2 negm,
+                                          float2 (&acc)[4], uint32_t (&p)[16]) {
+    float4 c4 = make_float4(sl2x2.x, sl2x2.x, sl2x2.x, sl2x2.x);
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+        if (kCoef && (e & 1) == 0) c4 = coef[e >> 1];
+        const float2 cc = kCoef ? ((e & 1) ? make_float2(c4.z, c4.w) : make_float2(c4.x, c4.y)) : sl2x2;
+        const float2 x = __ffma2_rn(make_float2(__uint_as_float(s[2 * e]), __uint_as_float(s[2 * e + 1])), cc, negm);
+        float2 y;
+        if ((e & 7) < kPoly)
+            y = exp2_fma2(x);
+        else
+            y = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+        acc[e & 3] = __fadd2_rn(acc[e & 3], y);
+        p[e] = pack_bf16x2(y.x, y.y);
+    }
+}
+
+// P = 2^(s * c - m) of one full 128-key S row, written as packed BF16 pairs
+// over the first 64 columns of the row's S block; returns the fp32 row sum
+// (four independent packed accumulators). The TMEM loads are software
+// pipelined: chunk c + 1 is in flight while chunk c is exponentiated. P chunk c
+// lands on columns [16c, 16c + 16), all of which were read with chunks <= c.
+template <int kPoly, bool kCoef>
+__device__ __forceinline__ float row_exp_store_full(uint32_t t_s, const float4* coef, float sl2, float m) {
+    const float2 sl2x2 = make_float2(sl2, sl2);
     const float2 negm = make_float2(-m, -m);
     float2 acc[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) acc[k] = make_float2(0.0f, 0.0f);
+    uint32_t sa[32], sb[32], p[16];
+    tmem_ld32_issue(t_s, sa);
+    tmem_ld32_wait(sa);
+    tmem_ld32_issue(t_s + 32, sb);
+    exp_chunk<kPoly, kCoef>(sa, coef, sl2x2, negm, acc, p);
+    tmem_st16(t_s, p);
+    tmem_ld32_wait(sb);
+    tmem_ld32_issue(t_s + 64, sa);
+    exp_chunk<kPoly, kCoef>(sb, coef + 8, sl2x2, negm, acc, p);
+    tmem_st16(t_s + 16, p);
+    tmem_ld32_wait(sa);
+    tmem_ld32_issue(t_s + 96, sb);
+    exp_chunk<kPoly, kCoef>(sa, coef + 16, sl2x2, negm, acc, p);
+    tmem_st16(t_s + 32, p);
+    tmem_ld32_wait(sb);
+    exp_chunk<kPoly, kCoef>(sb, coef + 24, sl2x2, negm, acc, p);
+    tmem_st16(t_s + 48, p);
+    const float2 t = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+    return t.x + t.y;
+}
+
+// Masked form for a ragged last tile (columns >= vc get P = 0): MUFU only,
+// one 32-column chunk at a time; coef may be null (scalar scale_log2).
+__device__ __forceinline__ float row_exp_store_masked_impl(uint32_t t_s, const float4* coef, float sl2, float m,
+                                                           int vc) {
+    const float2 negm = make_float2(-m, -m);
+    float2 acc[4];
 #pragma unroll
+    for (int k = 0; k < 4; ++k) acc[k] = make_float2(0.0f, 0.0f);
+#pragma unroll 1
     for (int c = 0; c < 4; ++c) {
+        uint32_t s[32];
+        tmem_ld32(t_s + c * 32, s);
         uint32_t p[16];
-        float4 c4 = make_float4(sl2, sl2, sl2, sl2);
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
+            float2 cc = make_float2(sl2, sl2);
+            if (coef) {
+                const float4 c4 = coef[c * 8 + (e >> 1)];
+                cc = (e & 1) ? make_float2(c4.z, c4.w) : make_float2(c4.x, c4.y);
+            }
+            float2 x = __ffma2_rn(make_float2(__uint_as_float(s[2 * e]), __uint_as_float(s[2 * e + 1])), cc, negm);
             const int col = c * 32 + 2 * e;
-            if (kCoef && (e & 1) == 0) c4 = coef[col >> 2];
-            const float2 cc = (e & 1) ? make_float2(c4.z, c4.w) : make_float2(c4.x, c4.y);
-            const float2 x = __ffma2_rn(make_float2(__uint_as_float(s[col]), __uint_as_float(s[col + 1])), cc, negm);
-            float2 y;
-            if ((e & 7) < kPoly)
-                y = exp2_fma2(x);
-            else
-                y = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-            acc[e & 3] = __fadd2_rn(acc[e & 3], y);
-            p[e] = pack_bf16x2(y.x, y.y);
+            x.x = col < vc ? x.x : -INFINITY;
+            x.y = col + 1 < vc ? x.y : -INFINITY;
+            const float p0 = ex2_approx(x.x), p1 = ex2_approx(x.y);
+            acc[e & 3] = __fadd2_rn(acc[e & 3], make_float2(p0, p1));
+            p[e] = pack_bf16x2(p0, p1);
         }
         tmem_st16(t_s + c * 16, p);
     }
@@ -278,22 +361,15 @@ __device__ __forceinline__ float exp_row(const uint32_t (&s)[128], const float4*
     return t.x + t.y;
 }
 
-// Exact maximum of s_j * c_j over a row (used when the cheap bound of a tile
-// is too loose to serve as the reference: keys of very different scales).
-__device__ __forceinline__ float max_scaled(const uint32_t (&s)[128], const float4* coef) {
-    float m0 = -INFINITY, m1 = -INFINITY;
-#pragma unroll
-    for (int k = 0; k < 32; ++k) {
-        const float4 c = coef[k];
-        m0 = max3(m0, __uint_as_float(s[4 * k]) * c.x, __uint_as_float(s[4 * k + 1]) * c.y);
-        m1 = max3(m1, __uint_as_float(s[4 * k + 2]) * c.z, __uint_as_float(s[4 * k + 3]) * c.w);
-    }
-    return fmaxf(m0, m1);
+// Cold paths kept out of line, so they do not add to the register pressure of
+// the per-tile loop: tail tiles (masked), O rescaling, the epilogues.
+__device__ __noinline__ float row_max_masked(uint32_t t_s, int vc) { return row_max<true>(t_s, vc); }
+__device__ __noinline__ float row_exp_store_masked(uint32_t t_s, const float4* coef, float sl2, float m, int vc) {
+    return row_exp_store_masked_impl(t_s, coef, sl2, m, vc);
 }
 
-// O *= alpha for one row (one thread), in TMEM. Inline: it runs while the
-// thread's S row is held in registers, which a call would have to preserve.
-__device__ __forceinline__ void rescale_o(uint32_t t_o, float alpha) {
+// O *= alpha for one row (one thread), in TMEM.
+__device__ __noinline__ void rescale_o(uint32_t t_o, float alpha) {
 #pragma unroll 1
     for (int c = 0; c < 4; ++c) {
         uint32_t o[32];
@@ -304,9 +380,6 @@ __device__ __forceinline__ void rescale_o(uint32_t t_o, float alpha) {
         tmem_st_wait();
     }
 }
-
-// Cold paths kept out of line, so they do not add to the register pressure of
-// the per-tile loop: the epilogues.
 
 // Final output row: O / l -> BF16 (all lanes load from TMEM; only valid rows store).
 __device__ __noinline__ void store_out_row(uint32_t t_o, float inv_l, uint16_t* dst, bool row_ok) {
@@ -344,36 +417,46 @@ __device__ __noinline__ void store_partial_row(uint32_t t_o, float4* dst) {
 }
 
 // Merge of the splits of one row (run by the last CTA of a unit to arrive):
-// O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s with M = max_s m_s.
+// O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s with M = max_s m_s. Eight
+// 16-byte loads per split are in flight at a time.
 __device__ __noinline__ void merge_row(const AttnArgs& a, int unit, int row, uint16_t* dst, float* lse_dst) {
     const int units = a.heads * a.pairs;
     float mmax = -INFINITY;
     for (int s = 0; s < a.splits; ++s)
         mmax = fmaxf(mmax, __ldcg(&a.part_ml[(static_cast<int64_t>(s) * units + unit) * 256 + row]).x);
     float L = 0.0f;
-    float wgt[8];
     for (int s = 0; s < a.splits; ++s) {
         const float2 ml = __ldcg(&a.part_ml[(static_cast<int64_t>(s) * units + unit) * 256 + row]);
-        const float g = exp2f(ml.x - mmax);
-        if (s < 8) wgt[s] = g;
-        L += ml.y * g;
+        L += ml.y * exp2f(ml.x - mmax);
     }
     const float inv = 1.0f / L;
 #pragma unroll 1
-    for (int c = 0; c < 32; c += 2) {
-        float4 acc0 = make_float4(0.f, 0.f, 0.f, 0.f), acc1 = acc0;
+    for (int c0 = 0; c0 < 32; c0 += 8) {
+        float4 acc[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 1
         for (int s = 0; s < a.splits; ++s) {
-            const float g = s < 8 ? wgt[s]
-                                  : exp2f(__ldcg(&a.part_ml[(static_cast<int64_t>(s) * units + unit) * 256 + row]).x -
-                                          mmax);
-            const float4* base = a.part_o + (static_cast<int64_t>(s) * units + unit) * 32 * 256 + row;
-            const float4 o0 = __ldcg(base + c * 256), o1 = __ldcg(base + (c + 1) * 256);
-            acc0.x += o0.x * g; acc0.y += o0.y * g; acc0.z += o0.z * g; acc0.w += o0.w * g;
-            acc1.x += o1.x * g; acc1.y += o1.y * g; acc1.z += o1.z * g; acc1.w += o1.w * g;
+            const int64_t pu = static_cast<int64_t>(s) * units + unit;
+            const float g = exp2f(__ldcg(&a.part_ml[pu * 256 + row]).x - mmax);
+            const float4* base = a.part_o + pu * 32 * 256 + row;
+            float4 o[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) o[k] = __ldcg(base + (c0 + k) * 256);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                acc[k].x += o[k].x * g;
+                acc[k].y += o[k].y * g;
+                acc[k].z += o[k].z * g;
+                acc[k].w += o[k].w * g;
+            }
         }
-        reinterpret_cast<uint4*>(dst)[c >> 1] =
-            make_uint4(pack_bf16x2(acc0.x * inv, acc0.y * inv), pack_bf16x2(acc0.z * inv, acc0.w * inv),
-                       pack_bf16x2(acc1.x * inv, acc1.y * inv), pack_bf16x2(acc1.z * inv, acc1.w * inv));
+#pragma unroll
+        for (int k = 0; k < 8; k += 2)
+            reinterpret_cast<uint4*>(dst)[(c0 + k) >> 1] =
+                make_uint4(pack_bf16x2(acc[k].x * inv, acc[k].y * inv), pack_bf16x2(acc[k].z * inv, acc[k].w * inv),
+                           pack_bf16x2(acc[k + 1].x * inv, acc[k + 1].y * inv),
+                           pack_bf16x2(acc[k + 1].z * inv, acc[k + 1].w * inv));
     }
     if (lse_dst) *lse_dst = (mmax + log2f(L)) * 0.69314718055994531f;
 }
@@ -418,11 +501,13 @@ __device__ __forceinline__ void drain_armed(const int (&k_armed)[kStages], const
     }
 }
 
-template <bool kInt8>
-__global__ void __launch_bounds__(kInt8 ? 512 : 384, 1)
+template <int kMode>
+__global__ void __launch_bounds__(kMode == kFused ? 512 : 384, 1)
     attn_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CUtensorMap tm_q,
                 const __grid_constant__ CUtensorMap tm_kcur, const __grid_constant__ CUtensorMap tm_vcur,
                 const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CUtensorMap tm_vc) {
+    constexpr bool kInt8 = kMode != kBf16;   // cache tiles carry per-key K coefficients
+    constexpr bool kFill = kMode == kFused;  // cache tiles converted by the filler warpgroup
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
@@ -450,7 +535,7 @@ __global__ void __launch_bounds__(kInt8 ? 512 : 384, 1)
     int t_end = t_begin + a.tiles_per_split;
     if (t_end > t_total) t_end = t_total;
     const int n = t_end - t_begin; // >= 1 by construction of the split count
-    // cache tiles of this CTA come first: i < nci (INT8 caches: converted by the filler)
+    // cache tiles of this CTA come first: i < nci (INT8 caches: K coefficients per tile)
     const int nci = kInt8 ? max(0, min(t_end, a.tiles_c) - t_begin) : 0;
 
     // ---- setup
@@ -488,20 +573,32 @@ __global__ void __launch_bounds__(kInt8 ? 512 : 384, 1)
     // are set up while it finishes; nothing it wrote is read before this point
     grid_dep_wait();
 
-    // Roles by warpgroup. Each warpgroup first sets its register budget (one
-    // setmaxnreg for its four warps, at the top of its own branch, so that
-    // the compiler allocates each role's code under that role's budget): the
-    // control warpgroup and the filler give registers back, the softmax
-    // warpgroups take them.
-    if (warp < 4) {
-        regs_dec<Regs<kInt8>::kCtl>();
-        if (warp == 0) {
+    // the K coefficients of cache tile t into coefficient slot `slot`: scale_log2
+    // times the key's K scale (keys past the end get scale_log2, so that a masked
+    // score -inf stays -inf), and per writer warp the range over valid keys
+    auto put_coef = [&](int t, float ks, bool key_ok, int key_local, uint32_t slot, int bound_idx) {
+        const float c = key_ok ? a.scale_log2 * ks : a.scale_log2;
+        float cmax = key_ok ? c : -INFINITY, cmin = key_ok ? c : INFINITY;
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) {
+            cmax = fmaxf(cmax, __shfl_xor_sync(0xFFFFFFFFu, cmax, off));
+            cmin = fminf(cmin, __shfl_xor_sync(0xFFFFFFFFu, cmin, off));
+        }
+        reinterpret_cast<float*>(smem + kOffCoef + slot * (BN * 4))[key_local] = c;
+        if (lane == 0) reinterpret_cast<float2*>(smem + kOffBound + slot * 32)[bound_idx] = make_float2(cmax, cmin);
+        (void)t;
+    };
+
+    if (warp == 0) {
         // ================================================================ producer
+        // The whole warp runs the loop (warp-uniform waits); lane 0 issues the TMA
+        // copies, and in the kWindow form all lanes load the K scales of each
+        // cache tile (4 keys per lane) into the coefficient ring.
         if (lane == 0) {
             tma_prefetch_desc(&tm_q);
             tma_prefetch_desc(&tm_kcur);
             tma_prefetch_desc(&tm_vcur);
-            if (!kInt8) {
+            if (!kFill) {
                 tma_prefetch_desc(&tm_kc);
                 tma_prefetch_desc(&tm_vc);
             }
@@ -511,27 +608,44 @@ __global__ void __launch_bounds__(kInt8 ? 512 : 384, 1)
                 tma_load_3d(dst, &tm_q, 0, (qt0 + w) * BM, head, bar(B_QFULL));
                 tma_load_3d(dst + kHalfBytes, &tm_q, 64, (qt0 + w) * BM, head, bar(B_QFULL));
             }
-            // An INT8 cache has one filler for every stage, the converting warpgroup
-            // (codes for cache tiles, TMA for current-segment tiles): with a single
-            // filler in tile order every parity wait on the stage ring is exact.
-            if (!kInt8) {
-                int k_armed[kStages] = {-1, -1}, v_armed[kStages] = {-1, -1};
-                for (int i = 0; i < n; ++i) {
-                    const int st = i % kStages;
-                    const uint32_t free_ph = ((i / kStages) & 1) ^ 1;
-                    if (i >= kStages && !mbar_wait(bar(B_KEMPTY + st), free_ph, ctl)) break;
+        }
+        // kFused: one filler for every stage, the converting warpgroup (codes for
+        // cache tiles, TMA for current-segment tiles): with a single filler in
+        // tile order every parity wait on the stage ring is exact.
+        if (!kFill) {
+            int k_armed[kStages] = {-1, -1}, v_armed[kStages] = {-1, -1};
+            for (int i = 0; i < n; ++i) {
+                const int st = i % kStages;
+                const uint32_t free_ph = ((i / kStages) & 1) ^ 1;
+                if (i >= kStages && !mbar_wait_warp(bar(B_KEMPTY + st), free_ph, ctl)) break;
+                if (lane == 0)
                     load_k_tile(a, t_begin + i, head, sbase + kOffK + st * kTileBytes, bar(B_KFULL + st), &tm_kc,
                                 &tm_kcur);
-                    k_armed[st] = (i / kStages) & 1;
-                    if (i >= kStages && !mbar_wait(bar(B_VEMPTY + st), free_ph, ctl)) break;
+                k_armed[st] = (i / kStages) & 1;
+                if (i >= kStages && !mbar_wait_warp(bar(B_VEMPTY + st), free_ph, ctl)) break;
+                if (lane == 0)
                     load_v_tile(a, t_begin + i, head, sbase + kOffV + st * kTileBytes, bar(B_VFULL + st), &tm_vc,
                                 &tm_vcur);
-                    v_armed[st] = (i / kStages) & 1;
+                v_armed[st] = (i / kStages) & 1;
+                if (kInt8 && i < nci) {
+                    const uint32_t slot = static_cast<uint32_t>(i % kCoefSlots);
+                    if (i >= kCoefSlots && !mbar_wait_warp(bar(B_CEMPTY + slot), ((i / kCoefSlots) & 1) ^ 1, ctl))
+                        break;
+                    const int t = t_begin + i;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int key = t * BN + q * 32 + lane;
+                        const bool key_ok = key < a.nc;
+                        const float ks = key_ok ? __ldg(a.ksc + static_cast<int64_t>(head) * a.cap_tok + key) : 0.0f;
+                        put_coef(t, ks, key_ok, q * 32 + lane, slot, q);
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar(B_CFULL + slot));
                 }
-                drain_armed(k_armed, v_armed, bar(B_KFULL), bar(B_VFULL));
             }
+            if (lane == 0) drain_armed(k_armed, v_armed, bar(B_KFULL), bar(B_VFULL));
         }
-        } else if (warp == 1) {
+    } else if (warp == 1) {
         // ================================================================ MMA issuer
         // The whole warp runs the loop (warp-uniform waits and conditions) and
         // one elected lane issues each MMA and commit; MMAs issued by a single
@@ -609,9 +723,7 @@ __global__ void __launch_bounds__(kInt8 ? 512 : 384, 1)
         while (!mbar_try_wait(bar(B_DRAIN), 0)) {
             if (global_timer_ns() - t0 > NOMAS_WAIT_NS) break;
         }
-        }
-    } else if (warp < 12) {
-        regs_inc<Regs<kInt8>::kSoftmax>();
+    } else if (warp >= 4 && warp < 12) {
         // ================================================================ softmax
         const int w = (warp - 4) >> 2;
         const int quad = warp & 3;
@@ -632,19 +744,10 @@ __global__ void __launch_bounds__(kInt8 ? 512 : 384, 1)
                 if (!(ok = mbar_wait(bar(B_SFULL + w), i & 1, ctl))) break;
                 tc_fence_after();
                 const int vc = tile_valid(a, t);
-                // the whole S row into registers: the second half loads while the
-                // first half's maximum is taken
-                uint32_t s[128];
-                tmem_ld64_issue(t_s, s);
-                tmem_ld64_wait(s);
-                tmem_ld64_issue(t_s + 64, s + 64);
-                if (vc < BN) mask64(s, 0, vc);
-                float mx = max64(s, -INFINITY);
-                tmem_ld64_wait(s + 64);
-                if (vc < BN) mask64(s + 64, 64, vc);
-                mx = max64(s + 64, mx);
-                // bounds of the tile's scaled maximum: x_j = s_j * c_j with every c_j in
-                // [clo, chi], so max_j x_j lies in [lo, hi] below
+                const bool full = (vc == BN);
+                // pass 1: the tile's raw maximum; x_j = s_j * c_j with every c_j in
+                // [clo, chi], so the scaled maximum lies in [lo, hi] below
+                const float mx = full ? row_max<false>(t_s, vc) : row_max_masked(t_s, vc);
                 float chi = sl2, clo = sl2;
                 const float4* cf = nullptr;
                 if (coef) {
@@ -658,23 +761,31 @@ __global__ void __launch_bounds__(kInt8 ? 512 : 384, 1)
                 const float hi = mx >= 0.0f ? mx * chi : mx * clo;
                 const float lo = mx >= 0.0f ? mx * clo : mx * chi;
                 // the reference moves only when the tile may exceed it by more than the
-                // threshold; it moves to the upper bound when the bound is within the
-                // threshold of the true maximum, else to the exact maximum
+                // threshold: to the upper bound when that is within the threshold of
+                // the true maximum (always so without coefficients), else to the
+                // exact scaled maximum
                 const bool up = hi > m_ref + kRescaleThreshold;
-                float m_new = m_ref;
-                if (up) m_new = (coef && hi - lo > kRescaleThreshold) ? max_scaled(s, cf) : hi;
+                const bool exact = up && hi - lo > kRescaleThreshold;
+                float m_new = up ? hi : m_ref;
+                if (coef && __any_sync(0xFFFFFFFFu, exact)) {
+                    const float me = row_max_scaled(t_s, cf, vc);
+                    if (exact) m_new = me;
+                }
                 const float alpha = up ? ex2_approx(m_ref - m_new) : 1.0f; // 0 on the first tile
                 if (i > 0 && __any_sync(0xFFFFFFFFu, up)) rescale_o(t_o, alpha);
                 l *= alpha;
                 m_ref = m_new;
-                // P into TMEM, row sum in fp32
+                // pass 2: P into TMEM, row sum in fp32
                 if (coef) {
-                    l += exp_row<kExp2PolyPairsInt8, true>(s, cf, sl2, m_ref, t_s);
+                    l += full ? row_exp_store_full<kFill ? kExp2PolyPairsFused : kExp2PolyPairs, true>(t_s, cf, sl2,
+                                                                                                      m_ref)
+                              : row_exp_store_masked(t_s, cf, sl2, m_ref, vc);
                     __syncwarp();
                     if (lane == 0) mbar_arrive(bar(B_CEMPTY + slot));
                 } else {
-                    l += exp_row<kInt8 ? kExp2PolyPairsInt8 : kExp2PolyPairsBf16, false>(s, nullptr, sl2, m_ref,
-                                                                                        t_s);
+                    l += full ? row_exp_store_full<kFill ? kExp2PolyPairsFused : kExp2PolyPairs, false>(t_s, nullptr,
+                                                                                                       sl2, m_ref)
+                              : row_exp_store_masked(t_s, nullptr, sl2, m_ref, vc);
                 }
                 tmem_st_wait();
                 tc_fence_before();
@@ -720,8 +831,7 @@ __global__ void __launch_bounds__(kInt8 ? 512 : 384, 1)
                               a.lse ? a.lse + static_cast<int64_t>(head) * a.nq + qrow : nullptr);
             }
         }
-    } else if constexpr (kInt8) {
-        regs_dec<Regs<kInt8>::kFiller>();
+    } else if (kFill && warp >= 12) {
         // ================================================================ INT8 filler
         // Warp wq converts rows [32 wq, 32 wq + 32) of a cache tile; in step j a
         // warp covers rows 2j and 2j+1, 16 lanes per row, 8 codes per lane, so a
@@ -735,7 +845,6 @@ __global__ void __launch_bounds__(kInt8 ? 512 : 384, 1)
         const int half = lane >> 4;
         const int l16 = lane & 15;
         const bool elected = (f == 0);
-        const float sl2 = a.scale_log2;
         const uint32_t chunk_off = (l16 >> 3) * kHalfBytes;
         uint2 kb[16], vb[16];
         float ks_own = 0.0f, vs_own = 0.0f; // scales of key f of the tile whose codes are in kb / vb
@@ -808,20 +917,9 @@ __global__ void __launch_bounds__(kInt8 ? 512 : 384, 1)
                 const uint32_t slot = static_cast<uint32_t>(i % kCoefSlots);
                 convert_k(ktile);
                 if (next_cached) load_codes(a.kc8, t + 1, kb);
-                // the tile's K coefficients (scale_log2 * K scale; keys past the end
-                // get scale_log2 so that a masked score -inf stays -inf) and their
-                // range per warp, into the coefficient ring
+                // the tile's K coefficients into the coefficient ring
                 if (i >= kCoefSlots && !group_wait(bar(B_CEMPTY + slot), ((i / kCoefSlots) & 1) ^ 1)) break;
-                const float c = key_ok ? sl2 * ks_own : sl2;
-                float cmax = key_ok ? c : -INFINITY, cmin = key_ok ? c : INFINITY;
-#pragma unroll
-                for (int off = 16; off >= 1; off >>= 1) {
-                    cmax = fmaxf(cmax, __shfl_xor_sync(0xFFFFFFFFu, cmax, off));
-                    cmin = fminf(cmin, __shfl_xor_sync(0xFFFFFFFFu, cmin, off));
-                }
-                reinterpret_cast<float*>(smem + kOffCoef + slot * (BN * 4))[f] = c;
-                if (lane == 0)
-                    reinterpret_cast<float2*>(smem + kOffBound + slot * 32)[wq] = make_float2(cmax, cmin);
+                put_coef(t, ks_own, key_ok, f, slot, wq);
                 fence_proxy_async_smem();
                 named_bar_sync(1, 128);
                 if (elected) {
@@ -859,11 +957,46 @@ __global__ void __launch_bounds__(kInt8 ? 512 : 384, 1)
     }
 }
 
+// One work item = 16 codes (16 bytes) of one row of K or V; 8 items per row,
+// consecutive threads on consecutive items, so loads (128 B per row) and
+// stores (256 B per row) are fully coalesced. Grid-stride over both tensors.
+// K rows are written as their codes (exact in BF16; the K scale reaches the
+// scores through the attention kernel's coefficients), V rows as code * scale.
+__global__ void __launch_bounds__(512) dequant_window_kernel(const __grid_constant__ DequantArgs a) {
+    // Launched dependent on the RoPE prep kernel and overlapping it: it reads
+    // only the cache, which was complete before prep started. It lets the
+    // attention kernel launch early, and before it exits it waits for prep, so
+    // the attention kernel's wait on it covers prep too.
+    grid_dep_launch();
+    const uint32_t rows = static_cast<uint32_t>(a.heads) * static_cast<uint32_t>(a.nc); // per tensor, < 2^31
+    const uint32_t items = 2u * rows * 8u;                                              // < 2^32 by the host check
+    for (uint32_t it = blockIdx.x * blockDim.x + threadIdx.x; it < items; it += gridDim.x * blockDim.x) {
+        const uint32_t trow = it >> 3;
+        const uint32_t part = it & 7u;
+        const bool is_v = trow >= rows;
+        const uint32_t r = is_v ? trow - rows : trow;
+        const uint32_t head = fast_div(r, a.div_nc);
+        const uint32_t tok = r - head * static_cast<uint32_t>(a.nc);
+        const int64_t src_row = static_cast<int64_t>(head) * a.cap_tok + tok;
+        const uint4 w = __ldg(reinterpret_cast<const uint4*>((is_v ? a.vc : a.kc) + src_row * kD) + part);
+        uint4* dst = reinterpret_cast<uint4*>((is_v ? a.vd : a.kd) + static_cast<int64_t>(r) * kD) + 2 * part;
+        if (is_v) {
+            const float sc = __ldg(a.vs + src_row);
+            dst[0] = codes_to_bf16<true>(make_uint2(w.x, w.y), sc);
+            dst[1] = codes_to_bf16<true>(make_uint2(w.z, w.w), sc);
+        } else {
+            dst[0] = codes_to_bf16<false>(make_uint2(w.x, w.y), 0.0f);
+            dst[1] = codes_to_bf16<false>(make_uint2(w.z, w.w), 0.0f);
+        }
+    }
+    grid_dep_wait();
+}
+
 // The dynamic shared-memory limit of a kernel is an attribute of the kernel in
 // one device's context: it is raised once per device (and per kernel), the
 // first time that device launches it. Concurrent first launches may both set
 // it, which is harmless.
-template <bool kInt8>
+template <int kMode>
 cudaError_t ensure_smem_attr() {
     constexpr int kMaxDev = 64;
     static std::atomic<bool> done[kMaxDev];
@@ -871,27 +1004,40 @@ cudaError_t ensure_smem_attr() {
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < kMaxDev && done[dev].load(std::memory_order_acquire)) return cudaSuccess;
-    e = cudaFuncSetAttribute(attn_kernel<kInt8>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    e = cudaFuncSetAttribute(attn_kernel<kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e == cudaSuccess && dev >= 0 && dev < kMaxDev) done[dev].store(true, std::memory_order_release);
     return e;
 }
 
-} // namespace
-
-cudaError_t launch_attn(const AttnArgs& a, bool int8_cache, const CUtensorMap& tm_q, const CUtensorMap& tm_kcur,
+template <int kMode>
+cudaError_t launch_mode(const AttnArgs& a, const CUtensorMap& tm_q, const CUtensorMap& tm_kcur,
                         const CUtensorMap& tm_vcur, const CUtensorMap& tm_kc, const CUtensorMap& tm_vc,
                         cudaStream_t s) {
-    const int grid = a.heads * a.pairs * a.splits;
-    if (int8_cache) {
-        cudaError_t e = ensure_smem_attr<true>();
-        if (e != cudaSuccess) return e;
-        return launch_dependent(attn_kernel<true>, dim3(grid), dim3(512), kSmemBytes, s, a, tm_q, tm_kcur, tm_vcur,
-                                tm_kc, tm_vc);
-    }
-    cudaError_t e = ensure_smem_attr<false>();
+    cudaError_t e = ensure_smem_attr<kMode>();
     if (e != cudaSuccess) return e;
-    return launch_dependent(attn_kernel<false>, dim3(grid), dim3(384), kSmemBytes, s, a, tm_q, tm_kcur, tm_vcur,
-                            tm_kc, tm_vc);
+    return launch_dependent(attn_kernel<kMode>, dim3(a.heads * a.pairs * a.splits), dim3(kMode == kFused ? 512 : 384),
+                            kSmemBytes, s, a, tm_q, tm_kcur, tm_vcur, tm_kc, tm_vc);
+}
+
+} // namespace
+
+cudaError_t launch_dequant_window(const DequantArgs& a, cudaStream_t s) {
+    const uint64_t items = 2ull * static_cast<uint64_t>(a.heads) * static_cast<uint64_t>(a.nc) * 8ull;
+    if (items == 0) return cudaSuccess;
+    uint64_t blocks = (items + 511) / 512;
+    const uint64_t cap = 148ull * 4ull; // persistent: 4 blocks of 512 threads per SM
+    if (blocks > cap) blocks = cap;
+    return launch_dependent(dequant_window_kernel, dim3(static_cast<unsigned>(blocks)), dim3(512), 0, s, a);
+}
+
+cudaError_t launch_attn(const AttnArgs& a, AttnForm form, const CUtensorMap& tm_q, const CUtensorMap& tm_kcur,
+                        const CUtensorMap& tm_vcur, const CUtensorMap& tm_kc, const CUtensorMap& tm_vc,
+                        cudaStream_t s) {
+    switch (form) {
+    case AttnForm::kBf16Cache: return launch_mode<kBf16>(a, tm_q, tm_kcur, tm_vcur, tm_kc, tm_vc, s);
+    case AttnForm::kInt8Window: return launch_mode<kWindow>(a, tm_q, tm_kcur, tm_vcur, tm_kc, tm_vc, s);
+    default: return launch_mode<kFused>(a, tm_q, tm_kcur, tm_vcur, tm_kc, tm_vc, s);
+    }
 }
 
 } // namespace nomas

@@ -172,11 +172,12 @@ def test_workspace_plans_between_the_minimum_and_the_full_size():
     # and K (16 heads x 2896 tokens x 256 B each, rounded up to 256 bytes)
     qk = -(-16 * 2896 * 128 * 2 // 256) * 256
     assert low == 256 + 2 * qk
-    # the full plan adds the KV-split partials: per split, 16 heads x 12 Q-tile pairs x
-    # 256 rows of 128 fp32 values and an fp32 (max, sum) pair, and one counter per unit
-    part = full - low
+    # the full plan adds the BF16 copy of the INT8 window (2 x 16 heads x 15,840 tokens x
+    # 256 B) and the KV-split partials: per split, 16 heads x 12 Q-tile pairs x 256 rows
+    # of 128 fp32 values and an fp32 (max, sum) pair, and one counter per unit
+    copy = 2 * 16 * 18 * 880 * 256
     per_split = 16 * 12 * 256 * (128 * 4 + 8)
-    assert part >= 2 * per_split and part % 256 == 0
+    assert full - low >= copy + 2 * per_split and full % 256 == 0
     call = lambda wsb: nm.nomas_seg_attn(d, FAKE, FAKE, FAKE, 2048, 3, 256, FAKE, None, FAKE, wsb, None)
     assert call(low - 1) == nm.NOMAS_ERR_WORKSPACE
     # the minimum, the full size and any size in between (a plan with fewer splits)
