@@ -93,6 +93,12 @@ static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 
 enum { kBf16 = 0, kWindow = 1, kFused = 2 };
 
+// kWindow register budgets (setmaxnreg, one per warpgroup): the softmax
+// warpgroups hold a tile's 128 K coefficients in registers. The CTA is
+// launched with 384 threads x 168 registers; 128 x 72 + 256 x 216 is exactly that.
+constexpr uint32_t kWindowRegsCtl = 72, kWindowRegsSoftmax = 216;
+static_assert(128 * kWindowRegsCtl + 256 * kWindowRegsSoftmax == 384 * 168, "kWindow register split");
+
 // mbar_wait run by every lane of a converged warp; lane 0's outcome is
 // broadcast so the warp leaves the wait converged.
 __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, const WaitCtl& ctl) {
@@ -323,6 +329,49 @@ __device__ __forceinline__ float row_exp_store_full(uint32_t t_s, const float4* 
     tmem_ld32_wait(sb);
     exp_chunk<kPoly, kCoef>(sb, coef + 24, sl2x2, negm, acc, p);
     tmem_st16(t_s + 48, p);
+    const float2 t = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+    return t.x + t.y;
+}
+
+// Full-tile exp pass with the tile's coefficients held in registers (c[k] =
+// columns 4k .. 4k+3), in 16-column chunks: chunk q + 1 of S loads from TMEM
+// while chunk q is exponentiated.
+template <int kPoly>
+__device__ __forceinline__ void exp_chunk16(const uint32_t (&s)[16], const float4* c, float2 negm, float2 (&acc)[4],
+                                            uint32_t (&p)[8]) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        const float4 c4 = c[e >> 1];
+        const float2 cc = (e & 1) ? make_float2(c4.z, c4.w) : make_float2(c4.x, c4.y);
+        const float2 x = __ffma2_rn(make_float2(__uint_as_float(s[2 * e]), __uint_as_float(s[2 * e + 1])), cc, negm);
+        float2 y;
+        if ((e & 7) < kPoly)
+            y = exp2_fma2(x);
+        else
+            y = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+        acc[e & 3] = __fadd2_rn(acc[e & 3], y);
+        p[e] = pack_bf16x2(y.x, y.y);
+    }
+}
+template <int kPoly>
+__device__ __forceinline__ float row_exp_store_regcoef(uint32_t t_s, const float4 (&c)[32], float m) {
+    const float2 negm = make_float2(-m, -m);
+    float2 acc[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) acc[k] = make_float2(0.0f, 0.0f);
+    uint32_t sa[16], sb[16], p[8];
+    tmem_ld16_issue(t_s, sa);
+#pragma unroll
+    for (int q = 0; q < 8; q += 2) {
+        tmem_ld16_wait(sa);
+        tmem_ld16_issue(t_s + 16 * (q + 1), sb);
+        exp_chunk16<kPoly>(sa, c + 4 * q, negm, acc, p);
+        tmem_st8(t_s + 8 * q, p);
+        tmem_ld16_wait(sb);
+        if (q + 2 < 8) tmem_ld16_issue(t_s + 16 * (q + 2), sa);
+        exp_chunk16<kPoly>(sb, c + 4 * (q + 1), negm, acc, p);
+        tmem_st8(t_s + 8 * (q + 1), p);
+    }
     const float2 t = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
     return t.x + t.y;
 }
@@ -589,11 +638,10 @@ __global__ void __launch_bounds__(kMode == kFused ? 512 : 384, 1)
         (void)t;
     };
 
-    if (warp == 0) {
+    if (warp < 4) {
+      if constexpr (kMode == kWindow) regs_dec<kWindowRegsCtl>();
+      if (warp == 0) {
         // ================================================================ producer
-        // The whole warp runs the loop (warp-uniform waits); lane 0 issues the TMA
-        // copies, and in the kWindow form all lanes load the K scales of each
-        // cache tile (4 keys per lane) into the coefficient ring.
         if (lane == 0) {
             tma_prefetch_desc(&tm_q);
             tma_prefetch_desc(&tm_kcur);
@@ -608,44 +656,51 @@ __global__ void __launch_bounds__(kMode == kFused ? 512 : 384, 1)
                 tma_load_3d(dst, &tm_q, 0, (qt0 + w) * BM, head, bar(B_QFULL));
                 tma_load_3d(dst + kHalfBytes, &tm_q, 64, (qt0 + w) * BM, head, bar(B_QFULL));
             }
-        }
-        // kFused: one filler for every stage, the converting warpgroup (codes for
-        // cache tiles, TMA for current-segment tiles): with a single filler in
-        // tile order every parity wait on the stage ring is exact.
-        if (!kFill) {
-            int k_armed[kStages] = {-1, -1}, v_armed[kStages] = {-1, -1};
-            for (int i = 0; i < n; ++i) {
-                const int st = i % kStages;
-                const uint32_t free_ph = ((i / kStages) & 1) ^ 1;
-                if (i >= kStages && !mbar_wait_warp(bar(B_KEMPTY + st), free_ph, ctl)) break;
-                if (lane == 0)
+            // kFused: one filler for every stage, the converting warpgroup (codes for
+            // cache tiles, TMA for current-segment tiles): with a single filler in
+            // tile order every parity wait on the stage ring is exact.
+            if (!kFill) {
+                int k_armed[kStages] = {-1, -1}, v_armed[kStages] = {-1, -1};
+                for (int i = 0; i < n; ++i) {
+                    const int st = i % kStages;
+                    const uint32_t free_ph = ((i / kStages) & 1) ^ 1;
+                    if (i >= kStages && !mbar_wait(bar(B_KEMPTY + st), free_ph, ctl)) break;
                     load_k_tile(a, t_begin + i, head, sbase + kOffK + st * kTileBytes, bar(B_KFULL + st), &tm_kc,
                                 &tm_kcur);
-                k_armed[st] = (i / kStages) & 1;
-                if (i >= kStages && !mbar_wait_warp(bar(B_VEMPTY + st), free_ph, ctl)) break;
-                if (lane == 0)
+                    k_armed[st] = (i / kStages) & 1;
+                    if (i >= kStages && !mbar_wait(bar(B_VEMPTY + st), free_ph, ctl)) break;
                     load_v_tile(a, t_begin + i, head, sbase + kOffV + st * kTileBytes, bar(B_VFULL + st), &tm_vc,
                                 &tm_vcur);
-                v_armed[st] = (i / kStages) & 1;
-                if (kInt8 && i < nci) {
-                    const uint32_t slot = static_cast<uint32_t>(i % kCoefSlots);
-                    if (i >= kCoefSlots && !mbar_wait_warp(bar(B_CEMPTY + slot), ((i / kCoefSlots) & 1) ^ 1, ctl))
-                        break;
-                    const int t = t_begin + i;
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const int key = t * BN + q * 32 + lane;
-                        const bool key_ok = key < a.nc;
-                        const float ks = key_ok ? __ldg(a.ksc + static_cast<int64_t>(head) * a.cap_tok + key) : 0.0f;
-                        put_coef(t, ks, key_ok, q * 32 + lane, slot, q);
-                    }
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(bar(B_CFULL + slot));
+                    v_armed[st] = (i / kStages) & 1;
                 }
+                drain_armed(k_armed, v_armed, bar(B_KFULL), bar(B_VFULL));
             }
-            if (lane == 0) drain_armed(k_armed, v_armed, bar(B_KFULL), bar(B_VFULL));
         }
-    } else if (warp == 1) {
+      } else if (warp == 2) {
+        // ================================================================ K coefficients
+        // kWindow: the K scales of every cache tile (4 keys per lane) into the
+        // coefficient ring, off the TMA producer's path (their global loads
+        // would hold up the stage ring).
+        if (kMode == kWindow) {
+            for (int i = 0; i < nci; ++i) {
+                const uint32_t slot = static_cast<uint32_t>(i % kCoefSlots);
+                const int t = t_begin + i;
+                float ks[4];
+                bool ko[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int key = t * BN + q * 32 + lane;
+                    ko[q] = key < a.nc;
+                    ks[q] = ko[q] ? __ldg(a.ksc + static_cast<int64_t>(head) * a.cap_tok + key) : 0.0f;
+                }
+                if (i >= kCoefSlots && !mbar_wait_warp(bar(B_CEMPTY + slot), ((i / kCoefSlots) & 1) ^ 1, ctl)) break;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) put_coef(t, ks[q], ko[q], q * 32 + lane, slot, q);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(B_CFULL + slot));
+            }
+        }
+      } else if (warp == 1) {
         // ================================================================ MMA issuer
         // The whole warp runs the loop (warp-uniform waits and conditions) and
         // one elected lane issues each MMA and commit; MMAs issued by a single
@@ -723,7 +778,9 @@ __global__ void __launch_bounds__(kMode == kFused ? 512 : 384, 1)
         while (!mbar_try_wait(bar(B_DRAIN), 0)) {
             if (global_timer_ns() - t0 > NOMAS_WAIT_NS) break;
         }
-    } else if (warp >= 4 && warp < 12) {
+      }
+    } else if (warp < 12) {
+        if constexpr (kMode == kWindow) regs_inc<kWindowRegsSoftmax>();
         // ================================================================ softmax
         const int w = (warp - 4) >> 2;
         const int quad = warp & 3;
@@ -735,9 +792,25 @@ __global__ void __launch_bounds__(kMode == kFused ? 512 : 384, 1)
         float m_ref = -INFINITY; // reference max, log2 units
         float l = 0.0f;
         bool ok = true;
+        // kWindow: a full cache tile's 128 K coefficients in registers (creg), and
+        // the per-warp coefficient ranges of the tile (bnext), for the next tile
+        float4 creg[kMode == kWindow ? 32 : 1];
+        float4 bnext[2];
+        auto load_coefs = [&](int i) -> bool {
+            const uint32_t slot = static_cast<uint32_t>(i % kCoefSlots);
+            if (!mbar_wait(bar(B_CFULL + slot), (i / kCoefSlots) & 1, ctl)) return false;
+            const uint32_t bd = sbase + kOffBound + slot * 32;
+            bnext[0] = lds128_ordered(bd);
+            bnext[1] = lds128_ordered(bd + 16);
+            const uint32_t ca = sbase + kOffCoef + slot * (BN * 4);
+#pragma unroll
+            for (int k = 0; k < (kMode == kWindow ? 32 : 1); ++k) creg[k] = lds128_ordered(ca + 16 * k);
+            return true;
+        };
         if (active) {
             const float sl2 = a.scale_log2;
-            for (int i = 0; i < n; ++i) {
+            if (kMode == kWindow && nci > 0) ok = load_coefs(0);
+            for (int i = 0; ok && i < n; ++i) {
                 const int t = t_begin + i;
                 const bool coef = kInt8 && i < nci; // warp-uniform
                 const uint32_t slot = static_cast<uint32_t>(i % kCoefSlots);
@@ -745,18 +818,28 @@ __global__ void __launch_bounds__(kMode == kFused ? 512 : 384, 1)
                 tc_fence_after();
                 const int vc = tile_valid(a, t);
                 const bool full = (vc == BN);
+                float4 b0 = make_float4(sl2, sl2, sl2, sl2), b1 = b0;
+                const float4* cf = nullptr;
+                if (coef) {
+                    cf = reinterpret_cast<const float4*>(smem + kOffCoef + slot * (BN * 4));
+                    if (kMode == kWindow) {
+                        // loaded (after their CFULL wait) at the end of the previous tile
+                        b0 = bnext[0];
+                        b1 = bnext[1];
+                    } else {
+                        if (!(ok = mbar_wait(bar(B_CFULL + slot), (i / kCoefSlots) & 1, ctl))) break;
+                        const uint32_t bd = sbase + kOffBound + slot * 32;
+                        b0 = lds128_ordered(bd);
+                        b1 = lds128_ordered(bd + 16);
+                    }
+                }
                 // pass 1: the tile's raw maximum; x_j = s_j * c_j with every c_j in
                 // [clo, chi], so the scaled maximum lies in [lo, hi] below
                 const float mx = full ? row_max<false>(t_s, vc) : row_max_masked(t_s, vc);
                 float chi = sl2, clo = sl2;
-                const float4* cf = nullptr;
                 if (coef) {
-                    if (!(ok = mbar_wait(bar(B_CFULL + slot), (i / kCoefSlots) & 1, ctl))) break;
-                    const float4* bd = reinterpret_cast<const float4*>(smem + kOffBound + slot * 32);
-                    const float4 b0 = bd[0], b1 = bd[1];
                     chi = fmaxf(fmaxf(b0.x, b0.z), fmaxf(b1.x, b1.z));
                     clo = fminf(fminf(b0.y, b0.w), fminf(b1.y, b1.w));
-                    cf = reinterpret_cast<const float4*>(smem + kOffCoef + slot * (BN * 4));
                 }
                 const float hi = mx >= 0.0f ? mx * chi : mx * clo;
                 const float lo = mx >= 0.0f ? mx * clo : mx * chi;
@@ -777,9 +860,12 @@ __global__ void __launch_bounds__(kMode == kFused ? 512 : 384, 1)
                 m_ref = m_new;
                 // pass 2: P into TMEM, row sum in fp32
                 if (coef) {
-                    l += full ? row_exp_store_full<kFill ? kExp2PolyPairsFused : kExp2PolyPairs, true>(t_s, cf, sl2,
-                                                                                                      m_ref)
-                              : row_exp_store_masked(t_s, cf, sl2, m_ref, vc);
+                    if constexpr (kMode == kWindow)
+                        l += full ? row_exp_store_regcoef<kExp2PolyPairs>(t_s, creg, m_ref)
+                                  : row_exp_store_masked(t_s, cf, sl2, m_ref, vc);
+                    else
+                        l += full ? row_exp_store_full<kExp2PolyPairsFused, true>(t_s, cf, sl2, m_ref)
+                                  : row_exp_store_masked(t_s, cf, sl2, m_ref, vc);
                     __syncwarp();
                     if (lane == 0) mbar_arrive(bar(B_CEMPTY + slot));
                 } else {
@@ -791,6 +877,10 @@ __global__ void __launch_bounds__(kMode == kFused ? 512 : 384, 1)
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar(B_PFULL + w));
+                // kWindow: the next cache tile's coefficients, loaded now so that their
+                // shared-memory loads (which queue behind the tensor core's operand
+                // reads) complete while this warp waits for the next S
+                if (kMode == kWindow && i + 1 < nci && !(ok = load_coefs(i + 1))) break;
             }
             // ---- epilogue
             if (ok) ok = mbar_wait(bar(B_OFULL + w), 0, ctl);
