@@ -403,7 +403,7 @@ def run_extra(args, torch, nm, dev):
         flop_attn = 4.0 * 16 * HEAD_DIM * (3 * F + 256) * (18 * F + 3 * F + 256)
 
         # the finished segment's K/V of every layer come out of one forward pass, so all
-        # 54 layers are committed by one nomas_kv_commit_layers call (3 launches of <= 24 layers)
+        # 54 layers are committed by one nomas_kv_commit_layers call (one launch)
         kl, vl = [kseg] * layers, [vseg] * layers
 
         def turn():

@@ -146,7 +146,7 @@ int nomas_kv_commit(nomas_cache *c, const void *k, const void *v, int64_t token_
 
 /*
  * nomas_kv_commit_layers -- nomas_kv_commit of one finished segment into
- * n_layers per-layer caches at once (one launch per 24 layers instead of one
+ * n_layers per-layer caches at once (one launch per 128 layers instead of one
  * per layer). The pages describe the per-layer commit; batching the layers of
  * a model step is a service of this library.
  *   caches : host array of n_layers descriptors (distinct caches) that share

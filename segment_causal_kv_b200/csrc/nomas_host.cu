@@ -74,25 +74,17 @@ float2 rope_cs(double pos, double theta, int j, int d) {
     return make_float2(static_cast<float>(cos(ang)), static_cast<float>(sin(ang)));
 }
 
-// Spatial rows are fixed per (theta, grid); cache the last one per thread.
-struct HwCache {
-    float theta = -1.0f;
-    int gh = -1, gw = -1;
-    float2 hw[NOMAS_MAX_GRID_HW][kHWPairs];
-};
-
-void fill_hw(RopeTab& tab, float theta, int gh, int gw) {
-    thread_local HwCache hc;
-    if (hc.theta != theta || hc.gh != gh || hc.gw != gw) {
-        for (int r = 0; r < gh; ++r)
-            for (int j = 0; j < kHWPairs; ++j) hc.hw[r][j] = rope_cs(static_cast<double>(r), theta, j, 56);
-        for (int col = 0; col < gw; ++col)
-            for (int j = 0; j < kHWPairs; ++j) hc.hw[gh + col][j] = rope_cs(static_cast<double>(col), theta, j, 56);
-        hc.theta = theta;
-        hc.gh = gh;
-        hc.gw = gw;
-    }
-    std::memcpy(tab.hw, hc.hw, sizeof(float2) * kHWPairs * (gh + gw));
+// Device address of the spatial rows (grid rows, then grid columns) of a
+// configuration; computed here and uploaded by rope_hw_device on first use.
+int spatial_rows(float theta, int gh, int gw, const float2** dev) {
+    RopeHW h;
+    for (int r = 0; r < gh; ++r)
+        for (int j = 0; j < kHWPairs; ++j) h.hw[r][j] = rope_cs(static_cast<double>(r), theta, j, 56);
+    for (int col = 0; col < gw; ++col)
+        for (int j = 0; j < kHWPairs; ++j) h.hw[gh + col][j] = rope_cs(static_cast<double>(col), theta, j, 56);
+    const cudaError_t e = rope_hw_device(h, theta, gh, gw, dev);
+    if (e == cudaErrorMemoryAllocation) return NOMAS_ERR_ARG; // too many distinct configurations on this device
+    return e == cudaSuccess ? NOMAS_OK : NOMAS_ERR_CUDA;
 }
 
 void fill_t(RopeTab& tab, float theta, int64_t abs_frame0, int n_frames) {
@@ -294,8 +286,9 @@ static int commit_layers(nomas_cache* const* cs, const void* const* ks, const vo
 
     const int tpf = c->grid_h * c->grid_w;
     const int first = (W > 0 && n_frames > W) ? n_frames - W : 0;
+    const float2* hw = nullptr;
+    if ((rc = spatial_rows(c->rope_theta, c->grid_h, c->grid_w, &hw)) != NOMAS_OK) return rc;
     RopeTab tab;
-    fill_hw(tab, c->rope_theta, c->grid_h, c->grid_w);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     for (int f0 = first; f0 < n_frames; f0 += kMaxFramesPerLaunch) {
         const int nf = (n_frames - f0) < kMaxFramesPerLaunch ? (n_frames - f0) : kMaxFramesPerLaunch;
@@ -315,8 +308,9 @@ static int commit_layers(nomas_cache* const* cs, const void* const* ks, const vo
         a.div_heads = make_fastdiv(static_cast<uint32_t>(c->heads));
         a.div_tpf = make_fastdiv(static_cast<uint32_t>(tpf));
         a.div_gw = make_fastdiv(static_cast<uint32_t>(c->grid_w));
+        a.hw = hw;
         fill_t(tab, c->rope_theta, a.abs_frame0, nf);
-        // launches of equal size (54 layers: 3 x 18, not 24 + 24 + 6)
+        // launches of equal size when the layers need more than one
         const int n_launch = (n_layers + kMaxLayersPerLaunch - 1) / kMaxLayersPerLaunch;
         const int per_launch = (n_layers + n_launch - 1) / n_launch;
         for (int l0 = 0; l0 < n_layers; l0 += per_launch) {
@@ -493,8 +487,9 @@ int nomas_seg_attn(const nomas_cache* c, const void* q, const void* k, const voi
 
     // 1) RoPE + relayout of the current Q and K (video frames in chunks); the
     //    first launch also zeroes the split-KV arrival counters
+    const float2* hw = nullptr;
+    if ((rc = spatial_rows(c->rope_theta, c->grid_h, c->grid_w, &hw)) != NOMAS_OK) return rc;
     RopeTab tab;
-    fill_hw(tab, c->rope_theta, c->grid_h, c->grid_w);
     {
         int f0 = 0;
         do {
@@ -520,6 +515,7 @@ int nomas_seg_attn(const nomas_cache* c, const void* q, const void* k, const voi
             a.div_gw = make_fastdiv(static_cast<uint32_t>(c->grid_w));
             a.counters = counters;
             a.n_counters = (f0 == 0 && p.splits > 1) ? units : 0;
+            a.hw = hw;
             if (nf > 0) fill_t(tab, c->rope_theta, c->frames_committed + f0, nf);
             if (a.tok1 > a.tok0 && launch_prep(a, tab, s) != cudaSuccess) return NOMAS_ERR_CUDA;
             f0 += nf;

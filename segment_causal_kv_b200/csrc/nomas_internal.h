@@ -17,14 +17,26 @@ constexpr int kTPairs = 8;          // pairs of the t block (dims [0,16))
 constexpr int kHWPairs = 28;        // pairs of the h and w blocks (dims [16,72), [72,128))
 constexpr int kMaxFramesPerLaunch = 128;
 
-// RoPE cos/sin tables handed to kernels as launch arguments (read through the
-// constant bank). t rows are the latent frames one launch touches; hw rows
-// are grid rows [0, grid_h) followed by grid columns [grid_h, grid_h+grid_w).
+// RoPE cos/sin rows. The t rows of the latent frames one launch touches travel
+// as a launch argument (RopeTab). The spatial rows -- grid rows [0, grid_h)
+// followed by grid columns [grid_h, grid_h + grid_w) -- depend only on
+// (theta, grid) and are uploaded once per device and configuration into a
+// table in the library's device image (rope_hw_device); kernels read them
+// through L1. All values are computed on the host, so every launch sees the
+// same fp32 bits as the oracle's tables.
 struct RopeTab {
     float2 t[kMaxFramesPerLaunch][kTPairs];
+};
+struct RopeHW {
     float2 hw[NOMAS_MAX_GRID_HW][kHWPairs];
 };
-static_assert(sizeof(RopeTab) <= 30 * 1024, "RoPE table must fit the launch-argument limit");
+constexpr int kRopeConfigs = 16; // distinct (theta, grid) configurations per device
+
+// Device address of the spatial rows of configuration (theta, grid_h, grid_w)
+// on the current device, uploading `host` on the first use of that
+// configuration on that device (a blocking copy). cudaErrorMemoryAllocation
+// when kRopeConfigs configurations are already in use on the device.
+cudaError_t rope_hw_device(const RopeHW& host, float theta, int grid_h, int grid_w, const float2** dev);
 
 // Unsigned division by a runtime constant d for n < 2^31 (Granlund-Montgomery
 // round-up method): q = (umulhi(n, m) + n) >> s with s = ceil(log2 d) and
@@ -55,7 +67,7 @@ struct CommitLayer {
     float* cks;             // cache K scales (INT8 mode)
     float* cvs;
 };
-constexpr int kMaxLayersPerLaunch = 24; // keeps RopeTab + CommitArgs + CommitLayers under the 32 KB argument limit
+constexpr int kMaxLayersPerLaunch = 128; // RopeTab + CommitArgs + CommitLayers stay under the 32 KB argument limit
 struct CommitLayers {
     CommitLayer l[kMaxLayersPerLaunch];
 };
@@ -75,6 +87,7 @@ struct CommitArgs {
     int32_t head_group;     // heads of one token handled by one warp task (set by launch_commit)
     FastDiv div_groups;     // ceil(heads / head_group)
     FastDiv div_layer_tasks; // warp tasks per layer (set by launch_commit)
+    const float2* hw;       // spatial RoPE rows in device memory (rope_hw_device)
 };
 static_assert(sizeof(RopeTab) + sizeof(CommitArgs) + sizeof(CommitLayers) <= 32764,
               "commit launch arguments exceed the 32,764-byte limit");
@@ -92,6 +105,7 @@ struct PrepArgs {
     FastDiv div_heads, div_tpf, div_gw;
     unsigned* counters;     // split-KV arrival counters of the attention call, zeroed here
     int32_t n_counters;     // (by the launch with tok0 == 0 only)
+    const float2* hw;       // spatial RoPE rows in device memory (rope_hw_device)
 };
 
 struct AttnArgs {

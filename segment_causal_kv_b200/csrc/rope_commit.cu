@@ -9,7 +9,8 @@
 //
 // Work split: a half-warp owns one (token, head) row of 128 elements at a
 // time; each lane moves 16 bytes (8 BF16 = 4 RoPE pairs) with one 128-bit load
-// per tensor. The 16 lanes of a row fall into exactly one RoPE axis block each
+// per tensor, marked evict-first (each input byte is read once; kept out of
+// L1, it leaves room there for the RoPE rows every task reads). The 16 lanes of a row fall into exactly one RoPE axis block each
 // (lanes 0-1: t, 2-8: h, 9-15: w). In the commit a warp walks the heads of one
 // token (or of a group of its heads), so position, RoPE coefficients and ring
 // slot are set up once per token; every row write is one full 128-byte
@@ -25,6 +26,8 @@
 #include "nomas_ptx.cuh"
 
 #include <cuda_bf16.h>
+
+#include <mutex>
 
 namespace nomas {
 
@@ -43,25 +46,28 @@ __device__ __forceinline__ uint32_t rne_bf16x2(float lo, float hi) {
     return a | (b << 16);
 }
 
-// Stage the RoPE rows a block needs into shared memory.
-__device__ __forceinline__ void stage_tables(const RopeTab& tab, int n_t, int n_hw, float2* s_t, float2* s_hw) {
-    for (int i = threadIdx.x; i < n_t * kTPairs; i += blockDim.x) s_t[i] = tab.t[i / kTPairs][i % kTPairs];
-    for (int i = threadIdx.x; i < n_hw * kHWPairs; i += blockDim.x) s_hw[i] = tab.hw[i / kHWPairs][i % kHWPairs];
-    __syncthreads();
-}
+// Spatial RoPE rows of up to kRopeConfigs configurations per device, uploaded
+// once each by rope_hw_device (host code below).
+__device__ __align__(16) float2 g_rope_hw[kRopeConfigs][NOMAS_MAX_GRID_HW][kHWPairs];
 
 // cos/sin of the 4 pairs a lane owns (pairs 4*l .. 4*l+3 of the head): 32
-// contiguous bytes of one table row (t row for lanes 0-1, h row for 2-8, w row
-// for 9-15), read as two 16-byte loads from an address picked without
-// branching, so the half-warp's three axis groups do not diverge. Row starts
-// and in-row offsets are multiples of 32 bytes (t rows 64 B, h/w rows 224 B).
-__device__ __forceinline__ void lane_coeffs(int l, int frame, int hh, int ww, int grid_h, const float2* s_t,
-                                            const float2* s_hw, float2 (&cs)[4]) {
-    const float2* src = l < 2 ? s_t + frame * kTPairs + 4 * l
-                              : s_hw + (l < 9 ? hh * kHWPairs + (4 * l - kTPairs)
-                                              : (grid_h + ww) * kHWPairs + (4 * l - kTPairs - kHWPairs));
-    const float4 a = reinterpret_cast<const float4*>(src)[0];
-    const float4 b = reinterpret_cast<const float4*>(src)[1];
+// contiguous bytes of one table row -- the frame's t row (a launch argument)
+// for lanes 0-1, the h row for lanes 2-8, the w row for lanes 9-15 (device
+// memory, through L1: the rows of a half-warp are contiguous). Spatial rows
+// are 224 B and the in-row offsets multiples of 32 B, so both loads are
+// aligned 16-byte loads; lanes 0-1 load a valid spatial address too and keep
+// the t row, so the half-warp does not diverge around the loads.
+__device__ __forceinline__ void lane_coeffs(int l, int frame, int hh, int ww, int grid_h, const RopeTab& tab,
+                                            const float2* hw, float2 (&cs)[4]) {
+    const float2* src = hw + (l < 9 ? hh * kHWPairs + (l < 2 ? 0 : 4 * l - kTPairs)
+                                    : (grid_h + ww) * kHWPairs + (4 * l - kTPairs - kHWPairs));
+    float4 a = __ldg(reinterpret_cast<const float4*>(src));
+    float4 b = __ldg(reinterpret_cast<const float4*>(src) + 1);
+    if (l < 2) {
+        const float2* t = &tab.t[frame][4 * l];
+        a = make_float4(t[0].x, t[0].y, t[1].x, t[1].y);
+        b = make_float4(t[2].x, t[2].y, t[3].x, t[3].y);
+    }
     cs[0] = make_float2(a.x, a.y);
     cs[1] = make_float2(a.z, a.w);
     cs[2] = make_float2(b.x, b.y);
@@ -166,10 +172,6 @@ template <bool kGrouped, bool kInt8>
 __global__ void __launch_bounds__(kThreads) commit_kernel(const __grid_constant__ CommitArgs a,
                                                           const __grid_constant__ CommitLayers L,
                                                           const __grid_constant__ RopeTab tab) {
-    __shared__ __align__(16) float2 s_t[kMaxFramesPerLaunch * kTPairs];
-    __shared__ __align__(16) float2 s_hw[NOMAS_MAX_GRID_HW * kHWPairs];
-    stage_tables(tab, a.n_frames, a.grid_h + a.grid_w, s_t, s_hw);
-
     // A warp task is one layer's token and a group of `head_group` of its heads; the
     // two half-warps walk the group's heads h = g0 + half, g0 + half + 2, ...
     // (one (token, head) row per half-warp per step). Position, RoPE
@@ -206,8 +208,8 @@ __global__ void __launch_bounds__(kThreads) commit_kernel(const __grid_constant_
     if (task < tasks) {
         uint32_t ly, tk;
         const int h0 = min(task_token(task, ly, tk) + half, a.heads - 1); // out-of-range heads load a valid row, not stored
-        kx = __ldg(row_ptr(L.l[ly].k, tk, h0));
-        vx = __ldg(row_ptr(L.l[ly].v, tk, h0));
+        kx = __ldcs(row_ptr(L.l[ly].k, tk, h0));
+        vx = __ldcs(row_ptr(L.l[ly].v, tk, h0));
     }
     for (; task < tasks; task += warps) {
         uint32_t layer, tok;
@@ -219,7 +221,7 @@ __global__ void __launch_bounds__(kThreads) commit_kernel(const __grid_constant_
         const uint32_t hh = fast_div(rif, a.div_gw);
         const uint32_t ww = rif - hh * a.grid_w;
         float2 cs[4];
-        lane_coeffs(l, fi, hh, ww, a.grid_h, s_t, s_hw, cs);
+        lane_coeffs(l, fi, hh, ww, a.grid_h, tab, a.hw, cs);
         // slot of frame fi: ring slots advance with the frame (fi < window within a launch)
         int64_t slot;
         if (a.window > 0) {
@@ -237,13 +239,13 @@ __global__ void __launch_bounds__(kThreads) commit_kernel(const __grid_constant_
             uint4 kn = kx, vn = vx;
             if (j + 1 < steps) {
                 const int hn = min(h + 2, a.heads - 1);
-                kn = __ldg(row_ptr(P.k, tok, hn));
-                vn = __ldg(row_ptr(P.v, tok, hn));
+                kn = __ldcs(row_ptr(P.k, tok, hn));
+                vn = __ldcs(row_ptr(P.v, tok, hn));
             } else if (task_next < tasks) {
                 uint32_t ln, tn;
                 const int hn = min(task_token(task_next, ln, tn) + half, a.heads - 1);
-                kn = __ldg(row_ptr(L.l[ln].k, tn, hn));
-                vn = __ldg(row_ptr(L.l[ln].v, tn, hn));
+                kn = __ldcs(row_ptr(L.l[ln].k, tn, hn));
+                vn = __ldcs(row_ptr(L.l[ln].v, tn, hn));
             }
             float ky[8], vy[8];
             rotate8(kx, cs, ky);
@@ -283,12 +285,6 @@ __global__ void __launch_bounds__(kThreads) prep_kernel(const __grid_constant__ 
     grid_dep_launch();
     if (blockIdx.x == 0)
         for (int i = threadIdx.x; i < a.n_counters; i += blockDim.x) a.counters[i] = 0u;
-    __shared__ __align__(16) float2 s_t[kMaxFramesPerLaunch * kTPairs];
-    __shared__ __align__(16) float2 s_hw[NOMAS_MAX_GRID_HW * kHWPairs];
-    const int vid_lo = a.tok0 < a.nv ? a.tok0 : a.nv;
-    const int vid_hi = a.tok1 < a.nv ? a.tok1 : a.nv;
-    const int n_t = vid_hi > vid_lo ? (vid_hi - 1) / a.tpf - a.frame0 + 1 : 0;
-    stage_tables(tab, n_t, a.grid_h + a.grid_w, s_t, s_hw);
 
     const int lane = threadIdx.x & 31;
     const int l = lane & 15;
@@ -299,8 +295,8 @@ __global__ void __launch_bounds__(kThreads) prep_kernel(const __grid_constant__ 
         const int tok = a.tok0 + static_cast<int>(tq);
         const int h = static_cast<int>(r - tq * a.heads);
         const int64_t in_off = static_cast<int64_t>(tok) * a.token_stride + h * kD + l * 8;
-        const uint4 qx = __ldg(reinterpret_cast<const uint4*>(a.q + in_off));
-        const uint4 kx = __ldg(reinterpret_cast<const uint4*>(a.k + in_off));
+        const uint4 qx = __ldcs(reinterpret_cast<const uint4*>(a.q + in_off));
+        const uint4 kx = __ldcs(reinterpret_cast<const uint4*>(a.k + in_off));
         uint4 qo = qx, ko = kx;
         if (tok < a.nv) {
             const uint32_t fa = fast_div(static_cast<uint32_t>(tok), a.div_tpf);
@@ -308,7 +304,7 @@ __global__ void __launch_bounds__(kThreads) prep_kernel(const __grid_constant__ 
             const uint32_t rif = static_cast<uint32_t>(tok) - fa * a.tpf;
             const uint32_t hh = fast_div(rif, a.div_gw);
             float2 cs[4];
-            lane_coeffs(l, fi, hh, rif - hh * a.grid_w, a.grid_h, s_t, s_hw, cs);
+            lane_coeffs(l, fi, hh, rif - hh * a.grid_w, a.grid_h, tab, a.hw, cs);
             float qy[8], ky[8];
             rotate8(qx, cs, qy);
             rotate8(kx, cs, ky);
@@ -337,7 +333,7 @@ int grid_for(int64_t work_items, int items_per_block) {
             n = 148;
         return n;
     }();
-    // a persistent grid: every block stages the RoPE rows once and then loops
+    // a persistent grid: two blocks of 512 threads per SM, grid-stride loops
     int64_t want = (work_items + items_per_block - 1) / items_per_block;
     const int64_t cap = static_cast<int64_t>(sms) * 2;
     if (want > cap) want = cap;
@@ -346,6 +342,49 @@ int grid_for(int64_t work_items, int items_per_block) {
 }
 
 } // namespace
+
+// One table per (device, configuration): the host keeps which configuration
+// each slot of g_rope_hw holds on each device; a slot is written once (a
+// blocking copy, before its first kernel) and never changes afterwards.
+cudaError_t rope_hw_device(const RopeHW& host, float theta, int grid_h, int grid_w, const float2** dev) {
+    struct Key {
+        float theta;
+        int gh, gw;
+    };
+    struct Table {
+        std::mutex mu;
+        Key keys[64][kRopeConfigs];
+        int used[64] = {};
+        const float2* base[64] = {};
+    };
+    static Table t;
+    int d = 0;
+    cudaError_t e = cudaGetDevice(&d);
+    if (e != cudaSuccess) return e;
+    if (d < 0 || d >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(t.mu);
+    if (!t.base[d]) {
+        void* p = nullptr;
+        if ((e = cudaGetSymbolAddress(&p, g_rope_hw)) != cudaSuccess) return e;
+        t.base[d] = static_cast<const float2*>(p);
+    }
+    const size_t slot_elems = static_cast<size_t>(NOMAS_MAX_GRID_HW) * kHWPairs;
+    for (int i = 0; i < t.used[d]; ++i) {
+        const Key& k = t.keys[d][i];
+        if (k.theta == theta && k.gh == grid_h && k.gw == grid_w) {
+            *dev = t.base[d] + i * slot_elems;
+            return cudaSuccess;
+        }
+    }
+    if (t.used[d] == kRopeConfigs) return cudaErrorMemoryAllocation;
+    const int i = t.used[d];
+    const size_t bytes = sizeof(float2) * kHWPairs * static_cast<size_t>(grid_h + grid_w);
+    if ((e = cudaMemcpyToSymbol(g_rope_hw, host.hw, bytes, i * slot_elems * sizeof(float2))) != cudaSuccess) return e;
+    t.keys[d][i] = Key{theta, grid_h, grid_w};
+    t.used[d] = i + 1;
+    *dev = t.base[d] + i * slot_elems;
+    return cudaSuccess;
+}
 
 cudaError_t launch_commit(const CommitArgs& a_in, const CommitLayers& layers, const RopeTab& tab, cudaStream_t s) {
     // heads per warp task: all of a token's heads when there are enough tokens

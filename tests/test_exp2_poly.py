@@ -42,11 +42,12 @@ def exp2_fma2_emulated(x: np.ndarray, c: np.ndarray) -> np.ndarray:
 
 def test_kernel_constants_are_the_minimax_fit():
     pytest.importorskip("scipy")
-    sys.path.insert(0, CSRC)
+    tools = os.path.join(os.path.dirname(os.path.abspath(__file__)), "tools")
+    sys.path.insert(0, tools)
     try:
         import exp2_poly_fit
     finally:
-        sys.path.remove(CSRC)
+        sys.path.remove(tools)
     fitted, bound = exp2_poly_fit.fit()
     np.testing.assert_allclose(kernel_constants(), fitted, rtol=0, atol=2e-6)
     assert bound < 8e-5

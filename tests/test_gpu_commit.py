@@ -138,10 +138,11 @@ def test_commit_subnormal_tiny_and_large_rows():
     assert gpu.k[0, 0].abs().max().item() == 127
 
 
-@pytest.mark.parametrize("mode,n_layers", [("int8", 3), ("bf16", 3), ("int8", 26)])
+@pytest.mark.parametrize("mode,n_layers", [("int8", 3), ("bf16", 3), ("int8", 54), ("int8", 130)])
 def test_layered_commit_matches_per_layer_commits(mode, n_layers):
     """nomas_kv_commit_layers writes into every layer cache exactly what the
-    oracle's commit of that layer's segment writes (26 layers: two launches)."""
+    oracle's commit of that layer's segment writes (54 layers, the model's
+    depth: one launch; 130 layers: two launches)."""
     import segment_causal_kv_b200 as nm
     H, gh, gw, W = 2, 3, 5, 4
     geo = synth.Geometry(H, gh, gw)

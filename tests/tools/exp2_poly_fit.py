@@ -8,7 +8,7 @@ dense grid (variables c0..c3 and the bound E; |p(f_i) - 2^f_i| <= E 2^f_i),
 then rounds the coefficients to fp32 and reports the error of the fp32 Horner
 evaluation. Run it to reprint the constants:
 
-    python segment_causal_kv_b200/csrc/exp2_poly_fit.py
+    python tests/tools/exp2_poly_fit.py
 """
 
 from __future__ import annotations
