@@ -306,16 +306,30 @@ int nomas_device_status(void *workspace, void *stream);
  * nomas_seg_attn_workspace_min_bytes does, and a shape whose minimum exceeds
  * it is rejected with NOMAS_ERR_WORKSPACE before anything is enqueued. The
  * call allocates and frees nothing.
- * The first call on a device (with that device current) sets the array up:
- * it looks up its device address and clears its status header, a blocking
- * step; make that first call before any stream capture. All calls share the
- * one array and it keeps the last call's contents, so calls that overlap on
- * the GPU race with each other: order them (one stream, or events). Device
- * timeouts of this call are not reported through nomas_device_status.
+ * The first call in a CUDA context (with that context current) sets the
+ * array up: it looks up its device address and clears its status header
+ * with an asynchronous memset on `stream`, ahead of the call's kernels; make
+ * that first call before any stream capture. The set-up is redone in a new
+ * context (after a device reset, for instance). All calls share the one
+ * array and it keeps the last call's contents, so calls that overlap on the
+ * GPU race with each other: order them (one stream, or events), the first
+ * call included. Bounded device waits of this call that run out are reported
+ * by nomas_seg_attn_static_status, not by nomas_device_status.
  */
 #define NOMAS_STATIC_SCRATCH_BYTES (64u << 20)
 int nomas_seg_attn_static(const nomas_cache *c, const void *q, const void *k, const void *v, int64_t token_stride,
                           int32_t n_video_frames, int32_t n_text, void *out, float *lse, void *stream);
+
+/*
+ * nomas_seg_attn_static_status -- nomas_device_status for the fixed array of
+ * nomas_seg_attn_static in the current context: synchronise `stream`, read
+ * and clear the array's status header. Returns NOMAS_OK,
+ * NOMAS_ERR_DEVICE_TIMEOUT (a call's kernel abandoned a bounded wait; its
+ * outputs are invalid) or NOMAS_ERR_CUDA. It sets the array up first if no
+ * static call has run in this context yet. No counterpart on the pages: a
+ * service of this library, like the static call itself.
+ */
+int nomas_seg_attn_static_status(void *stream);
 
 /*
  * nomas_selftest_bounded_wait -- run the bounded-wait failure path of the

@@ -37,7 +37,8 @@ HEAD_DIM = 128
 EXPORTS = ("nomas_cache_reset", "nomas_kv_commit", "nomas_kv_commit_layers", "nomas_seg_attn_workspace_bytes",
            "nomas_seg_attn_workspace_min_bytes", "nomas_seg_attn",
            "nomas_device_status", "nomas_status_string", "nomas_seg_attn_static", "nomas_selftest_bounded_wait",
-           "nomas_kv_evicted_frames", "nomas_kv_archive_evicted", "nomas_camera_attn", "nomas_selftest_div127")
+           "nomas_kv_evicted_frames", "nomas_kv_archive_evicted", "nomas_camera_attn", "nomas_selftest_div127",
+           "nomas_seg_attn_static_status")
 NOMAS_STATIC_SCRATCH_BYTES = 64 << 20
 
 
@@ -100,6 +101,8 @@ def lib():
         L.nomas_seg_attn_static.restype = ctypes.c_int
         L.nomas_selftest_bounded_wait.argtypes = [P, P]
         L.nomas_selftest_bounded_wait.restype = ctypes.c_int
+        L.nomas_seg_attn_static_status.argtypes = [P]
+        L.nomas_seg_attn_static_status.restype = ctypes.c_int
         L.nomas_selftest_div127.argtypes = [P, P]
         L.nomas_selftest_div127.restype = ctypes.c_int
         L.nomas_kv_evicted_frames.argtypes = [D, I32, ctypes.POINTER(I32), ctypes.POINTER(I64)]
@@ -215,6 +218,11 @@ def nomas_seg_attn_static(desc: NomasCacheDesc, q_ptr: int, k_ptr: int, v_ptr: i
     """nomas_seg_attn with the library's static scratch, for callers that cannot allocate a workspace."""
     return lib().nomas_seg_attn_static(ctypes.byref(desc), q_ptr, k_ptr, v_ptr, token_stride, n_video_frames,
                                        n_text, out_ptr, lse_ptr, stream)
+
+
+def nomas_seg_attn_static_status(stream: int | None) -> int:
+    """Synchronise and read/clear the status header of nomas_seg_attn_static's fixed array."""
+    return lib().nomas_seg_attn_static_status(stream)
 
 
 def nomas_selftest_bounded_wait(ws_ptr: int, stream: int | None) -> int:

@@ -24,9 +24,11 @@ constexpr int kMaxFramesPerLaunch = 128;
 // table in the library's device image (rope_hw_device); kernels read them
 // through L1. All values are computed on the host, so every launch sees the
 // same fp32 bits as the oracle's tables.
-struct RopeTab {
-    float2 t[kMaxFramesPerLaunch][kTPairs];
+template <int kFrames>
+struct RopeTabT {
+    float2 t[kFrames][kTPairs];
 };
+using RopeTab = RopeTabT<kMaxFramesPerLaunch>;
 struct RopeHW {
     float2 hw[NOMAS_MAX_GRID_HW][kHWPairs];
 };
@@ -68,9 +70,16 @@ struct CommitLayer {
     float* cvs;
 };
 constexpr int kMaxLayersPerLaunch = 128; // RopeTab + CommitArgs + CommitLayers stay under the 32 KB argument limit
-struct CommitLayers {
-    CommitLayer l[kMaxLayersPerLaunch];
+template <int kLayers>
+struct CommitLayersT {
+    CommitLayer l[kLayers];
 };
+using CommitLayers = CommitLayersT<kMaxLayersPerLaunch>;
+// Launches of at most kSmallFrames frames and kSmallLayers layers (the common
+// few-frame commit of one layer, the RoPE prep of a short segment) carry
+// argument tables of that size: a launch's arguments are copied with it, and
+// the full-size tables would be ~14 KB for a few hundred bytes used.
+constexpr int kSmallFrames = 8, kSmallLayers = 8;
 
 struct CommitArgs {
     int32_t n_layers;       // layers of this launch (entries of CommitLayers)

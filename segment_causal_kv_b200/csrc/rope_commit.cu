@@ -57,7 +57,8 @@ __device__ __align__(16) float2 g_rope_hw[kRopeConfigs][NOMAS_MAX_GRID_HW][kHWPa
 // are 224 B and the in-row offsets multiples of 32 B, so both loads are
 // aligned 16-byte loads; lanes 0-1 load a valid spatial address too and keep
 // the t row, so the half-warp does not diverge around the loads.
-__device__ __forceinline__ void lane_coeffs(int l, int frame, int hh, int ww, int grid_h, const RopeTab& tab,
+template <class Tab>
+__device__ __forceinline__ void lane_coeffs(int l, int frame, int hh, int ww, int grid_h, const Tab& tab,
                                             const float2* hw, float2 (&cs)[4]) {
     const float2* src = hw + (l < 9 ? hh * kHWPairs + (l < 2 ? 0 : 4 * l - kTPairs)
                                     : (grid_h + ww) * kHWPairs + (4 * l - kTPairs - kHWPairs));
@@ -168,10 +169,10 @@ __device__ __forceinline__ uint2 quantize8(const float (&y)[8], float& scale_out
     return r;
 }
 
-template <bool kGrouped, bool kInt8>
+template <bool kGrouped, bool kInt8, int kF, int kL>
 __global__ void __launch_bounds__(kThreads) commit_kernel(const __grid_constant__ CommitArgs a,
-                                                          const __grid_constant__ CommitLayers L,
-                                                          const __grid_constant__ RopeTab tab) {
+                                                          const __grid_constant__ CommitLayersT<kL> L,
+                                                          const __grid_constant__ RopeTabT<kF> tab) {
     // A warp task is one layer's token and a group of `head_group` of its heads; the
     // two half-warps walk the group's heads h = g0 + half, g0 + half + 2, ...
     // (one (token, head) row per half-warp per step). Position, RoPE
@@ -278,8 +279,9 @@ __global__ void __launch_bounds__(kThreads) commit_kernel(const __grid_constant_
     }
 }
 
+template <int kF>
 __global__ void __launch_bounds__(kThreads) prep_kernel(const __grid_constant__ PrepArgs a,
-                                                        const __grid_constant__ RopeTab tab) {
+                                                        const __grid_constant__ RopeTabT<kF> tab) {
     // the attention kernel of the call (which waits for this one before it
     // reads anything) may start launching right away
     grid_dep_launch();
@@ -386,6 +388,18 @@ cudaError_t rope_hw_device(const RopeHW& host, float theta, int grid_h, int grid
     return cudaSuccess;
 }
 
+template <int kF, int kL>
+void commit_variant(const CommitArgs& a, int grid, const CommitLayersT<kL>& L, const RopeTabT<kF>& tab,
+                    cudaStream_t s) {
+    if (a.head_group < a.heads) {
+        if (a.int8_mode) commit_kernel<true, true, kF, kL><<<grid, kThreads, 0, s>>>(a, L, tab);
+        else commit_kernel<true, false, kF, kL><<<grid, kThreads, 0, s>>>(a, L, tab);
+    } else {
+        if (a.int8_mode) commit_kernel<false, true, kF, kL><<<grid, kThreads, 0, s>>>(a, L, tab);
+        else commit_kernel<false, false, kF, kL><<<grid, kThreads, 0, s>>>(a, L, tab);
+    }
+}
+
 cudaError_t launch_commit(const CommitArgs& a_in, const CommitLayers& layers, const RopeTab& tab, cudaStream_t s) {
     // heads per warp task: all of a token's heads when there are enough tokens
     // to give every resident warp several tasks, else halves of that, down to 2,
@@ -400,19 +414,31 @@ cudaError_t launch_commit(const CommitArgs& a_in, const CommitLayers& layers, co
     const int64_t layer_tasks = static_cast<int64_t>(a.n_frames) * a.tpf * a.div_groups.d;
     a.div_layer_tasks = make_fastdiv(static_cast<uint32_t>(layer_tasks));
     const int grid = grid_for(layer_tasks * a.n_layers, kThreads / 32);
-    if (hg < a.heads) {
-        if (a.int8_mode) commit_kernel<true, true><<<grid, kThreads, 0, s>>>(a, layers, tab);
-        else commit_kernel<true, false><<<grid, kThreads, 0, s>>>(a, layers, tab);
+    if (a.n_frames <= kSmallFrames && a.n_layers <= kSmallLayers) {
+        RopeTabT<kSmallFrames> t{};
+        CommitLayersT<kSmallLayers> L{};
+        for (int f = 0; f < a.n_frames; ++f)
+            for (int j = 0; j < kTPairs; ++j) t.t[f][j] = tab.t[f][j];
+        for (int i = 0; i < a.n_layers; ++i) L.l[i] = layers.l[i];
+        commit_variant(a, grid, L, t, s);
     } else {
-        if (a.int8_mode) commit_kernel<false, true><<<grid, kThreads, 0, s>>>(a, layers, tab);
-        else commit_kernel<false, false><<<grid, kThreads, 0, s>>>(a, layers, tab);
+        commit_variant(a, grid, layers, tab, s);
     }
     return cudaGetLastError();
 }
 
 cudaError_t launch_prep(const PrepArgs& a, const RopeTab& tab, cudaStream_t s) {
     const int64_t rows = static_cast<int64_t>(a.tok1 - a.tok0) * a.heads;
-    prep_kernel<<<grid_for(rows, kThreads / 16), kThreads, 0, s>>>(a, tab);
+    const int grid = grid_for(rows, kThreads / 16);
+    const int nv_frames = a.tok0 < a.nv ? (min(a.tok1, a.nv) - 1) / a.tpf - a.frame0 + 1 : 0;
+    if (nv_frames <= kSmallFrames) {
+        RopeTabT<kSmallFrames> t{};
+        for (int f = 0; f < nv_frames; ++f)
+            for (int j = 0; j < kTPairs; ++j) t.t[f][j] = tab.t[f][j];
+        prep_kernel<kSmallFrames><<<grid, kThreads, 0, s>>>(a, t);
+    } else {
+        prep_kernel<kMaxFramesPerLaunch><<<grid, kThreads, 0, s>>>(a, tab);
+    }
     return cudaGetLastError();
 }
 

@@ -68,6 +68,8 @@ def _check_static_equals_workspace_call(nm, cache, q, k, v, n_video_frames, n_te
         torch.cuda.synchronize()
         assert torch.equal(out, ref), call
         assert torch.equal(lse, ref_lse), call
+    # no bounded wait of the static calls ran out
+    assert nm.nomas_seg_attn_static_status(torch.cuda.current_stream().cuda_stream) == nm.NOMAS_OK
     return ref, ref_lse
 
 
