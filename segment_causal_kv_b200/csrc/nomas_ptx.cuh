@@ -362,21 +362,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return r;
 }
 
-// Per-warpgroup register budget (all four warps of a warpgroup execute the
-// same instruction): dec gives registers back to the CTA's pool, inc waits
-// until the pool holds enough. The counts of a kernel's warpgroups must add up
-// to at most the registers the CTA was launched with.
-template <uint32_t N>
-__device__ __forceinline__ void regs_dec() {
-    static_assert(N % 8 == 0 && N >= 24 && N <= 256, "setmaxnreg count");
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
-}
-template <uint32_t N>
-__device__ __forceinline__ void regs_inc() {
-    static_assert(N % 8 == 0 && N >= 24 && N <= 256, "setmaxnreg count");
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
-}
-
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }

@@ -93,12 +93,6 @@ static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 
 enum { kBf16 = 0, kWindow = 1, kFused = 2 };
 
-// kWindow register budgets (setmaxnreg, one per warpgroup): the softmax
-// warpgroups hold a tile's 128 K coefficients in registers. The CTA is
-// launched with 384 threads x 168 registers; 128 x 72 + 256 x 216 is exactly that.
-constexpr uint32_t kWindowRegsCtl = 72, kWindowRegsSoftmax = 216;
-static_assert(128 * kWindowRegsCtl + 256 * kWindowRegsSoftmax == 384 * 168, "kWindow register split");
-
 // mbar_wait run by every lane of a converged warp; lane 0's outcome is
 // broadcast so the warp leaves the wait converged.
 __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, const WaitCtl& ctl) {
@@ -222,6 +216,26 @@ __device__ __forceinline__ float row_max(uint32_t t_s, int vc) {
     return mx;
 }
 
+// row_max in 32-column pieces (fewer registers live: the kWindow softmax holds
+// its tile's 128 coefficients in registers meanwhile).
+__device__ __forceinline__ float row_max32(uint32_t t_s) {
+    float mx = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        uint32_t s[32];
+        tmem_ld32(t_s + c * 32, s);
+        float m[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) m[k] = mx;
+#pragma unroll
+        for (int e = 0; e < 32; e += 2)
+            m[(e >> 1) & 3] = max3(m[(e >> 1) & 3], __uint_as_float(s[e]), __uint_as_float(s[e + 1]));
+        mx = fmaxf(max3(m[0], m[1], m[2]), m[3]);
+        asm volatile("" : "+f"(mx));
+    }
+    return mx;
+}
+
 // Exact maximum of s_j * c_j over the valid columns of a row (used when the
 // cheap bound of a tile is too loose to serve as the reference: keys of very
 // different scales). Cold: run by a whole warp only when one of its rows needs it.
@@ -333,9 +347,10 @@ __device__ __forceinline__ float row_exp_store_full(uint32_t t_s, const float4* 
     return t.x + t.y;
 }
 
-// Full-tile exp pass with the tile's coefficients held in registers (c[k] =
-// columns 4k .. 4k+3), in 16-column chunks: chunk q + 1 of S loads from TMEM
-// while chunk q is exponentiated.
+// Full-tile exp pass with per-column coefficients read from shared memory, in
+// 16-column chunks (chunk q + 1 of S loads from TMEM while chunk q is
+// exponentiated): fewer registers live than the 32-column form, which with
+// its coefficients would not fit the softmax warps' registers.
 template <int kPoly>
 __device__ __forceinline__ void exp_chunk16(const uint32_t (&s)[16], const float4* c, float2 negm, float2 (&acc)[4],
                                             uint32_t (&p)[8]) {
@@ -354,7 +369,7 @@ __device__ __forceinline__ void exp_chunk16(const uint32_t (&s)[16], const float
     }
 }
 template <int kPoly>
-__device__ __forceinline__ float row_exp_store_regcoef(uint32_t t_s, const float4 (&c)[32], float m) {
+__device__ __forceinline__ float row_exp_store_coef16(uint32_t t_s, const float4* coef, float m) {
     const float2 negm = make_float2(-m, -m);
     float2 acc[4];
 #pragma unroll
@@ -365,11 +380,11 @@ __device__ __forceinline__ float row_exp_store_regcoef(uint32_t t_s, const float
     for (int q = 0; q < 8; q += 2) {
         tmem_ld16_wait(sa);
         tmem_ld16_issue(t_s + 16 * (q + 1), sb);
-        exp_chunk16<kPoly>(sa, c + 4 * q, negm, acc, p);
+        exp_chunk16<kPoly>(sa, coef + 4 * q, negm, acc, p);
         tmem_st8(t_s + 8 * q, p);
         tmem_ld16_wait(sb);
         if (q + 2 < 8) tmem_ld16_issue(t_s + 16 * (q + 2), sa);
-        exp_chunk16<kPoly>(sb, c + 4 * (q + 1), negm, acc, p);
+        exp_chunk16<kPoly>(sb, coef + 4 * (q + 1), negm, acc, p);
         tmem_st8(t_s + 8 * (q + 1), p);
     }
     const float2 t = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
@@ -639,7 +654,6 @@ __global__ void __launch_bounds__(kMode == kFused ? 512 : 384, 1)
     };
 
     if (warp < 4) {
-      if constexpr (kMode == kWindow) regs_dec<kWindowRegsCtl>();
       if (warp == 0) {
         // ================================================================ producer
         if (lane == 0) {
@@ -780,7 +794,6 @@ __global__ void __launch_bounds__(kMode == kFused ? 512 : 384, 1)
         }
       }
     } else if (warp < 12) {
-        if constexpr (kMode == kWindow) regs_inc<kWindowRegsSoftmax>();
         // ================================================================ softmax
         const int w = (warp - 4) >> 2;
         const int quad = warp & 3;
@@ -792,19 +805,16 @@ __global__ void __launch_bounds__(kMode == kFused ? 512 : 384, 1)
         float m_ref = -INFINITY; // reference max, log2 units
         float l = 0.0f;
         bool ok = true;
-        // kWindow: a full cache tile's 128 K coefficients in registers (creg), and
-        // the per-warp coefficient ranges of the tile (bnext), for the next tile
-        float4 creg[kMode == kWindow ? 32 : 1];
-        float4 bnext[2];
+        // kWindow: the coefficient range of the next cache tile, read (after its
+        // CFULL wait) at the end of the previous tile
+        float chi_next = 0.0f, clo_next = 0.0f;
         auto load_coefs = [&](int i) -> bool {
             const uint32_t slot = static_cast<uint32_t>(i % kCoefSlots);
             if (!mbar_wait(bar(B_CFULL + slot), (i / kCoefSlots) & 1, ctl)) return false;
             const uint32_t bd = sbase + kOffBound + slot * 32;
-            bnext[0] = lds128_ordered(bd);
-            bnext[1] = lds128_ordered(bd + 16);
-            const uint32_t ca = sbase + kOffCoef + slot * (BN * 4);
-#pragma unroll
-            for (int k = 0; k < (kMode == kWindow ? 32 : 1); ++k) creg[k] = lds128_ordered(ca + 16 * k);
+            const float4 b0 = lds128_ordered(bd), b1 = lds128_ordered(bd + 16);
+            chi_next = fmaxf(fmaxf(b0.x, b0.z), fmaxf(b1.x, b1.z));
+            clo_next = fminf(fminf(b0.y, b0.w), fminf(b1.y, b1.w));
             return true;
         };
         if (active) {
@@ -818,29 +828,27 @@ __global__ void __launch_bounds__(kMode == kFused ? 512 : 384, 1)
                 tc_fence_after();
                 const int vc = tile_valid(a, t);
                 const bool full = (vc == BN);
-                float4 b0 = make_float4(sl2, sl2, sl2, sl2), b1 = b0;
+                float chi = sl2, clo = sl2;
                 const float4* cf = nullptr;
                 if (coef) {
                     cf = reinterpret_cast<const float4*>(smem + kOffCoef + slot * (BN * 4));
                     if (kMode == kWindow) {
                         // loaded (after their CFULL wait) at the end of the previous tile
-                        b0 = bnext[0];
-                        b1 = bnext[1];
+                        chi = chi_next;
+                        clo = clo_next;
                     } else {
                         if (!(ok = mbar_wait(bar(B_CFULL + slot), (i / kCoefSlots) & 1, ctl))) break;
                         const uint32_t bd = sbase + kOffBound + slot * 32;
-                        b0 = lds128_ordered(bd);
-                        b1 = lds128_ordered(bd + 16);
+                        const float4 b0 = lds128_ordered(bd), b1 = lds128_ordered(bd + 16);
+                        chi = fmaxf(fmaxf(b0.x, b0.z), fmaxf(b1.x, b1.z));
+                        clo = fminf(fminf(b0.y, b0.w), fminf(b1.y, b1.w));
                     }
                 }
                 // pass 1: the tile's raw maximum; x_j = s_j * c_j with every c_j in
                 // [clo, chi], so the scaled maximum lies in [lo, hi] below
-                const float mx = full ? row_max<false>(t_s, vc) : row_max_masked(t_s, vc);
-                float chi = sl2, clo = sl2;
-                if (coef) {
-                    chi = fmaxf(fmaxf(b0.x, b0.z), fmaxf(b1.x, b1.z));
-                    clo = fminf(fminf(b0.y, b0.w), fminf(b1.y, b1.w));
-                }
+                const float mx = !full ? row_max_masked(t_s, vc)
+                                 : (kMode == kWindow && coef) ? row_max32(t_s)
+                                                               : row_max<false>(t_s, vc);
                 const float hi = mx >= 0.0f ? mx * chi : mx * clo;
                 const float lo = mx >= 0.0f ? mx * clo : mx * chi;
                 // the reference moves only when the tile may exceed it by more than the
@@ -861,7 +869,7 @@ __global__ void __launch_bounds__(kMode == kFused ? 512 : 384, 1)
                 // pass 2: P into TMEM, row sum in fp32
                 if (coef) {
                     if constexpr (kMode == kWindow)
-                        l += full ? row_exp_store_regcoef<kExp2PolyPairs>(t_s, creg, m_ref)
+                        l += full ? row_exp_store_coef16<kExp2PolyPairs>(t_s, cf, m_ref)
                                   : row_exp_store_masked(t_s, cf, sl2, m_ref, vc);
                     else
                         l += full ? row_exp_store_full<kExp2PolyPairsFused, true>(t_s, cf, sl2, m_ref)
