@@ -67,8 +67,8 @@ def parse():
     p.add_argument("--shard", default="replica", choices=["replica", "heads", "ulysses"],
                    help="how N > 1 ranks split the work (see the module docstring)")
     p.add_argument("--workload", default=WORKLOAD,
-                   help=f"{WORKLOAD} (default: the headline line), full_history_bf16, commit_72f_int8, "
-                        "history_sweep, layers54_turn, camera_xattn")
+                   help=f"{WORKLOAD} (default: the headline line), single_gpu_bf16_18f, full_history_bf16, "
+                        "commit_72f_int8, history_sweep, layers54_turn, camera_xattn")
     return p.parse_args()
 
 
@@ -413,6 +413,44 @@ def run_extra(args, torch, nm, dev):
                                     "sample": f"{len(rows)} query rows x 16 heads over all {nk} keys "
                                               f"(fp64 two-pass softmax), {dt:.1f} s, {fl / 1e9:.1f} GFLOP"}
         print(json.dumps(line), flush=True)
+        return 0
+    if args.workload == "single_gpu_bf16_18f":
+        # the headline shape (16 heads, 3 frames + 256 text over 18 history frames)
+        # with the history kept in BF16: the same attention without the INT8 form's
+        # window copy and K-scale coefficients
+        cache = nm.KVCache("bf16", 16, 22, 40, 0, 18, device=dev)
+        for s_ in range(6):
+            k, v = synth.history_kv(geo, 3, 1, s_)
+            cache.commit(to_dev(k), to_dev(v), 3, stream=stream)
+        q, k, v = (to_dev(x) for x in synth.segment_qkv(geo, 3, 256, 1, segment=6))
+        out = torch.empty_like(q)
+        ws = cache.workspace(3, 256)
+        nq, nk = 3 * F + 256, 18 * F + 3 * F + 256
+        flop = 4.0 * 16 * HEAD_DIM * nq * nk
+        for _ in range(W):
+            cache.seg_attn(q, k, v, 3, 256, out=out, workspace=ws, stream=stream)
+        ts = []
+        for _ in range(K):
+            flush.zero_()
+            a, b = device_events(torch, 2)
+            a.record(stream)
+            cache.seg_attn(q, k, v, 3, 256, out=out, workspace=ws, stream=stream)
+            b.record(stream)
+            b.synchronize()
+            ts.append(a.elapsed_time(b))
+        if cache.device_status(stream) != nm.NOMAS_OK:
+            raise RuntimeError("a kernel reported a timed-out wait")
+        ms = statistics.mean(ts)
+        tf = flop / (ms * 1e-3) / 1e12
+        peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+        print(json.dumps({"metric": "seg_attn_tflops_bf16_cache", "value": tf, "unit": "TFLOP/s", "ms_per_call": ms,
+                          "steps": K, "warmup": W, "higher_is_better": True,
+                          "config": {"workload": "single_gpu_bf16_18f", "heads": 16, "grid": [22, 40],
+                                     "history_frames": 18, "cache": "bf16", "nq": nq, "nk": nk, "flop_per_call": flop,
+                                     "l2": "flushed before each call"},
+                          "roofline": {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s",
+                                       "frac": tf / peak, "frac_of_nominal_2250": tf / 2250.0,
+                                       "peak_kind": f"bf16 dense GEMM, burst, {peak_src}"}}), flush=True)
         return 0
     if args.workload == "history_sweep":
         out_rows = []

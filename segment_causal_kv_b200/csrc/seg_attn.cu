@@ -352,8 +352,8 @@ __device__ __forceinline__ float row_exp_store_full(uint32_t t_s, const float4* 
 // exponentiated): fewer registers live than the 32-column form, which with
 // its coefficients would not fit the softmax warps' registers.
 template <int kPoly>
-__device__ __forceinline__ void exp_chunk16(const uint32_t (&s)[16], const float4* c, float2 negm, float2 (&acc)[4],
-                                            uint32_t (&p)[8]) {
+__device__ __forceinline__ void exp_chunk16(const uint32_t (&s)[16], const float4 (&c)[4], float2 negm,
+                                            float2 (&acc)[4], uint32_t (&p)[8]) {
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
         const float4 c4 = c[e >> 1];
@@ -368,6 +368,9 @@ __device__ __forceinline__ void exp_chunk16(const uint32_t (&s)[16], const float
         p[e] = pack_bf16x2(y.x, y.y);
     }
 }
+// The coefficients of chunk q + 1 are read together with its TMEM load, one
+// chunk ahead of their use: the TMEM waits order every memory access around
+// them, so a read issued after a wait would expose its full latency.
 template <int kPoly>
 __device__ __forceinline__ float row_exp_store_coef16(uint32_t t_s, const float4* coef, float m) {
     const float2 negm = make_float2(-m, -m);
@@ -375,16 +378,25 @@ __device__ __forceinline__ float row_exp_store_coef16(uint32_t t_s, const float4
 #pragma unroll
     for (int k = 0; k < 4; ++k) acc[k] = make_float2(0.0f, 0.0f);
     uint32_t sa[16], sb[16], p[8];
+    float4 ca[4], cb[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) ca[k] = coef[k];
     tmem_ld16_issue(t_s, sa);
 #pragma unroll
     for (int q = 0; q < 8; q += 2) {
         tmem_ld16_wait(sa);
         tmem_ld16_issue(t_s + 16 * (q + 1), sb);
-        exp_chunk16<kPoly>(sa, coef + 4 * q, negm, acc, p);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) cb[k] = coef[4 * (q + 1) + k];
+        exp_chunk16<kPoly>(sa, ca, negm, acc, p);
         tmem_st8(t_s + 8 * q, p);
         tmem_ld16_wait(sb);
-        if (q + 2 < 8) tmem_ld16_issue(t_s + 16 * (q + 2), sa);
-        exp_chunk16<kPoly>(sb, coef + 4 * (q + 1), negm, acc, p);
+        if (q + 2 < 8) {
+            tmem_ld16_issue(t_s + 16 * (q + 2), sa);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) ca[k] = coef[4 * (q + 2) + k];
+        }
+        exp_chunk16<kPoly>(sb, cb, negm, acc, p);
         tmem_st8(t_s + 8 * (q + 1), p);
     }
     const float2 t = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
