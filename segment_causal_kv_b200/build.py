@@ -15,7 +15,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 SOURCES = ["nomas_host.cu", "rope_commit.cu", "seg_attn.cu", "camera_attn.cu", "nomas_static.cu",
            "nomas_selftest.cu"]
-HEADERS = ["nomas_internal.h", "nomas_ptx.cuh"]
+HEADERS = ["nomas_internal.h", "nomas_ptx.cuh", "nomas_f16.cuh", "nomas_div127.cuh"]
 LIB = os.path.join(HERE, "libnomas.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

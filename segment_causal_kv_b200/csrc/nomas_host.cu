@@ -141,8 +141,8 @@ bool make_tmap(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint6
 struct Plan {
     int64_t tpf, nv, nq, nc;
     int tiles_c, tiles_q, pairs, splits, tiles_per_split;
-    bool window;  // INT8 cache read through a BF16 copy of its visible window
-    size_t off_qt, off_kt, off_po, off_pml, off_cnt, off_kd, off_vd;
+    bool window;  // INT8 cache read through an FP16 copy of its visible window
+    size_t off_qt, off_kt, off_te, off_qs, off_po, off_pml, off_cnt, off_kd, off_vd;
     size_t total; // workspace bytes of this plan
 };
 
@@ -170,14 +170,16 @@ void choose_splits(int units, int tiles, int max_splits, int& splits, int& tps) 
     }
 }
 
-// The window copy's dequantisation kernel indexes (tensor, row, 16-code part)
-// in 32 bits, with a few grid strides of headroom.
+// The window copy's dequantisation kernel counts its (tensor, head, tile)
+// tasks and the attention kernel its tiles in 32 bits.
 bool window_copy_fits(int heads, int64_t nc) { return static_cast<int64_t>(heads) * nc < (int64_t(1) << 27); }
 
-// Workspace layout of a plan: status header, rotated Q and K (head-major);
+// Workspace layout of a plan: status header, rotated Q and K (head-major; BF16,
+// or FP16 for an INT8 cache); for an INT8 cache the tile records
+// [heads][tiles_c + tiles_q] float4 and the Q row factors [heads][nq] fp32;
 // with splits > 1 the split partials [splits][units][32][256] float4, their
 // (max, sum) pairs [splits][units][256] and one arrival counter per unit; with
-// the window form the BF16 copy of the visible window, K then V [heads][nc][128].
+// the window form the FP16 copy of the visible window, K then V [heads][nc][128].
 Plan make_plan(const nomas_cache* c, int32_t n_video_frames, int32_t n_text, int max_splits, bool window) {
     Plan p{};
     p.tpf = static_cast<int64_t>(c->grid_h) * c->grid_w;
@@ -193,9 +195,12 @@ Plan make_plan(const nomas_cache* c, int32_t n_video_frames, int32_t n_text, int
     const size_t qk_bytes = static_cast<size_t>(c->heads) * p.nq * kD * 2;
     const size_t prow = static_cast<size_t>(p.splits) * units * 2 * kBM;
     const bool sp = p.splits > 1;
+    const bool int8 = c->mode == NOMAS_CACHE_INT8;
     p.off_qt = kWsHeader;
     p.off_kt = round_up(p.off_qt + qk_bytes, 256);
-    p.off_po = round_up(p.off_kt + qk_bytes, 256);
+    p.off_te = round_up(p.off_kt + qk_bytes, 256);
+    p.off_qs = round_up(p.off_te + (int8 ? static_cast<size_t>(c->heads) * (p.tiles_c + p.tiles_q) * 16 : 0), 256);
+    p.off_po = round_up(p.off_qs + (int8 ? static_cast<size_t>(c->heads) * p.nq * 4 : 0), 256);
     p.off_pml = p.off_po + (sp ? prow * kD * sizeof(float) : 0);
     p.off_cnt = round_up(p.off_pml + (sp ? prow * sizeof(float2) : 0), 256);
     p.off_kd = p.off_vd = p.total = round_up(p.off_cnt + (sp ? static_cast<size_t>(units) * sizeof(unsigned) : 0), 256);
@@ -216,9 +221,9 @@ bool window_form(const nomas_cache* c) {
 }
 
 // The fastest plan whose workspace fits in `bytes`: for an INT8 cache the
-// window form before the in-shared-memory form (it runs at about twice the
-// rate per KV tile), and within a form more splits before fewer (fewer need
-// less room: splits = 1 keeps no partials). False when nothing fits.
+// window form before the in-shared-memory form, and within a form more splits
+// before fewer (fewer need less room: splits = 1 keeps no partials). False
+// when nothing fits.
 bool fit_plan(const nomas_cache* c, int32_t n_video_frames, int32_t n_text, size_t bytes, Plan& out) {
     for (int form = window_form(c) ? 1 : 0; form >= 0; --form) {
         int cap = kMaxSplits;
@@ -483,10 +488,15 @@ int nomas_seg_attn(const nomas_cache* c, const void* q, const void* k, const voi
     uint16_t* qt = reinterpret_cast<uint16_t*>(ws + p.off_qt);
     uint16_t* kt = reinterpret_cast<uint16_t*>(ws + p.off_kt);
     unsigned* counters = reinterpret_cast<unsigned*>(ws + p.off_cnt);
+    float4* te = reinterpret_cast<float4*>(ws + p.off_te);
+    float* qs = reinterpret_cast<float*>(ws + p.off_qs);
     const int units = c->heads * p.pairs;
+    const bool int8 = c->mode == NOMAS_CACHE_INT8;
+    const int64_t cap_tok = static_cast<int64_t>(c->capacity_frames) * p.tpf;
 
     // 1) RoPE + relayout of the current Q and K (video frames in chunks); the
-    //    first launch also zeroes the split-KV arrival counters
+    //    first launch also zeroes the split-KV arrival counters and, for an
+    //    INT8 cache, writes the cache tiles' records
     const float2* hw = nullptr;
     if ((rc = spatial_rows(c->rope_theta, c->grid_h, c->grid_w, &hw)) != NOMAS_OK) return rc;
     RopeTab tab;
@@ -516,6 +526,17 @@ int nomas_seg_attn(const nomas_cache* c, const void* q, const void* k, const voi
             a.counters = counters;
             a.n_counters = (f0 == 0 && p.splits > 1) ? units : 0;
             a.hw = hw;
+            if (int8) {
+                a.te = te;
+                a.qs = qs;
+                a.ksc = c->k_scale;
+                a.vsc = c->v_scale;
+                a.cap_tok = cap_tok;
+                a.nc = static_cast<int32_t>(p.nc);
+                a.tiles_c = p.tiles_c;
+                a.tiles_q = p.tiles_q;
+                a.te_cache_tasks = f0 == 0 ? c->heads * p.tiles_c : 0;
+            }
             if (nf > 0) fill_t(tab, c->rope_theta, c->frames_committed + f0, nf);
             if (a.tok1 > a.tok0 && launch_prep(a, tab, s) != cudaSuccess) return NOMAS_ERR_CUDA;
             f0 += nf;
@@ -523,22 +544,21 @@ int nomas_seg_attn(const nomas_cache* c, const void* q, const void* k, const voi
         } while (true);
     }
 
-    // 2) an INT8 window is dequantised once into its BF16 copy (window form)
-    const bool int8 = c->mode == NOMAS_CACHE_INT8;
-    const int64_t cap_tok = static_cast<int64_t>(c->capacity_frames) * p.tpf;
+    // 2) an INT8 window is dequantised once into its FP16 copy (window form)
     uint16_t* kd = reinterpret_cast<uint16_t*>(ws + p.off_kd);
     uint16_t* vd = reinterpret_cast<uint16_t*>(ws + p.off_vd);
     if (p.window) {
         DequantArgs d{};
         d.kc = static_cast<const int8_t*>(c->k);
         d.vc = static_cast<const int8_t*>(c->v);
+        d.ks = c->k_scale;
         d.vs = c->v_scale;
         d.kd = kd;
         d.vd = vd;
         d.cap_tok = cap_tok;
         d.nc = static_cast<int32_t>(p.nc);
         d.heads = c->heads;
-        d.div_nc = make_fastdiv(static_cast<uint32_t>(p.nc));
+        d.tiles_c = p.tiles_c;
         if (launch_dequant_window(d, s) != cudaSuccess) return NOMAS_ERR_CUDA;
     }
 
@@ -583,6 +603,8 @@ int nomas_seg_attn(const nomas_cache* c, const void* q, const void* k, const voi
     a.counters = counters;
     a.err = reinterpret_cast<unsigned*>(ws);
     a.scale_log2 = static_cast<float>(1.4426950408889634 / sqrt(static_cast<double>(kD)));
+    a.te = int8 ? te : nullptr;
+    a.qs = int8 ? qs : nullptr;
     const AttnForm form = !int8 ? AttnForm::kBf16Cache : p.window ? AttnForm::kInt8Window : AttnForm::kInt8Fused;
     if (launch_attn(a, form, tm_q, tm_kcur, tm_vcur, tm_kc, tm_vc, s) != cudaSuccess) return NOMAS_ERR_CUDA;
     return NOMAS_OK;

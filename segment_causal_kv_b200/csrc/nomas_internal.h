@@ -115,6 +115,14 @@ struct PrepArgs {
     unsigned* counters;     // split-KV arrival counters of the attention call, zeroed here
     int32_t n_counters;     // (by the launch with tok0 == 0 only)
     const float2* hw;       // spatial RoPE rows in device memory (rope_hw_device)
+    // INT8 caches (FP16 operands, nomas_f16.cuh); null te for a BF16 cache
+    float4* te;             // [heads][tiles_c + tiles_q] tile records
+    float* qs;              // [heads][nq] 2^a_i of each Q row
+    const float* ksc;       // cache K / V scales [heads][cap_tok]
+    const float* vsc;
+    int64_t cap_tok;
+    int32_t nc, tiles_c, tiles_q;
+    int32_t te_cache_tasks; // heads * tiles_c on the launch with tok0 == 0, else 0
 };
 
 struct AttnArgs {
@@ -138,27 +146,30 @@ struct AttnArgs {
     unsigned* counters;     // splits > 1: [units] arrivals; the last CTA of a unit merges the splits
     unsigned* err;          // workspace status word
     float scale_log2;       // log2(e) / sqrt(128)
+    const float4* te;       // INT8: [heads][tiles_c + tiles_q] tile records (2^b, 2^-b, c, 2^-c)
+    const float* qs;        // INT8: [heads][nq] 2^a_i of each FP16 Q row
 };
 
-// Dequantisation of an INT8 cache's visible window into a BF16 copy, once per
+// Dequantisation of an INT8 cache's visible window into an FP16 copy, once per
 // attention call: rows [0, nc) of every head, written head-major
-// [heads][nc][128]. K rows are the codes themselves (exact in BF16; the K scale
-// is applied to the scores by the attention kernel), V rows code * scale
-// rounded to BF16 (the values the in-shared-memory conversion produces).
+// [heads][nc][128], each 128-key tile as code * RN16(scale * 2^-e) with the
+// tile's exponent e (nomas_f16.cuh) -- the values the in-shared-memory
+// conversion produces.
 struct DequantArgs {
     const int8_t* kc;
     const int8_t* vc;
+    const float* ks;
     const float* vs;
     uint16_t* kd;
     uint16_t* vd;
     int64_t cap_tok; // token capacity of one head's slab in the cache
     int32_t nc;      // visible tokens per head
     int32_t heads;
-    FastDiv div_nc;
+    int32_t tiles_c; // ceil(nc / 128)
 };
 
 // Forms of the attention kernel: a BF16 cache; an INT8 cache read through its
-// dequantised window copy; an INT8 cache converted in shared memory.
+// FP16 window copy; an INT8 cache converted to FP16 in shared memory.
 enum class AttnForm { kBf16Cache, kInt8Window, kInt8Fused };
 
 // Per-latent-frame camera cross-attention: rows are (video token, head) pairs,

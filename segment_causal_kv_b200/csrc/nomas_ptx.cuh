@@ -338,11 +338,12 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes
 }
 constexpr uint32_t kSwizzle128B = 2;
 
-// Instruction descriptor for kind::f16 with BF16 A/B and fp32 D.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_major, bool b_mn_major) {
+// Instruction descriptor for kind::f16 with fp32 D and A/B both BF16 (or,
+// with f16, both FP16: one MMA never mixes the two).
+__host__ __device__ constexpr uint32_t idesc_f32(int M, int N, bool a_mn_major, bool b_mn_major, bool f16) {
     return (1u << 4)                                 // D format: f32
-           | (1u << 7)                               // A format: bf16
-           | (1u << 10)                              // B format: bf16
+           | ((f16 ? 0u : 1u) << 7)                  // A format: f16 / bf16
+           | ((f16 ? 0u : 1u) << 10)                 // B format: f16 / bf16
            | ((a_mn_major ? 1u : 0u) << 15)          // A major
            | ((b_mn_major ? 1u : 0u) << 16)          // B major
            | ((static_cast<uint32_t>(N) >> 3) << 17) // N / 8
@@ -360,6 +361,28 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     uint32_t r;
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
     return r;
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// Per-warpgroup register budget (all four warps of a warpgroup execute the
+// same instruction): dec gives registers back to the CTA's pool, inc waits
+// until the pool holds enough. The counts of a kernel's warpgroups must add up
+// to at most the registers the CTA was launched with (threads x registers per
+// thread at launch), or an inc waits for ever.
+template <uint32_t N>
+__device__ __forceinline__ void regs_dec() {
+    static_assert(N % 8 == 0 && N >= 24 && N <= 256, "setmaxnreg count");
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_inc() {
+    static_assert(N % 8 == 0 && N >= 24 && N <= 256, "setmaxnreg count");
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {

@@ -22,6 +22,7 @@
 // use the _rn intrinsics (no contraction freedom), the scale is an IEEE
 // division absmax / 127, codes are round-half-even of an IEEE division.
 #include "nomas_div127.cuh"
+#include "nomas_f16.cuh"
 #include "nomas_internal.h"
 #include "nomas_ptx.cuh"
 
@@ -325,6 +326,139 @@ __global__ void __launch_bounds__(kThreads) prep_kernel(const __grid_constant__ 
     }
 }
 
+// INT8 caches: RoPE of Q and K in fp32 to FP16 operands with power-of-two
+// exponents (nomas_f16.cuh), and every tile record of the attention call.
+// A block takes one (128-token tile, head) task at a time; half-warp g of the
+// block owns rows g, g + 32, g + 64, g + 96 of the tile. Each Q row gets its
+// own exponent (a half-warp reduction); the K rows stay in registers until the
+// block has the tile's maximum, then go out with the tile's exponent. Launch
+// chunks start at multiples of 128 frames, so a tile never spans two launches.
+// The launch with tok0 == 0 also writes the records of the cache tiles (a warp
+// per tile: the maxima of its 128 K and V scales).
+template <int kF>
+__global__ void __launch_bounds__(kThreads) prep16_kernel(const __grid_constant__ PrepArgs a,
+                                                          const __grid_constant__ RopeTabT<kF> tab) {
+    grid_dep_launch();
+    if (blockIdx.x == 0)
+        for (int i = threadIdx.x; i < a.n_counters; i += blockDim.x) a.counters[i] = 0u;
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const int ttot = a.tiles_c + a.tiles_q;
+
+    // ---- cache tile records
+    const int nwarps = gridDim.x * (kThreads / 32);
+    for (int task = blockIdx.x * (kThreads / 32) + warp; task < a.te_cache_tasks; task += nwarps) {
+        const int h = task / a.tiles_c;
+        const int T = task - h * a.tiles_c;
+        float mk = 0.0f, mv = 0.0f;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int key = T * 128 + q * 32 + lane;
+            if (key < a.nc) {
+                const int64_t g = static_cast<int64_t>(h) * a.cap_tok + key;
+                mk = fmaxf(mk, __ldg(a.ksc + g));
+                mv = fmaxf(mv, __ldg(a.vsc + g));
+            }
+        }
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) {
+            mk = fmaxf(mk, __shfl_xor_sync(0xFFFFFFFFu, mk, off));
+            mv = fmaxf(mv, __shfl_xor_sync(0xFFFFFFFFu, mv, off));
+        }
+        if (lane == 0)
+            a.te[static_cast<int64_t>(h) * ttot + T] =
+                tile_record(pow2_exponent(mk, kTopCode), pow2_exponent(mv, kTopCode));
+    }
+
+    // ---- current tiles
+    __shared__ float red[kThreads / 32];
+    const int l = lane & 15;
+    const int g = threadIdx.x >> 4;
+    const int T0 = a.tok0 / 128;
+    const int T1 = (a.tok1 + 127) / 128;
+    const int tasks = (T1 - T0) * a.heads;
+    for (int task = blockIdx.x; task < tasks; task += gridDim.x) {
+        const int T = T0 + task / a.heads;
+        const int h = task - (task / a.heads) * a.heads;
+        uint4 qx[4], kx[4];
+#pragma unroll
+        for (int rr = 0; rr < 4; ++rr) {
+            const int tok = T * 128 + g + 32 * rr;
+            qx[rr] = kx[rr] = make_uint4(0u, 0u, 0u, 0u);
+            if (tok < a.tok1) {
+                const int64_t in_off = static_cast<int64_t>(tok) * a.token_stride + h * kD + l * 8;
+                qx[rr] = __ldcs(reinterpret_cast<const uint4*>(a.q + in_off));
+                kx[rr] = __ldcs(reinterpret_cast<const uint4*>(a.k + in_off));
+            }
+        }
+        float ky[4][8];
+        float kmax = 0.0f;
+#pragma unroll
+        for (int rr = 0; rr < 4; ++rr) {
+            const int tok = T * 128 + g + 32 * rr;
+            float qy[8];
+            if (tok < a.nv && tok < a.tok1) {
+                const uint32_t fa = fast_div(static_cast<uint32_t>(tok), a.div_tpf);
+                const int fi = static_cast<int>(fa) - a.frame0;
+                const uint32_t rif = static_cast<uint32_t>(tok) - fa * a.tpf;
+                const uint32_t hh = fast_div(rif, a.div_gw);
+                float2 cs[4];
+                lane_coeffs(l, fi, hh, rif - hh * a.grid_w, a.grid_h, tab, a.hw, cs);
+                rotate8(qx[rr], cs, qy);
+                rotate8(kx[rr], cs, ky[rr]);
+            } else {
+                const uint32_t wq[4] = {qx[rr].x, qx[rr].y, qx[rr].z, qx[rr].w};
+                const uint32_t wk[4] = {kx[rr].x, kx[rr].y, kx[rr].z, kx[rr].w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    qy[2 * i] = bf16lo(wq[i]);
+                    qy[2 * i + 1] = bf16hi(wq[i]);
+                    ky[rr][2 * i] = bf16lo(wk[i]);
+                    ky[rr][2 * i + 1] = bf16hi(wk[i]);
+                }
+            }
+            float qm = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                qm = fmaxf(qm, fabsf(qy[i]));
+                kmax = fmaxf(kmax, fabsf(ky[rr][i]));
+            }
+#pragma unroll
+            for (int off = 8; off >= 1; off >>= 1) qm = fmaxf(qm, __shfl_xor_sync(0xFFFFFFFFu, qm, off));
+            if (tok < a.tok1) {
+                const int ea = pow2_exponent(qm, kTopFloat);
+                const float f = exp2_int(-ea);
+                const int64_t out_off = (static_cast<int64_t>(h) * a.nq + tok) * kD + l * 8;
+                *reinterpret_cast<uint4*>(a.qt + out_off) =
+                    make_uint4(pack_f16x2(qy[0] * f, qy[1] * f), pack_f16x2(qy[2] * f, qy[3] * f),
+                               pack_f16x2(qy[4] * f, qy[5] * f), pack_f16x2(qy[6] * f, qy[7] * f));
+                if (l == 0) a.qs[static_cast<int64_t>(h) * a.nq + tok] = exp2_int(ea);
+            }
+        }
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) kmax = fmaxf(kmax, __shfl_xor_sync(0xFFFFFFFFu, kmax, off));
+        if (lane == 0) red[warp] = kmax;
+        __syncthreads();
+        float tmax = red[0];
+#pragma unroll
+        for (int i = 1; i < kThreads / 32; ++i) tmax = fmaxf(tmax, red[i]);
+        const int eb = pow2_exponent(tmax, kTopFloat);
+        const float f = exp2_int(-eb);
+#pragma unroll
+        for (int rr = 0; rr < 4; ++rr) {
+            const int tok = T * 128 + g + 32 * rr;
+            if (tok < a.tok1) {
+                const int64_t out_off = (static_cast<int64_t>(h) * a.nq + tok) * kD + l * 8;
+                *reinterpret_cast<uint4*>(a.kt + out_off) = make_uint4(
+                    pack_f16x2(ky[rr][0] * f, ky[rr][1] * f), pack_f16x2(ky[rr][2] * f, ky[rr][3] * f),
+                    pack_f16x2(ky[rr][4] * f, ky[rr][5] * f), pack_f16x2(ky[rr][6] * f, ky[rr][7] * f));
+            }
+        }
+        if (threadIdx.x == 0) a.te[static_cast<int64_t>(h) * ttot + a.tiles_c + T] = tile_record(eb, 0);
+        __syncthreads(); // red[] is reused by the next task
+    }
+}
+
 int grid_for(int64_t work_items, int items_per_block) {
     // SM count of the first device that launches (every device of this library is a B200);
     // a function-local static is initialised once, thread-safely
@@ -429,15 +563,22 @@ cudaError_t launch_commit(const CommitArgs& a_in, const CommitLayers& layers, co
 
 cudaError_t launch_prep(const PrepArgs& a, const RopeTab& tab, cudaStream_t s) {
     const int64_t rows = static_cast<int64_t>(a.tok1 - a.tok0) * a.heads;
-    const int grid = grid_for(rows, kThreads / 16);
+    const bool f16 = a.te != nullptr;
+    // FP16 form: one block per (tile, head) task, or enough blocks to give the
+    // cache tile records a warp each
+    const int64_t tasks = static_cast<int64_t>((a.tok1 + 127) / 128 - a.tok0 / 128) * a.heads;
+    int grid = f16 ? grid_for(tasks > 0 ? tasks : 1, 1) : grid_for(rows, kThreads / 16);
+    if (f16 && a.te_cache_tasks > 0) grid = max(grid, grid_for(a.te_cache_tasks, kThreads / 32));
     const int nv_frames = a.tok0 < a.nv ? (min(a.tok1, a.nv) - 1) / a.tpf - a.frame0 + 1 : 0;
     if (nv_frames <= kSmallFrames) {
         RopeTabT<kSmallFrames> t{};
         for (int f = 0; f < nv_frames; ++f)
             for (int j = 0; j < kTPairs; ++j) t.t[f][j] = tab.t[f][j];
-        prep_kernel<kSmallFrames><<<grid, kThreads, 0, s>>>(a, t);
+        if (f16) prep16_kernel<kSmallFrames><<<grid, kThreads, 0, s>>>(a, t);
+        else prep_kernel<kSmallFrames><<<grid, kThreads, 0, s>>>(a, t);
     } else {
-        prep_kernel<kMaxFramesPerLaunch><<<grid, kThreads, 0, s>>>(a, tab);
+        if (f16) prep16_kernel<kMaxFramesPerLaunch><<<grid, kThreads, 0, s>>>(a, tab);
+        else prep_kernel<kMaxFramesPerLaunch><<<grid, kThreads, 0, s>>>(a, tab);
     }
     return cudaGetLastError();
 }

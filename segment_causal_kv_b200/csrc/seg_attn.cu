@@ -6,24 +6,25 @@
 // visible cached tokens of earlier segments followed by every token of the
 // current segment (no mask inside a segment; causality across segments is
 // structural: later segments are never in the cache). An INT8 cache is
-// attended to in BF16 (model card, "Single-GPU Low-Memory Inference": INT8 KV
-// storage, BF16 attention computation): K as its integer codes, which BF16
-// holds exactly, with the per-key K scale applied to the scores in the
-// softmax; V as code * scale rounded to BF16.
+// attended to in 16-bit floating point (model card, "Single-GPU Low-Memory
+// Inference": INT8 KV storage, 16-bit attention computation), here FP16 with
+// power-of-two exponents per Q row and per 128-key tile (nomas_f16.cuh): the
+// scores of a tile are s = Q^.K^ * 2^(a_i + b_T), its V values V^ * 2^c_T.
 //
 // Three forms (template parameter kMode):
-//   kBf16   BF16 cache; every K/V tile arrives by TMA.
+//   kBf16   BF16 cache; every K/V tile arrives by TMA; BF16 Q, K, P.
 //   kWindow INT8 cache whose visible window dequant_window_kernel has written
-//           to a BF16 copy once per call (K codes, V code * scale); tiles by
-//           TMA, the K scales of each cache tile go into a coefficient ring.
-//   kFused  INT8 cache converted in shared memory tile by tile by a filler
-//           warpgroup (no copy: for workspaces too small to hold one).
+//           to an FP16 copy once per call; tiles by TMA.
+//   kFused  INT8 cache converted to FP16 in shared memory tile by tile by a
+//           filler warpgroup (no copy: for workspaces too small to hold one).
+// In both INT8 forms Q and K are FP16 for every tile; P.V is FP16 for cache
+// tiles and BF16 for the current segment's tiles (V is the caller's BF16).
 //
 // Structure of one CTA (one "unit" = two 128-row Q tiles of one head, and a
 // contiguous range of 128-key KV tiles: cache tiles first, then the current
 // segment's tiles):
 //   warp 0      TMA producer: Q tiles once, then (kBf16, kWindow) every K/V
-//               tile into a 2-stage ring; kWindow: the K coefficients
+//               tile into a 2-stage ring
 //   warp 1      TMEM allocator + tcgen05.mma issuer
 //   warps 4-7   softmax warpgroup for Q tile 0 (one thread per query row)
 //   warps 8-11  softmax warpgroup for Q tile 1
@@ -31,18 +32,22 @@
 //               converted from codes and scales; current-segment tiles are
 //               loaded by TMA. One filler in tile order keeps every parity
 //               wait on the ring exact.
-// TMEM (512 columns): S0 | S1 | O0 | O1, 128 fp32 columns each; the BF16
+// TMEM (512 columns): S0 | S1 | O0 | O1, 128 fp32 columns each; the 16-bit
 // probabilities P overwrite the first 64 columns of their S block and feed
 // the P.V product straight from TMEM (A operand in tensor memory).
 // MMA order per KV tile j: PV0(j-1) S0(j) | PV1(j-1) S1(j) -- while one
 // softmax warpgroup exponentiates, the tensor core works for the other. The
 // issuer waits for V(j-1) before PV0(j-1) and for K(j) only before S0(j).
 // Online softmax in base 2 with lazy rescaling: the running reference max is
-// raised only when a tile's max may exceed it by more than 8 (so P <= 256),
-// and only then is O rescaled in TMEM.
+// raised only when a tile's max may exceed it by more than 8 (so P <= 256,
+// inside FP16's range), and only then is O rescaled in TMEM. With INT8 caches
+// the reference follows x + c_T (x the log2-scaled score, c_T the V exponent
+// of its tile): P' = 2^(x + c_T - m) times V^ is 2^(x - m) times V, and the
+// row sum adds P' * 2^-c_T.
 // Split-KV: with splits > 1 each CTA leaves (O unnormalised, max, sum) in the
 // workspace and counts itself in per unit; the last CTA of a unit to arrive
 // merges the splits and writes the output (the partials are still in L2).
+#include "nomas_f16.cuh"
 #include "nomas_internal.h"
 #include "nomas_ptx.cuh"
 
@@ -55,8 +60,7 @@ namespace {
 constexpr int BM = 128;
 constexpr int BN = 128;
 constexpr int kStages = 2;
-constexpr int kCoefSlots = 4;                 // ring of per-tile K coefficients (INT8 caches)
-constexpr uint32_t kTileBytes = BM * kD * 2;  // one BF16 128x128 tile
+constexpr uint32_t kTileBytes = BM * kD * 2;  // one 16-bit 128x128 tile
 constexpr uint32_t kHalfBytes = kTileBytes / 2;
 constexpr float kRescaleThreshold = 8.0f;     // P <= 2^8 between rescales
 
@@ -64,9 +68,7 @@ constexpr float kRescaleThreshold = 8.0f;     // P <= 2^8 between rescales
 constexpr uint32_t kOffQ = 0;                                // 2 tiles
 constexpr uint32_t kOffK = kOffQ + 2 * kTileBytes;           // kStages tiles
 constexpr uint32_t kOffV = kOffK + kStages * kTileBytes;     // kStages tiles
-constexpr uint32_t kOffCoef = kOffV + kStages * kTileBytes;  // kCoefSlots x 128 fp32
-constexpr uint32_t kOffBound = kOffCoef + kCoefSlots * BN * 4; // kCoefSlots x 4 warps x (max, min)
-constexpr uint32_t kOffBar = kOffBound + kCoefSlots * 4 * 8; // barriers
+constexpr uint32_t kOffBar = kOffV + kStages * kTileBytes;   // barriers
 constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;        // + alignment slack
 
 // barrier slots (8 bytes each)
@@ -80,9 +82,7 @@ enum {
     B_PFULL = B_SFULL + 2,
     B_OFULL = B_PFULL + 2,
     B_DRAIN = B_OFULL + 2,
-    B_CFULL = B_DRAIN + 1,          // + coefficient slot: the filler wrote a tile's K coefficients
-    B_CEMPTY = B_CFULL + kCoefSlots, // + coefficient slot: every softmax warp is done with them
-    B_COUNT = B_CEMPTY + kCoefSlots
+    B_COUNT = B_DRAIN + 1
 };
 constexpr uint32_t kOffTmemSlot = B_COUNT * 8;
 constexpr uint32_t kOffAbort = kOffTmemSlot + 8;
@@ -92,6 +92,18 @@ static_assert(kOffLast + 4 <= 256, "barrier area overflow");
 static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 
 enum { kBf16 = 0, kWindow = 1, kFused = 2 };
+
+// kFused runs 512 threads, launched at 128 registers each (the whole register
+// file of one SM). Per-warpgroup budgets move registers from the producer/MMA
+// warpgroup and the filler to the two softmax warpgroups; they add up to the
+// launch's 4 x 128. The host checks the compiled register count before the
+// first launch (a smaller one would leave an inc waiting).
+constexpr uint32_t kFusedRegsLaunch = 128;
+constexpr uint32_t kFusedRegsCtl = 64;
+constexpr uint32_t kFusedRegsSoftmax = 168;
+constexpr uint32_t kFusedRegsFill = 112;
+static_assert(kFusedRegsCtl + 2 * kFusedRegsSoftmax + kFusedRegsFill == 4 * kFusedRegsLaunch,
+              "register budgets of the fused form");
 
 // mbar_wait run by every lane of a converged warp; lane 0's outcome is
 // broadcast so the warp leaves the wait converged.
@@ -126,7 +138,7 @@ __device__ __forceinline__ int tile_valid(const AttnArgs& a, int t) {
     return rem < BN ? rem : BN;
 }
 
-// K-major SW128 descriptor of k-step kk (16 dims) of a 128x128 BF16 tile.
+// K-major SW128 descriptor of k-step kk (16 dims) of a 128x128 16-bit tile.
 __device__ __forceinline__ uint64_t desc_kmajor(uint32_t tile, int kk) {
     return smem_desc(tile + (kk >> 2) * kHalfBytes + (kk & 3) * 32, 16, 1024, kSwizzle128B);
 }
@@ -142,33 +154,6 @@ __host__ __device__ constexpr uint64_t kstep_kmajor(int kk) {
     return static_cast<uint64_t>(((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4);
 }
 __host__ __device__ constexpr uint64_t kstep_mnmajor(int kk) { return static_cast<uint64_t>((kk * 2048) >> 4); }
-
-// 8 INT8 codes -> 8 BF16 values. A code c is read exactly as the float
-// 2^23 + (c + 128) (the byte of c ^ 0x80 placed under the exponent of 2^23),
-// minus 2^23 + 128. kScale: times the row scale in fp32, then rounded once to
-// BF16; otherwise the integer itself, which BF16 holds exactly (at most 7
-// significant bits), so its fp32 pattern's upper half is the BF16 pattern.
-template <bool kScale>
-__device__ __forceinline__ uint4 codes_to_bf16(uint2 w, float scale) {
-    const uint32_t w0 = w.x ^ 0x80808080u, w1 = w.y ^ 0x80808080u;
-    const float2 bias = make_float2(-8388736.0f, -8388736.0f);
-    uint32_t out[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        const uint32_t src = q < 2 ? w0 : w1;
-        const uint32_t b = (q & 1) * 2;
-        float2 f = make_float2(__uint_as_float(__byte_perm(src, 0x4B000000u, 0x7540u + b)),
-                               __uint_as_float(__byte_perm(src, 0x4B000000u, 0x7541u + b)));
-        f = __fadd2_rn(f, bias);
-        if (kScale) {
-            f = __fmul2_rn(f, make_float2(scale, scale));
-            out[q] = pack_bf16x2(f.x, f.y);
-        } else {
-            out[q] = __byte_perm(__float_as_uint(f.x), __float_as_uint(f.y), 0x7632u);
-        }
-    }
-    return make_uint4(out[0], out[1], out[2], out[3]);
-}
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
@@ -216,47 +201,6 @@ __device__ __forceinline__ float row_max(uint32_t t_s, int vc) {
     return mx;
 }
 
-// row_max in 32-column pieces (fewer registers live: the kWindow softmax holds
-// its tile's 128 coefficients in registers meanwhile).
-__device__ __forceinline__ float row_max32(uint32_t t_s) {
-    float mx = -INFINITY;
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-        uint32_t s[32];
-        tmem_ld32(t_s + c * 32, s);
-        float m[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) m[k] = mx;
-#pragma unroll
-        for (int e = 0; e < 32; e += 2)
-            m[(e >> 1) & 3] = max3(m[(e >> 1) & 3], __uint_as_float(s[e]), __uint_as_float(s[e + 1]));
-        mx = fmaxf(max3(m[0], m[1], m[2]), m[3]);
-        asm volatile("" : "+f"(mx));
-    }
-    return mx;
-}
-
-// Exact maximum of s_j * c_j over the valid columns of a row (used when the
-// cheap bound of a tile is too loose to serve as the reference: keys of very
-// different scales). Cold: run by a whole warp only when one of its rows needs it.
-__device__ __noinline__ float row_max_scaled(uint32_t t_s, const float4* coef, int vc) {
-    float mx = -INFINITY;
-#pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
-        uint32_t s[32];
-        tmem_ld32(t_s + c * 32, s);
-#pragma unroll
-        for (int e = 0; e < 32; e += 4) {
-            const float4 k = coef[(c * 32 + e) >> 2];
-            const float v[4] = {__uint_as_float(s[e]) * k.x, __uint_as_float(s[e + 1]) * k.y,
-                                __uint_as_float(s[e + 2]) * k.z, __uint_as_float(s[e + 3]) * k.w};
-#pragma unroll
-            for (int q = 0; q < 4; ++q) mx = (c * 32 + e + q < vc) ? fmaxf(mx, v[q]) : mx;
-        }
-    }
-    return mx;
-}
-
 // 2^x of two values on the FMA pipe, so that part of a row's exponentials
 // leave the MUFU unit (which alone would take as long as the tensor core needs
 // for the row's two products). Range reduction x = n + f with n = rint(x)
@@ -291,38 +235,34 @@ constexpr int kExp2PolyPairs = 3;
 constexpr int kExp2PolyPairsFused = 0;
 
 
-// One 32-column chunk of an unmasked S row -> 16 packed BF16 P columns;
-// x = s * c - m with c the scalar scale_log2, or with kCoef the tile's
-// per-column coefficients (scale_log2 times the key's K scale), read from
-// shared memory four at a time.
-template <int kPoly, bool kCoef>
-__device__ __forceinline__ void exp_chunk(const uint32_t (&s)[32], const float4* coef, float2 sl2x2, float2 negm,
-                                          float2 (&acc)[4], uint32_t (&p)[16]) {
-    float4 c4 = make_float4(sl2x2.x, sl2x2.x, sl2x2.x, sl2x2.x);
+// One 32-column chunk of an unmasked S row -> 16 packed 16-bit P columns
+// (kF16: FP16, else BF16), P = 2^(s * c + b) with the tile's scalars c (the
+// log2-scaled score coefficient) and b (the V exponent minus the reference).
+template <int kPoly, bool kF16>
+__device__ __forceinline__ void exp_chunk(const uint32_t (&s)[32], float2 cc, float2 bb, float2 (&acc)[4],
+                                          uint32_t (&p)[16]) {
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
-        if (kCoef && (e & 1) == 0) c4 = coef[e >> 1];
-        const float2 cc = kCoef ? ((e & 1) ? make_float2(c4.z, c4.w) : make_float2(c4.x, c4.y)) : sl2x2;
-        const float2 x = __ffma2_rn(make_float2(__uint_as_float(s[2 * e]), __uint_as_float(s[2 * e + 1])), cc, negm);
+        const float2 x = __ffma2_rn(make_float2(__uint_as_float(s[2 * e]), __uint_as_float(s[2 * e + 1])), cc, bb);
         float2 y;
         if ((e & 7) < kPoly)
             y = exp2_fma2(x);
         else
             y = make_float2(ex2_approx(x.x), ex2_approx(x.y));
         acc[e & 3] = __fadd2_rn(acc[e & 3], y);
-        p[e] = pack_bf16x2(y.x, y.y);
+        p[e] = kF16 ? pack_f16x2(y.x, y.y) : pack_bf16x2(y.x, y.y);
     }
 }
 
-// P = 2^(s * c - m) of one full 128-key S row, written as packed BF16 pairs
+// P = 2^(s * c + b) of one full 128-key S row, written as packed 16-bit pairs
 // over the first 64 columns of the row's S block; returns the fp32 row sum
 // (four independent packed accumulators). The TMEM loads are software
 // pipelined: chunk c + 1 is in flight while chunk c is exponentiated. P chunk c
 // lands on columns [16c, 16c + 16), all of which were read with chunks <= c.
-template <int kPoly, bool kCoef>
-__device__ __forceinline__ float row_exp_store_full(uint32_t t_s, const float4* coef, float sl2, float m) {
-    const float2 sl2x2 = make_float2(sl2, sl2);
-    const float2 negm = make_float2(-m, -m);
+template <int kPoly, bool kF16>
+__device__ __forceinline__ float row_exp_store_full(uint32_t t_s, float c, float b) {
+    const float2 cc = make_float2(c, c);
+    const float2 bb = make_float2(b, b);
     float2 acc[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) acc[k] = make_float2(0.0f, 0.0f);
@@ -330,108 +270,46 @@ __device__ __forceinline__ float row_exp_store_full(uint32_t t_s, const float4* 
     tmem_ld32_issue(t_s, sa);
     tmem_ld32_wait(sa);
     tmem_ld32_issue(t_s + 32, sb);
-    exp_chunk<kPoly, kCoef>(sa, coef, sl2x2, negm, acc, p);
+    exp_chunk<kPoly, kF16>(sa, cc, bb, acc, p);
     tmem_st16(t_s, p);
     tmem_ld32_wait(sb);
     tmem_ld32_issue(t_s + 64, sa);
-    exp_chunk<kPoly, kCoef>(sb, coef + 8, sl2x2, negm, acc, p);
+    exp_chunk<kPoly, kF16>(sb, cc, bb, acc, p);
     tmem_st16(t_s + 16, p);
     tmem_ld32_wait(sa);
     tmem_ld32_issue(t_s + 96, sb);
-    exp_chunk<kPoly, kCoef>(sa, coef + 16, sl2x2, negm, acc, p);
+    exp_chunk<kPoly, kF16>(sa, cc, bb, acc, p);
     tmem_st16(t_s + 32, p);
     tmem_ld32_wait(sb);
-    exp_chunk<kPoly, kCoef>(sb, coef + 24, sl2x2, negm, acc, p);
+    exp_chunk<kPoly, kF16>(sb, cc, bb, acc, p);
     tmem_st16(t_s + 48, p);
     const float2 t = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
     return t.x + t.y;
 }
 
-// Full-tile exp pass with per-column coefficients read from shared memory, in
-// 16-column chunks (chunk q + 1 of S loads from TMEM while chunk q is
-// exponentiated): fewer registers live than the 32-column form, which with
-// its coefficients would not fit the softmax warps' registers.
-template <int kPoly>
-__device__ __forceinline__ void exp_chunk16(const uint32_t (&s)[16], const float4 (&c)[4], float2 negm,
-                                            float2 (&acc)[4], uint32_t (&p)[8]) {
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-        const float4 c4 = c[e >> 1];
-        const float2 cc = (e & 1) ? make_float2(c4.z, c4.w) : make_float2(c4.x, c4.y);
-        const float2 x = __ffma2_rn(make_float2(__uint_as_float(s[2 * e]), __uint_as_float(s[2 * e + 1])), cc, negm);
-        float2 y;
-        if ((e & 7) < kPoly)
-            y = exp2_fma2(x);
-        else
-            y = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-        acc[e & 3] = __fadd2_rn(acc[e & 3], y);
-        p[e] = pack_bf16x2(y.x, y.y);
-    }
-}
-// The coefficients of chunk q + 1 are read together with its TMEM load, one
-// chunk ahead of their use: the TMEM waits order every memory access around
-// them, so a read issued after a wait would expose its full latency.
-template <int kPoly>
-__device__ __forceinline__ float row_exp_store_coef16(uint32_t t_s, const float4* coef, float m) {
-    const float2 negm = make_float2(-m, -m);
-    float2 acc[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) acc[k] = make_float2(0.0f, 0.0f);
-    uint32_t sa[16], sb[16], p[8];
-    float4 ca[4], cb[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) ca[k] = coef[k];
-    tmem_ld16_issue(t_s, sa);
-#pragma unroll
-    for (int q = 0; q < 8; q += 2) {
-        tmem_ld16_wait(sa);
-        tmem_ld16_issue(t_s + 16 * (q + 1), sb);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) cb[k] = coef[4 * (q + 1) + k];
-        exp_chunk16<kPoly>(sa, ca, negm, acc, p);
-        tmem_st8(t_s + 8 * q, p);
-        tmem_ld16_wait(sb);
-        if (q + 2 < 8) {
-            tmem_ld16_issue(t_s + 16 * (q + 2), sa);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) ca[k] = coef[4 * (q + 2) + k];
-        }
-        exp_chunk16<kPoly>(sb, cb, negm, acc, p);
-        tmem_st8(t_s + 8 * (q + 1), p);
-    }
-    const float2 t = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
-    return t.x + t.y;
-}
-
 // Masked form for a ragged last tile (columns >= vc get P = 0): MUFU only,
-// one 32-column chunk at a time; coef may be null (scalar scale_log2).
-__device__ __forceinline__ float row_exp_store_masked_impl(uint32_t t_s, const float4* coef, float sl2, float m,
-                                                           int vc) {
-    const float2 negm = make_float2(-m, -m);
+// one 32-column chunk at a time.
+__device__ __forceinline__ float row_exp_store_masked_impl(uint32_t t_s, float c, float b, int vc, bool f16) {
+    const float2 cc = make_float2(c, c), bb = make_float2(b, b);
     float2 acc[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) acc[k] = make_float2(0.0f, 0.0f);
 #pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
+    for (int ch = 0; ch < 4; ++ch) {
         uint32_t s[32];
-        tmem_ld32(t_s + c * 32, s);
+        tmem_ld32(t_s + ch * 32, s);
         uint32_t p[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-            float2 cc = make_float2(sl2, sl2);
-            if (coef) {
-                const float4 c4 = coef[c * 8 + (e >> 1)];
-                cc = (e & 1) ? make_float2(c4.z, c4.w) : make_float2(c4.x, c4.y);
-            }
-            float2 x = __ffma2_rn(make_float2(__uint_as_float(s[2 * e]), __uint_as_float(s[2 * e + 1])), cc, negm);
-            const int col = c * 32 + 2 * e;
+            float2 x = __ffma2_rn(make_float2(__uint_as_float(s[2 * e]), __uint_as_float(s[2 * e + 1])), cc, bb);
+            const int col = ch * 32 + 2 * e;
             x.x = col < vc ? x.x : -INFINITY;
             x.y = col + 1 < vc ? x.y : -INFINITY;
             const float p0 = ex2_approx(x.x), p1 = ex2_approx(x.y);
             acc[e & 3] = __fadd2_rn(acc[e & 3], make_float2(p0, p1));
-            p[e] = pack_bf16x2(p0, p1);
+            p[e] = f16 ? pack_f16x2(p0, p1) : pack_bf16x2(p0, p1);
         }
-        tmem_st16(t_s + c * 16, p);
+        tmem_st16(t_s + ch * 16, p);
     }
     const float2 t = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
     return t.x + t.y;
@@ -440,8 +318,8 @@ __device__ __forceinline__ float row_exp_store_masked_impl(uint32_t t_s, const f
 // Cold paths kept out of line, so they do not add to the register pressure of
 // the per-tile loop: tail tiles (masked), O rescaling, the epilogues.
 __device__ __noinline__ float row_max_masked(uint32_t t_s, int vc) { return row_max<true>(t_s, vc); }
-__device__ __noinline__ float row_exp_store_masked(uint32_t t_s, const float4* coef, float sl2, float m, int vc) {
-    return row_exp_store_masked_impl(t_s, coef, sl2, m, vc);
+__device__ __noinline__ float row_exp_store_masked(uint32_t t_s, float c, float b, int vc, bool f16) {
+    return row_exp_store_masked_impl(t_s, c, b, vc, f16);
 }
 
 // O *= alpha for one row (one thread), in TMEM.
@@ -582,7 +460,7 @@ __global__ void __launch_bounds__(kMode == kFused ? 512 : 384, 1)
     attn_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CUtensorMap tm_q,
                 const __grid_constant__ CUtensorMap tm_kcur, const __grid_constant__ CUtensorMap tm_vcur,
                 const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CUtensorMap tm_vc) {
-    constexpr bool kInt8 = kMode != kBf16;   // cache tiles carry per-key K coefficients
+    constexpr bool kInt8 = kMode != kBf16;   // FP16 Q/K, per-row and per-tile exponents
     constexpr bool kFill = kMode == kFused;  // cache tiles converted by the filler warpgroup
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -611,8 +489,8 @@ __global__ void __launch_bounds__(kMode == kFused ? 512 : 384, 1)
     int t_end = t_begin + a.tiles_per_split;
     if (t_end > t_total) t_end = t_total;
     const int n = t_end - t_begin; // >= 1 by construction of the split count
-    // cache tiles of this CTA come first: i < nci (INT8 caches: K coefficients per tile)
-    const int nci = kInt8 ? max(0, min(t_end, a.tiles_c) - t_begin) : 0;
+    // cache tiles of this CTA come first: i < nci
+    const int nci = max(0, min(t_end, a.tiles_c) - t_begin);
 
     // ---- setup
     if (threadIdx.x == 0) {
@@ -629,10 +507,6 @@ __global__ void __launch_bounds__(kMode == kFused ? 512 : 384, 1)
             mbar_init(bar(B_OFULL + w), 1);
         }
         mbar_init(bar(B_DRAIN), 1);
-        for (int c = 0; c < kCoefSlots; ++c) {
-            mbar_init(bar(B_CFULL + c), 1);
-            mbar_init(bar(B_CEMPTY + c), 4 * nq_tiles); // one arrival per active softmax warp
-        }
         *abort_flag = 0;
         fence_barrier_init();
         fence_proxy_async_smem();
@@ -649,23 +523,8 @@ __global__ void __launch_bounds__(kMode == kFused ? 512 : 384, 1)
     // are set up while it finishes; nothing it wrote is read before this point
     grid_dep_wait();
 
-    // the K coefficients of cache tile t into coefficient slot `slot`: scale_log2
-    // times the key's K scale (keys past the end get scale_log2, so that a masked
-    // score -inf stays -inf), and per writer warp the range over valid keys
-    auto put_coef = [&](int t, float ks, bool key_ok, int key_local, uint32_t slot, int bound_idx) {
-        const float c = key_ok ? a.scale_log2 * ks : a.scale_log2;
-        float cmax = key_ok ? c : -INFINITY, cmin = key_ok ? c : INFINITY;
-#pragma unroll
-        for (int off = 16; off >= 1; off >>= 1) {
-            cmax = fmaxf(cmax, __shfl_xor_sync(0xFFFFFFFFu, cmax, off));
-            cmin = fminf(cmin, __shfl_xor_sync(0xFFFFFFFFu, cmin, off));
-        }
-        reinterpret_cast<float*>(smem + kOffCoef + slot * (BN * 4))[key_local] = c;
-        if (lane == 0) reinterpret_cast<float2*>(smem + kOffBound + slot * 32)[bound_idx] = make_float2(cmax, cmin);
-        (void)t;
-    };
-
     if (warp < 4) {
+      if constexpr (kFill) regs_dec<kFusedRegsCtl>();
       if (warp == 0) {
         // ================================================================ producer
         if (lane == 0) {
@@ -702,30 +561,6 @@ __global__ void __launch_bounds__(kMode == kFused ? 512 : 384, 1)
                 drain_armed(k_armed, v_armed, bar(B_KFULL), bar(B_VFULL));
             }
         }
-      } else if (warp == 2) {
-        // ================================================================ K coefficients
-        // kWindow: the K scales of every cache tile (4 keys per lane) into the
-        // coefficient ring, off the TMA producer's path (their global loads
-        // would hold up the stage ring).
-        if (kMode == kWindow) {
-            for (int i = 0; i < nci; ++i) {
-                const uint32_t slot = static_cast<uint32_t>(i % kCoefSlots);
-                const int t = t_begin + i;
-                float ks[4];
-                bool ko[4];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int key = t * BN + q * 32 + lane;
-                    ko[q] = key < a.nc;
-                    ks[q] = ko[q] ? __ldg(a.ksc + static_cast<int64_t>(head) * a.cap_tok + key) : 0.0f;
-                }
-                if (i >= kCoefSlots && !mbar_wait_warp(bar(B_CEMPTY + slot), ((i / kCoefSlots) & 1) ^ 1, ctl)) break;
-#pragma unroll
-                for (int q = 0; q < 4; ++q) put_coef(t, ks[q], ko[q], q * 32 + lane, slot, q);
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar(B_CFULL + slot));
-            }
-        }
       } else if (warp == 1) {
         // ================================================================ MMA issuer
         // The whole warp runs the loop (warp-uniform waits and conditions) and
@@ -733,8 +568,9 @@ __global__ void __launch_bounds__(kMode == kFused ? 512 : 384, 1)
         // lane in a divergent branch run at little more than half the
         // tensor-core rate whenever a branch separates two groups of them.
         using I = Issuer<true>;
-        constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, BN, false, false);
-        constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, kD, false, true);
+        constexpr uint32_t idesc_qk = idesc_f32(BM, BN, false, false, kInt8);
+        constexpr uint32_t idesc_pv_c = idesc_f32(BM, kD, false, true, kInt8); // cache tiles
+        constexpr uint32_t idesc_pv_q = idesc_f32(BM, kD, false, true, false); // current tiles: BF16 V
         // TMEM columns: S of Q tile w at 128 w, O of Q tile w at 256 + 128 w
         auto tm_s = [&](int w) { return tmem + 128u * static_cast<uint32_t>(w); };
         auto tm_o = [&](int w) { return tmem + 256u + 128u * static_cast<uint32_t>(w); };
@@ -753,7 +589,7 @@ __global__ void __launch_bounds__(kMode == kFused ? 512 : 384, 1)
             for (int kk = 0; kk < kD / 16; ++kk)
                 I::ss(tm_s(w), qd + kstep_kmajor(kk), kd + kstep_kmajor(kk), idesc_qk, kk > 0 ? 1u : 0u);
         };
-        auto issue_pv = [&](int w, int st, bool first_tile) {
+        auto issue_pv = [&](int w, int st, bool first_tile, uint32_t idesc_pv) {
             const uint64_t vd = st ? v_desc1 : v_desc0;
 #pragma unroll
             for (int kk = 0; kk < BN / 16; ++kk)
@@ -775,11 +611,12 @@ __global__ void __launch_bounds__(kMode == kFused ? 512 : 384, 1)
             const int st1 = (i + 1) % kStages;
             const uint32_t ph1 = ((i + 1) / kStages) & 1;
             const bool last = (i + 1 == n);
+            const uint32_t idesc_pv = i < nci ? idesc_pv_c : idesc_pv_q;
             if (!(ok = I::wait(bar(B_VFULL + st), ph, ctl))) break;
             for (int w = 0; w < nq_tiles; ++w) {
                 if (!(ok = I::wait(bar(B_PFULL + w), i & 1, ctl))) break;
                 tc_fence_after();
-                issue_pv(w, st, i == 0);
+                issue_pv(w, st, i == 0, idesc_pv);
                 // each release is committed only when a later fill waits for it,
                 // so no arrival is left pending at exit
                 if (w == nq_tiles - 1 && i + kStages < n) I::commit(bar(B_VEMPTY + st));
@@ -806,6 +643,7 @@ __global__ void __launch_bounds__(kMode == kFused ? 512 : 384, 1)
         }
       }
     } else if (warp < 12) {
+        if constexpr (kFill) regs_inc<kFusedRegsSoftmax>();
         // ================================================================ softmax
         const int w = (warp - 4) >> 2;
         const int quad = warp & 3;
@@ -814,98 +652,55 @@ __global__ void __launch_bounds__(kMode == kFused ? 512 : 384, 1)
         const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
         const uint32_t t_s = tmem + lane_off + w * 128;
         const uint32_t t_o = tmem + lane_off + 256 + w * 128;
-        float m_ref = -INFINITY; // reference max, log2 units
+        const int qrow = (qt0 + w) * BM + r;
+        float m_ref = -INFINITY; // reference max, log2 units (INT8: of x + c_T)
         float l = 0.0f;
         bool ok = true;
-        // kWindow: the coefficient range of the next cache tile, read (after its
-        // CFULL wait) at the end of the previous tile
-        float chi_next = 0.0f, clo_next = 0.0f;
-        auto load_coefs = [&](int i) -> bool {
-            const uint32_t slot = static_cast<uint32_t>(i % kCoefSlots);
-            if (!mbar_wait(bar(B_CFULL + slot), (i / kCoefSlots) & 1, ctl)) return false;
-            const uint32_t bd = sbase + kOffBound + slot * 32;
-            const float4 b0 = lds128_ordered(bd), b1 = lds128_ordered(bd + 16);
-            chi_next = fmaxf(fmaxf(b0.x, b0.z), fmaxf(b1.x, b1.z));
-            clo_next = fminf(fminf(b0.y, b0.w), fminf(b1.y, b1.w));
-            return true;
-        };
         if (active) {
-            const float sl2 = a.scale_log2;
-            if (kMode == kWindow && nci > 0) ok = load_coefs(0);
+            // per-row score coefficient: log2(e)/sqrt(128), times 2^a_i for FP16 Q
+            float qc = a.scale_log2;
+            if (kInt8 && qrow < a.nq) qc *= __ldg(a.qs + static_cast<int64_t>(head) * a.nq + qrow);
+            const float4* te = kInt8 ? a.te + static_cast<int64_t>(head) * t_total : nullptr;
+            // INT8: the record of the next tile, read one tile ahead (its load
+            // completes while this warp waits for the tile's scores)
+            float4 rec_next = kInt8 ? __ldg(te + t_begin) : make_float4(1.0f, 1.0f, 0.0f, 1.0f);
             for (int i = 0; ok && i < n; ++i) {
                 const int t = t_begin + i;
-                const bool coef = kInt8 && i < nci; // warp-uniform
-                const uint32_t slot = static_cast<uint32_t>(i % kCoefSlots);
+                const float4 rec = rec_next;
+                if (kInt8 && i + 1 < n) rec_next = __ldg(te + t + 1);
+                const bool f16 = kInt8 && i < nci; // P in FP16 for cache tiles (warp-uniform)
                 if (!(ok = mbar_wait(bar(B_SFULL + w), i & 1, ctl))) break;
                 tc_fence_after();
                 const int vc = tile_valid(a, t);
                 const bool full = (vc == BN);
-                float chi = sl2, clo = sl2;
-                const float4* cf = nullptr;
-                if (coef) {
-                    cf = reinterpret_cast<const float4*>(smem + kOffCoef + slot * (BN * 4));
-                    if (kMode == kWindow) {
-                        // loaded (after their CFULL wait) at the end of the previous tile
-                        chi = chi_next;
-                        clo = clo_next;
-                    } else {
-                        if (!(ok = mbar_wait(bar(B_CFULL + slot), (i / kCoefSlots) & 1, ctl))) break;
-                        const uint32_t bd = sbase + kOffBound + slot * 32;
-                        const float4 b0 = lds128_ordered(bd), b1 = lds128_ordered(bd + 16);
-                        chi = fmaxf(fmaxf(b0.x, b0.z), fmaxf(b1.x, b1.z));
-                        clo = fminf(fminf(b0.y, b0.w), fminf(b1.y, b1.w));
-                    }
-                }
-                // pass 1: the tile's raw maximum; x_j = s_j * c_j with every c_j in
-                // [clo, chi], so the scaled maximum lies in [lo, hi] below
-                const float mx = !full ? row_max_masked(t_s, vc)
-                                 : (kMode == kWindow && coef) ? row_max32(t_s)
-                                                               : row_max<false>(t_s, vc);
-                const float hi = mx >= 0.0f ? mx * chi : mx * clo;
-                const float lo = mx >= 0.0f ? mx * clo : mx * chi;
-                // the reference moves only when the tile may exceed it by more than the
-                // threshold: to the upper bound when that is within the threshold of
-                // the true maximum (always so without coefficients), else to the
-                // exact scaled maximum
+                // x = s * c (c > 0), u = x + c_T: the tile's max of u is exact
+                const float c = qc * rec.x;
+                const float mx = full ? row_max<false>(t_s, vc) : row_max_masked(t_s, vc);
+                const float hi = mx * c + rec.z;
                 const bool up = hi > m_ref + kRescaleThreshold;
-                const bool exact = up && hi - lo > kRescaleThreshold;
-                float m_new = up ? hi : m_ref;
-                if (coef && __any_sync(0xFFFFFFFFu, exact)) {
-                    const float me = row_max_scaled(t_s, cf, vc);
-                    if (exact) m_new = me;
-                }
+                const float m_new = up ? hi : m_ref;
                 const float alpha = up ? ex2_approx(m_ref - m_new) : 1.0f; // 0 on the first tile
                 if (i > 0 && __any_sync(0xFFFFFFFFu, up)) rescale_o(t_o, alpha);
                 l *= alpha;
                 m_ref = m_new;
-                // pass 2: P into TMEM, row sum in fp32
-                if (coef) {
-                    if constexpr (kMode == kWindow)
-                        l += full ? row_exp_store_coef16<kExp2PolyPairs>(t_s, cf, m_ref)
-                                  : row_exp_store_masked(t_s, cf, sl2, m_ref, vc);
-                    else
-                        l += full ? row_exp_store_full<kExp2PolyPairsFused, true>(t_s, cf, sl2, m_ref)
-                                  : row_exp_store_masked(t_s, cf, sl2, m_ref, vc);
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(bar(B_CEMPTY + slot));
-                } else {
-                    l += full ? row_exp_store_full<kFill ? kExp2PolyPairsFused : kExp2PolyPairs, false>(t_s, nullptr,
-                                                                                                       sl2, m_ref)
-                              : row_exp_store_masked(t_s, nullptr, sl2, m_ref, vc);
-                }
+                // pass 2: P into TMEM, row sum in fp32 (scaled back by 2^-c_T)
+                const float b = rec.z - m_ref;
+                float ps;
+                if (f16)
+                    ps = full ? row_exp_store_full<kFill ? kExp2PolyPairsFused : kExp2PolyPairs, true>(t_s, c, b)
+                              : row_exp_store_masked(t_s, c, b, vc, true);
+                else
+                    ps = full ? row_exp_store_full<kFill ? kExp2PolyPairsFused : kExp2PolyPairs, false>(t_s, c, b)
+                              : row_exp_store_masked(t_s, c, b, vc, false);
+                l += kInt8 ? ps * rec.w : ps;
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar(B_PFULL + w));
-                // kWindow: the next cache tile's coefficients, loaded now so that their
-                // shared-memory loads (which queue behind the tensor core's operand
-                // reads) complete while this warp waits for the next S
-                if (kMode == kWindow && i + 1 < nci && !(ok = load_coefs(i + 1))) break;
             }
             // ---- epilogue
             if (ok) ok = mbar_wait(bar(B_OFULL + w), 0, ctl);
         }
-        const int qrow = (qt0 + w) * BM + r;
         const bool row_ok = active && ok && qrow < a.nq;
         if (a.splits == 1) {
             if (active && ok) {
@@ -942,23 +737,27 @@ __global__ void __launch_bounds__(kMode == kFused ? 512 : 384, 1)
             }
         }
     } else if (kFill && warp >= 12) {
+        if constexpr (kFill) regs_dec<kFusedRegsFill>();
         // ================================================================ INT8 filler
         // Warp wq converts rows [32 wq, 32 wq + 32) of a cache tile; in step j a
         // warp covers rows 2j and 2j+1, 16 lanes per row, 8 codes per lane, so a
-        // lane writes exactly one 16-byte BF16 chunk and each quarter-warp hits 8
+        // lane writes exactly one 16-byte FP16 chunk and each quarter-warp hits 8
         // distinct chunk slots of the swizzled row (no bank conflicts). Filler
-        // thread f (0..127) also loads the K and V scales of key f of the tile.
-        // The next cache tile's codes are loaded into registers as soon as the
-        // current tile has been converted, so global latency overlaps the MMAs.
+        // thread f (0..127) also loads the K and V scales of key f of the tile
+        // and forms its FP16 factors r = RN16(scale * 2^-e) with the tile's
+        // exponents. The next cache tile's codes are loaded into registers as
+        // soon as the current tile has been converted, so global latency
+        // overlaps the MMAs.
         const int f = threadIdx.x - 384;
         const int wq = warp - 12;
         const int half = lane >> 4;
         const int l16 = lane & 15;
         const bool elected = (f == 0);
         const uint32_t chunk_off = (l16 >> 3) * kHalfBytes;
+        const float4* te = a.te + static_cast<int64_t>(head) * t_total;
         uint2 kb[16], vb[16];
         float ks_own = 0.0f, vs_own = 0.0f; // scales of key f of the tile whose codes are in kb / vb
-        bool key_ok = false;
+        float4 rec = make_float4(1.0f, 1.0f, 0.0f, 1.0f);
         // row (32 wq + 2j + half) of a tile: (row & 7) = (2j & 7) ^ half, so the swizzled
         // chunk slot is slot0 ^ (2j & 7) and the byte offset is a constant per j
         const uint32_t slot0 = static_cast<uint32_t>((l16 & 7) ^ half);
@@ -975,24 +774,20 @@ __global__ void __launch_bounds__(kMode == kFused ? 512 : 384, 1)
         };
         auto load_scales = [&](int t) {
             const int key = t * BN + f;
-            key_ok = key < a.nc;
             const int64_t g = static_cast<int64_t>(head) * a.cap_tok + key;
+            const bool key_ok = key < a.nc;
             ks_own = key_ok ? __ldg(a.ksc + g) : 0.0f;
             vs_own = key_ok ? __ldg(a.vsc + g) : 0.0f;
+            rec = __ldg(te + t);
         };
-        auto convert_k = [&](uint32_t tile) {
+        // codes of the rows of step j times the factor of that row (held by lane 2j + half)
+        auto convert = [&](uint32_t tile, const uint2 (&buf)[16], float r_own) {
+            const uint32_t rbits = f16x2_splat(r_own);
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
+                const uint32_t r2 = __shfl_sync(0xFFFFFFFFu, rbits, 2 * j + half);
                 const uint32_t off = row_off0 + j * 256u + ((slot0 ^ static_cast<uint32_t>((2 * j) & 7)) << 4);
-                st_shared_v4(tile + off, codes_to_bf16<false>(kb[j], 0.0f));
-            }
-        };
-        auto convert_v = [&](uint32_t tile) {
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                const float sc = __shfl_sync(0xFFFFFFFFu, vs_own, 2 * j + half);
-                const uint32_t off = row_off0 + j * 256u + ((slot0 ^ static_cast<uint32_t>((2 * j) & 7)) << 4);
-                st_shared_v4(tile + off, codes_to_bf16<true>(vb[j], sc));
+                st_shared_v4(tile + off, codes_to_f16(buf[j], r2));
             }
         };
         // one elected thread waits; the group learns the outcome after a named
@@ -1024,18 +819,11 @@ __global__ void __launch_bounds__(kMode == kFused ? 512 : 384, 1)
                     k_armed[st] = (i / kStages) & 1;
                 }
             } else {
-                const uint32_t slot = static_cast<uint32_t>(i % kCoefSlots);
-                convert_k(ktile);
+                convert(ktile, kb, ks_own * rec.y);
                 if (next_cached) load_codes(a.kc8, t + 1, kb);
-                // the tile's K coefficients into the coefficient ring
-                if (i >= kCoefSlots && !group_wait(bar(B_CEMPTY + slot), ((i / kCoefSlots) & 1) ^ 1)) break;
-                put_coef(t, ks_own, key_ok, f, slot, wq);
                 fence_proxy_async_smem();
                 named_bar_sync(1, 128);
-                if (elected) {
-                    mbar_arrive(bar(B_KFULL + st));
-                    mbar_arrive(bar(B_CFULL + slot));
-                }
+                if (elected) mbar_arrive(bar(B_KFULL + st));
             }
             // ---- V (freed after the P.V MMAs of tile i - 2)
             if (i >= kStages && !group_wait(bar(B_VEMPTY + st), free_ph)) break;
@@ -1045,7 +833,7 @@ __global__ void __launch_bounds__(kMode == kFused ? 512 : 384, 1)
                     v_armed[st] = (i / kStages) & 1;
                 }
             } else {
-                convert_v(vtile);
+                convert(vtile, vb, vs_own * rec.w);
                 if (next_cached) {
                     load_codes(a.vc8, t + 1, vb);
                     load_scales(t + 1);
@@ -1067,36 +855,58 @@ __global__ void __launch_bounds__(kMode == kFused ? 512 : 384, 1)
     }
 }
 
-// One work item = 16 codes (16 bytes) of one row of K or V; 8 items per row,
-// consecutive threads on consecutive items, so loads (128 B per row) and
-// stores (256 B per row) are fully coalesced. Grid-stride over both tensors.
-// K rows are written as their codes (exact in BF16; the K scale reaches the
-// scores through the attention kernel's coefficients), V rows as code * scale.
-__global__ void __launch_bounds__(512) dequant_window_kernel(const __grid_constant__ DequantArgs a) {
+// One warp per (tensor, head, 128-key tile): the tile's exponent from the
+// maximum of its 128 scales (4 per lane, a shuffle reduction), then 32 steps of
+// 4 rows: lane l moves the 16 codes [16 (l & 7), 16 (l & 7) + 16) of row
+// 4 step + l / 8 (512 contiguous bytes of codes in, 1 KB of FP16 out per
+// step). Each row's factor RN16(scale * 2^-e) comes from the lane that loaded
+// its scale. Every key of the visible window is written; the tile record the
+// attention kernel reads is written by the RoPE prep kernel from the same
+// scales with the same exponent function.
+__global__ void __launch_bounds__(256, 1) dequant_window_kernel(const __grid_constant__ DequantArgs a) {
     // Launched dependent on the RoPE prep kernel and overlapping it: it reads
     // only the cache, which was complete before prep started. It lets the
     // attention kernel launch early, and before it exits it waits for prep, so
     // the attention kernel's wait on it covers prep too.
     grid_dep_launch();
-    const uint32_t rows = static_cast<uint32_t>(a.heads) * static_cast<uint32_t>(a.nc); // per tensor, < 2^31
-    const uint32_t items = 2u * rows * 8u;                                              // < 2^32 by the host check
-    for (uint32_t it = blockIdx.x * blockDim.x + threadIdx.x; it < items; it += gridDim.x * blockDim.x) {
-        const uint32_t trow = it >> 3;
-        const uint32_t part = it & 7u;
-        const bool is_v = trow >= rows;
-        const uint32_t r = is_v ? trow - rows : trow;
-        const uint32_t head = fast_div(r, a.div_nc);
-        const uint32_t tok = r - head * static_cast<uint32_t>(a.nc);
-        const int64_t src_row = static_cast<int64_t>(head) * a.cap_tok + tok;
-        const uint4 w = __ldg(reinterpret_cast<const uint4*>((is_v ? a.vc : a.kc) + src_row * kD) + part);
-        uint4* dst = reinterpret_cast<uint4*>((is_v ? a.vd : a.kd) + static_cast<int64_t>(r) * kD) + 2 * part;
-        if (is_v) {
-            const float sc = __ldg(a.vs + src_row);
-            dst[0] = codes_to_bf16<true>(make_uint2(w.x, w.y), sc);
-            dst[1] = codes_to_bf16<true>(make_uint2(w.z, w.w), sc);
-        } else {
-            dst[0] = codes_to_bf16<false>(make_uint2(w.x, w.y), 0.0f);
-            dst[1] = codes_to_bf16<false>(make_uint2(w.z, w.w), 0.0f);
+    const int lane = threadIdx.x & 31;
+    const int tasks = 2 * a.heads * a.tiles_c;
+    const int nwarps = gridDim.x * (blockDim.x >> 5);
+    for (int task = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); task < tasks; task += nwarps) {
+        const bool is_v = task >= a.heads * a.tiles_c;
+        const int tv = is_v ? task - a.heads * a.tiles_c : task;
+        const int head = tv / a.tiles_c;
+        const int T = tv - head * a.tiles_c;
+        const float* sc = (is_v ? a.vs : a.ks) + static_cast<int64_t>(head) * a.cap_tok + T * 128;
+        const int keys = min(128, a.nc - T * 128);
+        float own[4];
+        float mx = 0.0f;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            own[q] = (q * 32 + lane < keys) ? __ldg(sc + q * 32 + lane) : 0.0f;
+            mx = fmaxf(mx, own[q]);
+        }
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
+        const float inv = exp2_int(-pow2_exponent(mx, kTopCode));
+        const int8_t* src = (is_v ? a.vc : a.kc) + (static_cast<int64_t>(head) * a.cap_tok + T * 128) * kD;
+        uint16_t* dst = (is_v ? a.vd : a.kd) + (static_cast<int64_t>(head) * a.nc + T * 128) * kD;
+        const int part = lane & 7;
+        // rows 32 q .. 32 q + 31 have their scales in register own[q]
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+#pragma unroll 4
+            for (int k = 0; k < 8; ++k) {
+                const int row = 32 * q + 4 * k + (lane >> 3);
+                const float s_row = __shfl_sync(0xFFFFFFFFu, own[q], row & 31);
+                if (row < keys) {
+                    const uint4 w = __ldg(reinterpret_cast<const uint4*>(src + row * kD) + part);
+                    const uint32_t r2 = f16x2_splat(s_row * inv);
+                    uint4* d = reinterpret_cast<uint4*>(dst + row * kD) + 2 * part;
+                    d[0] = codes_to_f16(make_uint2(w.x, w.y), r2);
+                    d[1] = codes_to_f16(make_uint2(w.z, w.w), r2);
+                }
+            }
         }
     }
     grid_dep_wait();
@@ -1114,6 +924,13 @@ cudaError_t ensure_smem_attr() {
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < kMaxDev && done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+    if (kMode == kFused) {
+        // the register budgets assume the kernel launches at kFusedRegsLaunch
+        // registers per thread
+        cudaFuncAttributes fa{};
+        if ((e = cudaFuncGetAttributes(&fa, attn_kernel<kMode>)) != cudaSuccess) return e;
+        if (fa.numRegs != static_cast<int>(kFusedRegsLaunch)) return cudaErrorInvalidConfiguration;
+    }
     e = cudaFuncSetAttribute(attn_kernel<kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e == cudaSuccess && dev >= 0 && dev < kMaxDev) done[dev].store(true, std::memory_order_release);
     return e;
@@ -1132,12 +949,12 @@ cudaError_t launch_mode(const AttnArgs& a, const CUtensorMap& tm_q, const CUtens
 } // namespace
 
 cudaError_t launch_dequant_window(const DequantArgs& a, cudaStream_t s) {
-    const uint64_t items = 2ull * static_cast<uint64_t>(a.heads) * static_cast<uint64_t>(a.nc) * 8ull;
-    if (items == 0) return cudaSuccess;
-    uint64_t blocks = (items + 511) / 512;
-    const uint64_t cap = 148ull * 4ull; // persistent: 4 blocks of 512 threads per SM
+    const uint64_t tasks = 2ull * static_cast<uint64_t>(a.heads) * static_cast<uint64_t>(a.tiles_c);
+    if (tasks == 0) return cudaSuccess;
+    uint64_t blocks = (tasks + 7) / 8;
+    const uint64_t cap = 148ull * 8ull; // persistent: 8 blocks of 256 threads per SM
     if (blocks > cap) blocks = cap;
-    return launch_dependent(dequant_window_kernel, dim3(static_cast<unsigned>(blocks)), dim3(512), 0, s, a);
+    return launch_dependent(dequant_window_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, a);
 }
 
 cudaError_t launch_attn(const AttnArgs& a, AttnForm form, const CUtensorMap& tm_q, const CUtensorMap& tm_kcur,

@@ -168,11 +168,14 @@ def test_workspace_plans_between_the_minimum_and_the_full_size():
     d.valid_frames = 18  # as after 18 committed frames (state is not part of the stamp)
     full = nm.nomas_seg_attn_workspace_bytes(d, 3, 256)
     low = nm.nomas_seg_attn_workspace_min_bytes(d, 3, 256)
-    # the minimum is the one-split plan: the 256-byte status header and the rotated Q
-    # and K (16 heads x 2896 tokens x 256 B each, rounded up to 256 bytes)
-    qk = -(-16 * 2896 * 128 * 2 // 256) * 256
-    assert low == 256 + 2 * qk
-    # the full plan adds the BF16 copy of the INT8 window (2 x 16 heads x 15,840 tokens x
+    # the minimum is the one-split plan: the 256-byte status header, the rotated FP16 Q
+    # and K (16 heads x 2896 tokens x 256 B each), the tile records (16 heads x (124
+    # cache + 23 current tiles) x 16 B) and the Q row factors (16 x 2896 x 4 B), each
+    # rounded up to 256 bytes
+    up = lambda x: -(-x // 256) * 256
+    qk = up(16 * 2896 * 128 * 2)
+    assert low == 256 + 2 * qk + up(16 * (124 + 23) * 16) + up(16 * 2896 * 4)
+    # the full plan adds the FP16 copy of the INT8 window (2 x 16 heads x 15,840 tokens x
     # 256 B) and the KV-split partials: per split, 16 heads x 12 Q-tile pairs x 256 rows
     # of 128 fp32 values and an fp32 (max, sum) pair, and one counter per unit
     copy = 2 * 16 * 18 * 880 * 256
