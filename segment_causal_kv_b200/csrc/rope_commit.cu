@@ -133,9 +133,15 @@ __device__ __forceinline__ float rcp_approx(float x) {
 // finite, which makes every product finite) sends the lane to the exact
 // per-value path when any value needs it. Packed fp32 operations round each
 // half exactly as the scalar ones do.
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
 __device__ __forceinline__ uint2 quantize8(const float (&y)[8], float& scale_out) {
-    float amax = fmaxf(fmaxf(fmaxf(fabsf(y[0]), fabsf(y[1])), fmaxf(fabsf(y[2]), fabsf(y[3]))),
-                       fmaxf(fmaxf(fabsf(y[4]), fabsf(y[5])), fmaxf(fabsf(y[6]), fabsf(y[7]))));
+    float amax = max3f(max3f(fabsf(y[0]), fabsf(y[1]), fabsf(y[2])), max3f(fabsf(y[3]), fabsf(y[4]), fabsf(y[5])),
+                       fmaxf(fabsf(y[6]), fabsf(y[7])));
 #pragma unroll
     for (int off = 8; off >= 1; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off, 16));
     if (amax == 0.0f) {
@@ -155,7 +161,7 @@ __device__ __forceinline__ uint2 quantize8(const float (&y)[8], float& scale_out
         const float2 t = __fadd2_rn(q, make_float2(kMagic, kMagic));
         const float2 r = __fadd2_rn(t, make_float2(-kMagic, -kMagic));
         const float2 f = __ffma2_rn(r, make_float2(-1.0f, -1.0f), q); // q - rint(q), exact
-        fmax_abs = fmaxf(fmax_abs, fmaxf(fabsf(f.x), fabsf(f.y)));
+        fmax_abs = max3f(fmax_abs, fabsf(f.x), fabsf(f.y));
         w[2 * i] = __float_as_uint(t.x);
         w[2 * i + 1] = __float_as_uint(t.y);
     }
@@ -234,15 +240,23 @@ __global__ void __launch_bounds__(kThreads) commit_kernel(const __grid_constant_
         }
         const int64_t row0 = slot * a.tpf + rif; // row of head 0; head h adds h * cap_tok
         const uint32_t task_next = task + warps;
+        // pointers of this half-warp's first head; each step moves two heads on
+        const int hf = g0 + half;
+        const int64_t in_off = (tok0 + tok) * a.token_stride + static_cast<int64_t>(hf) * kD + l * 8;
+        const uint4* kp = reinterpret_cast<const uint4*>(P.k + in_off);
+        const uint4* vp = reinterpret_cast<const uint4*>(P.v + in_off);
+        const int64_t row_f = static_cast<int64_t>(hf) * a.cap_tok + row0;
+        const int64_t out_step = 2 * a.cap_tok; // rows between a half-warp's steps
         for (int j = 0; j < steps; ++j) {
-            const int h = g0 + 2 * j + half;
+            const int h = hf + 2 * j;
             const bool valid = h < g1;
             // next row of this half-warp: the following head, or the first of the next task
             uint4 kn = kx, vn = vx;
             if (j + 1 < steps) {
-                const int hn = min(h + 2, a.heads - 1);
-                kn = __ldcs(row_ptr(P.k, tok, hn));
-                vn = __ldcs(row_ptr(P.v, tok, hn));
+                if (h + 2 < a.heads) {
+                    kn = __ldcs(kp + (j + 1) * (2 * kD / 8));
+                    vn = __ldcs(vp + (j + 1) * (2 * kD / 8));
+                }
             } else if (task_next < tasks) {
                 uint32_t ln, tn;
                 const int hn = min(task_token(task_next, ln, tn) + half, a.heads - 1);
@@ -252,7 +266,7 @@ __global__ void __launch_bounds__(kThreads) commit_kernel(const __grid_constant_
             float ky[8], vy[8];
             rotate8(kx, cs, ky);
             unpack8(vx, vy);
-            const int64_t row = static_cast<int64_t>(valid ? h : 0) * a.cap_tok + row0;
+            const int64_t row = row_f + j * out_step;
             if (kInt8) {
                 float ks, vs;
                 const uint2 kc = quantize8(ky, ks);
@@ -328,16 +342,21 @@ __global__ void __launch_bounds__(kThreads) prep_kernel(const __grid_constant__ 
 
 // INT8 caches: RoPE of Q and K in fp32 to FP16 operands with power-of-two
 // exponents (nomas_f16.cuh), and every tile record of the attention call.
-// A block takes one (128-token tile, head) task at a time; half-warp g of the
-// block owns rows g, g + 32, g + 64, g + 96 of the tile. Each Q row gets its
-// own exponent (a half-warp reduction); the K rows stay in registers until the
-// block has the tile's maximum, then go out with the tile's exponent. Launch
-// chunks start at multiples of 128 frames, so a tile never spans two launches.
-// The launch with tok0 == 0 also writes the records of the cache tiles (a warp
-// per tile: the maxima of its 128 K and V scales).
+// A block of 256 threads takes one (128-token tile, head) task; half-warp g of
+// the block owns rows g, g + 16, ..., g + 112 of the tile. Each Q row gets its
+// own exponent (a half-warp reduction) and is written at once. K takes two
+// passes: the first finds the tile's maximum (a block reduction), the second
+// loads the rows again (from L1) and writes them with the tile's exponent; the
+// RoPE products are recomputed, bit for bit the same. Launch chunks start at
+// multiples of 128 frames, so a tile never spans two launches. The launch
+// with tok0 == 0 also writes the records of the cache tiles (a warp per tile:
+// the maxima of its 128 K and V scales).
+constexpr int kPrep16Threads = 256;
+constexpr int kPrep16Rows = 128 / (kPrep16Threads / 16); // rows per half-warp
+
 template <int kF>
-__global__ void __launch_bounds__(kThreads) prep16_kernel(const __grid_constant__ PrepArgs a,
-                                                          const __grid_constant__ RopeTabT<kF> tab) {
+__global__ void __launch_bounds__(kPrep16Threads, 3) prep16_kernel(const __grid_constant__ PrepArgs a,
+                                                                const __grid_constant__ RopeTabT<kF> tab) {
     grid_dep_launch();
     if (blockIdx.x == 0)
         for (int i = threadIdx.x; i < a.n_counters; i += blockDim.x) a.counters[i] = 0u;
@@ -346,8 +365,8 @@ __global__ void __launch_bounds__(kThreads) prep16_kernel(const __grid_constant_
     const int ttot = a.tiles_c + a.tiles_q;
 
     // ---- cache tile records
-    const int nwarps = gridDim.x * (kThreads / 32);
-    for (int task = blockIdx.x * (kThreads / 32) + warp; task < a.te_cache_tasks; task += nwarps) {
+    const int nwarps = gridDim.x * (kPrep16Threads / 32);
+    for (int task = blockIdx.x * (kPrep16Threads / 32) + warp; task < a.te_cache_tasks; task += nwarps) {
         const int h = task / a.tiles_c;
         const int T = task - h * a.tiles_c;
         float mk = 0.0f, mv = 0.0f;
@@ -371,68 +390,76 @@ __global__ void __launch_bounds__(kThreads) prep16_kernel(const __grid_constant_
     }
 
     // ---- current tiles
-    __shared__ float red[kThreads / 32];
+    __shared__ float red[kPrep16Threads / 32];
     const int l = lane & 15;
     const int g = threadIdx.x >> 4;
     const int T0 = a.tok0 / 128;
     const int T1 = (a.tok1 + 127) / 128;
     const int tasks = (T1 - T0) * a.heads;
+    // RoPE of one row's 8 elements owned by this lane (video rows), or the
+    // elements themselves (text rows)
+    auto rope8 = [&](int tok, uint4 x, float (&y)[8]) {
+        if (tok < a.nv) {
+            const uint32_t fa = fast_div(static_cast<uint32_t>(tok), a.div_tpf);
+            const int fi = static_cast<int>(fa) - a.frame0;
+            const uint32_t rif = static_cast<uint32_t>(tok) - fa * a.tpf;
+            const uint32_t hh = fast_div(rif, a.div_gw);
+            float2 cs[4];
+            lane_coeffs(l, fi, hh, rif - hh * a.grid_w, a.grid_h, tab, a.hw, cs);
+            rotate8(x, cs, y);
+        } else {
+            const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                y[2 * i] = bf16lo(w[i]);
+                y[2 * i + 1] = bf16hi(w[i]);
+            }
+        }
+    };
     for (int task = blockIdx.x; task < tasks; task += gridDim.x) {
         const int T = T0 + task / a.heads;
         const int h = task - (task / a.heads) * a.heads;
-        uint4 qx[4], kx[4];
-#pragma unroll
-        for (int rr = 0; rr < 4; ++rr) {
-            const int tok = T * 128 + g + 32 * rr;
-            qx[rr] = kx[rr] = make_uint4(0u, 0u, 0u, 0u);
-            if (tok < a.tok1) {
-                const int64_t in_off = static_cast<int64_t>(tok) * a.token_stride + h * kD + l * 8;
-                qx[rr] = __ldcs(reinterpret_cast<const uint4*>(a.q + in_off));
-                kx[rr] = __ldcs(reinterpret_cast<const uint4*>(a.k + in_off));
-            }
-        }
-        float ky[4][8];
+        const int tok0 = T * 128 + g;
         float kmax = 0.0f;
+        // pass 1 in two batches of rows (their loads in flight together)
 #pragma unroll
-        for (int rr = 0; rr < 4; ++rr) {
-            const int tok = T * 128 + g + 32 * rr;
-            float qy[8];
-            if (tok < a.nv && tok < a.tok1) {
-                const uint32_t fa = fast_div(static_cast<uint32_t>(tok), a.div_tpf);
-                const int fi = static_cast<int>(fa) - a.frame0;
-                const uint32_t rif = static_cast<uint32_t>(tok) - fa * a.tpf;
-                const uint32_t hh = fast_div(rif, a.div_gw);
-                float2 cs[4];
-                lane_coeffs(l, fi, hh, rif - hh * a.grid_w, a.grid_h, tab, a.hw, cs);
-                rotate8(qx[rr], cs, qy);
-                rotate8(kx[rr], cs, ky[rr]);
-            } else {
-                const uint32_t wq[4] = {qx[rr].x, qx[rr].y, qx[rr].z, qx[rr].w};
-                const uint32_t wk[4] = {kx[rr].x, kx[rr].y, kx[rr].z, kx[rr].w};
+        for (int b0 = 0; b0 < kPrep16Rows; b0 += kPrep16Rows / 2) {
+            uint4 qx[kPrep16Rows / 2], kx[kPrep16Rows / 2];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    qy[2 * i] = bf16lo(wq[i]);
-                    qy[2 * i + 1] = bf16hi(wq[i]);
-                    ky[rr][2 * i] = bf16lo(wk[i]);
-                    ky[rr][2 * i + 1] = bf16hi(wk[i]);
+            for (int rr = 0; rr < kPrep16Rows / 2; ++rr) {
+                const int tok = tok0 + 16 * (b0 + rr);
+                qx[rr] = kx[rr] = make_uint4(0u, 0u, 0u, 0u);
+                if (tok < a.tok1) {
+                    const int64_t in_off = static_cast<int64_t>(tok) * a.token_stride + h * kD + l * 8;
+                    qx[rr] = __ldcs(reinterpret_cast<const uint4*>(a.q + in_off));
+                    kx[rr] = __ldg(reinterpret_cast<const uint4*>(a.k + in_off));
                 }
             }
-            float qm = 0.0f;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                qm = fmaxf(qm, fabsf(qy[i]));
-                kmax = fmaxf(kmax, fabsf(ky[rr][i]));
-            }
+            for (int rr = 0; rr < kPrep16Rows / 2; ++rr) {
+                const int tok = tok0 + 16 * (b0 + rr);
+                if (tok < a.tok1) {
+                    float qy[8], ky[8];
+                    rope8(tok, qx[rr], qy);
+                    rope8(tok, kx[rr], ky);
+                    float qm = 0.0f;
 #pragma unroll
-            for (int off = 8; off >= 1; off >>= 1) qm = fmaxf(qm, __shfl_xor_sync(0xFFFFFFFFu, qm, off));
-            if (tok < a.tok1) {
-                const int ea = pow2_exponent(qm, kTopFloat);
-                const float f = exp2_int(-ea);
-                const int64_t out_off = (static_cast<int64_t>(h) * a.nq + tok) * kD + l * 8;
-                *reinterpret_cast<uint4*>(a.qt + out_off) =
-                    make_uint4(pack_f16x2(qy[0] * f, qy[1] * f), pack_f16x2(qy[2] * f, qy[3] * f),
-                               pack_f16x2(qy[4] * f, qy[5] * f), pack_f16x2(qy[6] * f, qy[7] * f));
-                if (l == 0) a.qs[static_cast<int64_t>(h) * a.nq + tok] = exp2_int(ea);
+                    for (int i = 0; i < 8; ++i) {
+                        qm = fmaxf(qm, fabsf(qy[i]));
+                        kmax = fmaxf(kmax, fabsf(ky[i]));
+                    }
+                    // rows of a half-warp are valid together: the shuffles stay in it
+#pragma unroll
+                    for (int off = 8; off >= 1; off >>= 1)
+                        qm = fmaxf(qm, __shfl_xor_sync(0xFFFFu << (lane & 16), qm, off));
+                    const int ea = pow2_exponent(qm, kTopFloat);
+                    const float f = exp2_int(-ea);
+                    const int64_t out_off = (static_cast<int64_t>(h) * a.nq + tok) * kD + l * 8;
+                    *reinterpret_cast<uint4*>(a.qt + out_off) =
+                        make_uint4(pack_f16x2(qy[0] * f, qy[1] * f), pack_f16x2(qy[2] * f, qy[3] * f),
+                                   pack_f16x2(qy[4] * f, qy[5] * f), pack_f16x2(qy[6] * f, qy[7] * f));
+                    if (l == 0) a.qs[static_cast<int64_t>(h) * a.nq + tok] = exp2_int(ea);
+                }
             }
         }
 #pragma unroll
@@ -441,17 +468,20 @@ __global__ void __launch_bounds__(kThreads) prep16_kernel(const __grid_constant_
         __syncthreads();
         float tmax = red[0];
 #pragma unroll
-        for (int i = 1; i < kThreads / 32; ++i) tmax = fmaxf(tmax, red[i]);
+        for (int i = 1; i < kPrep16Threads / 32; ++i) tmax = fmaxf(tmax, red[i]);
         const int eb = pow2_exponent(tmax, kTopFloat);
         const float f = exp2_int(-eb);
 #pragma unroll
-        for (int rr = 0; rr < 4; ++rr) {
-            const int tok = T * 128 + g + 32 * rr;
+        for (int rr = 0; rr < kPrep16Rows; ++rr) {
+            const int tok = tok0 + 16 * rr;
             if (tok < a.tok1) {
+                const int64_t in_off = static_cast<int64_t>(tok) * a.token_stride + h * kD + l * 8;
+                float ky[8];
+                rope8(tok, __ldcs(reinterpret_cast<const uint4*>(a.k + in_off)), ky);
                 const int64_t out_off = (static_cast<int64_t>(h) * a.nq + tok) * kD + l * 8;
-                *reinterpret_cast<uint4*>(a.kt + out_off) = make_uint4(
-                    pack_f16x2(ky[rr][0] * f, ky[rr][1] * f), pack_f16x2(ky[rr][2] * f, ky[rr][3] * f),
-                    pack_f16x2(ky[rr][4] * f, ky[rr][5] * f), pack_f16x2(ky[rr][6] * f, ky[rr][7] * f));
+                *reinterpret_cast<uint4*>(a.kt + out_off) =
+                    make_uint4(pack_f16x2(ky[0] * f, ky[1] * f), pack_f16x2(ky[2] * f, ky[3] * f),
+                               pack_f16x2(ky[4] * f, ky[5] * f), pack_f16x2(ky[6] * f, ky[7] * f));
             }
         }
         if (threadIdx.x == 0) a.te[static_cast<int64_t>(h) * ttot + a.tiles_c + T] = tile_record(eb, 0);
@@ -564,20 +594,25 @@ cudaError_t launch_commit(const CommitArgs& a_in, const CommitLayers& layers, co
 cudaError_t launch_prep(const PrepArgs& a, const RopeTab& tab, cudaStream_t s) {
     const int64_t rows = static_cast<int64_t>(a.tok1 - a.tok0) * a.heads;
     const bool f16 = a.te != nullptr;
-    // FP16 form: one block per (tile, head) task, or enough blocks to give the
-    // cache tile records a warp each
+    // FP16 form: one block per (tile, head) task, and enough blocks to give the
+    // cache tile records a warp each (at most 16 blocks per SM: all resident)
     const int64_t tasks = static_cast<int64_t>((a.tok1 + 127) / 128 - a.tok0 / 128) * a.heads;
-    int grid = f16 ? grid_for(tasks > 0 ? tasks : 1, 1) : grid_for(rows, kThreads / 16);
-    if (f16 && a.te_cache_tasks > 0) grid = max(grid, grid_for(a.te_cache_tasks, kThreads / 32));
+    int64_t want16 = tasks;
+    const int64_t te_blocks = (a.te_cache_tasks + kPrep16Threads / 32 - 1) / (kPrep16Threads / 32);
+    if (te_blocks > want16) want16 = te_blocks;
+    if (want16 > 148 * 16) want16 = 148 * 16;
+    if (want16 < 1) want16 = 1;
+    const int grid = f16 ? static_cast<int>(want16) : grid_for(rows, kThreads / 16);
+    const int block = f16 ? kPrep16Threads : kThreads;
     const int nv_frames = a.tok0 < a.nv ? (min(a.tok1, a.nv) - 1) / a.tpf - a.frame0 + 1 : 0;
     if (nv_frames <= kSmallFrames) {
         RopeTabT<kSmallFrames> t{};
         for (int f = 0; f < nv_frames; ++f)
             for (int j = 0; j < kTPairs; ++j) t.t[f][j] = tab.t[f][j];
-        if (f16) prep16_kernel<kSmallFrames><<<grid, kThreads, 0, s>>>(a, t);
+        if (f16) prep16_kernel<kSmallFrames><<<grid, block, 0, s>>>(a, t);
         else prep_kernel<kSmallFrames><<<grid, kThreads, 0, s>>>(a, t);
     } else {
-        if (f16) prep16_kernel<kMaxFramesPerLaunch><<<grid, kThreads, 0, s>>>(a, tab);
+        if (f16) prep16_kernel<kMaxFramesPerLaunch><<<grid, block, 0, s>>>(a, tab);
         else prep_kernel<kMaxFramesPerLaunch><<<grid, kThreads, 0, s>>>(a, tab);
     }
     return cudaGetLastError();
