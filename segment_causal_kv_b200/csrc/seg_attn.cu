@@ -23,8 +23,9 @@
 // Structure of one CTA (one "unit" = two 128-row Q tiles of one head, and a
 // contiguous range of 128-key KV tiles: cache tiles first, then the current
 // segment's tiles):
-//   warp 0      TMA producer: Q tiles once, then (kBf16, kWindow) every K/V
-//               tile into a 2-stage ring
+//   warp 0      TMA producer: Q tiles once, then (kBf16, kWindow) every K
+//               tile into a 3-stage ring
+//   warp 2      (kBf16, kWindow) TMA producer of every V tile, 2-stage ring
 //   warp 1      TMEM allocator + tcgen05.mma issuer
 //   warps 4-7   softmax warpgroup for Q tile 0 (one thread per query row)
 //   warps 8-11  softmax warpgroup for Q tile 1
@@ -37,7 +38,8 @@
 // the P.V product straight from TMEM (A operand in tensor memory).
 // MMA order per KV tile j: PV0(j-1) S0(j) | PV1(j-1) S1(j) -- while one
 // softmax warpgroup exponentiates, the tensor core works for the other. The
-// issuer waits for V(j-1) before PV0(j-1) and for K(j) only before S0(j).
+// issuer waits for the loads of later tiles only right after it has issued a
+// group of MMAs, so between groups it waits only for P.
 // Online softmax in base 2 with lazy rescaling: the running reference max is
 // raised only when a tile's max may exceed it by more than 8 (so P <= 256,
 // inside FP16's range), and only then is O rescaled in TMEM. With INT8 caches
@@ -59,26 +61,27 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BN = 128;
-constexpr int kStages = 2;
+constexpr int kKStages = 3;                   // K ring (a K stage is free again after the S MMAs)
+constexpr int kVStages = 2;                   // V ring (free after the P.V MMAs)
 constexpr uint32_t kTileBytes = BM * kD * 2;  // one 16-bit 128x128 tile
 constexpr uint32_t kHalfBytes = kTileBytes / 2;
 constexpr float kRescaleThreshold = 8.0f;     // P <= 2^8 between rescales
 
 // shared memory map (offsets from a 1024-byte aligned base)
 constexpr uint32_t kOffQ = 0;                                // 2 tiles
-constexpr uint32_t kOffK = kOffQ + 2 * kTileBytes;           // kStages tiles
-constexpr uint32_t kOffV = kOffK + kStages * kTileBytes;     // kStages tiles
-constexpr uint32_t kOffBar = kOffV + kStages * kTileBytes;   // barriers
+constexpr uint32_t kOffK = kOffQ + 2 * kTileBytes;           // kKStages tiles
+constexpr uint32_t kOffV = kOffK + kKStages * kTileBytes;    // kVStages tiles
+constexpr uint32_t kOffBar = kOffV + kVStages * kTileBytes;  // barriers
 constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;        // + alignment slack
 
 // barrier slots (8 bytes each)
 enum {
     B_QFULL = 0,
     B_KFULL = 1,                // + stage
-    B_VFULL = B_KFULL + kStages,
-    B_KEMPTY = B_VFULL + kStages,  // K and V stages are released separately: K as soon
-    B_VEMPTY = B_KEMPTY + kStages, // as the S MMAs that read it are done, V after P.V
-    B_SFULL = B_VEMPTY + kStages,  // + softmax warpgroup
+    B_VFULL = B_KFULL + kKStages,
+    B_KEMPTY = B_VFULL + kVStages,  // K and V stages are released separately: K as soon
+    B_VEMPTY = B_KEMPTY + kKStages, // as the S MMAs that read it are done, V after P.V
+    B_SFULL = B_VEMPTY + kVStages,  // + softmax warpgroup
     B_PFULL = B_SFULL + 2,
     B_OFULL = B_PFULL + 2,
     B_DRAIN = B_OFULL + 2,
@@ -231,7 +234,7 @@ __device__ __forceinline__ float2 exp2_fma2(float2 x) {
 // Of every 8 column pairs of a full tile, kPoly take exp2_fma2 and the rest
 // the MUFU ex2. In the kFused form the converting warps share the FMA pipe
 // and issue slots of every SM sub-partition, so there all go to the MUFU.
-constexpr int kExp2PolyPairs = 3;
+constexpr int kExp2PolyPairs = 2;
 constexpr int kExp2PolyPairsFused = 0;
 
 
@@ -444,12 +447,12 @@ __device__ __forceinline__ void load_v_tile(const AttnArgs& a, int t, int head, 
 
 // Bounded wait for the last armed phase of each K and V stage: no copy may
 // still be in flight when the CTA exits (matters only after an abort).
-__device__ __forceinline__ void drain_armed(const int (&k_armed)[kStages], const int (&v_armed)[kStages],
+__device__ __forceinline__ void drain_armed(const int (&k_armed)[kKStages], const int (&v_armed)[kVStages],
                                             uint32_t kfull0, uint32_t vfull0) {
-    for (int st = 0; st < kStages; ++st) {
+    for (int st = 0; st < kKStages; ++st) {
         const uint64_t t0 = global_timer_ns();
         while ((k_armed[st] >= 0 && !mbar_try_wait(kfull0 + 8u * st, k_armed[st])) ||
-               (v_armed[st] >= 0 && !mbar_try_wait(vfull0 + 8u * st, v_armed[st]))) {
+               (st < kVStages && v_armed[st] >= 0 && !mbar_try_wait(vfull0 + 8u * st, v_armed[st]))) {
             if (global_timer_ns() - t0 > NOMAS_WAIT_NS) break;
         }
     }
@@ -495,10 +498,12 @@ __global__ void __launch_bounds__(kMode == kFused ? 512 : 384, 1)
     // ---- setup
     if (threadIdx.x == 0) {
         mbar_init(bar(B_QFULL), 1);
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < kKStages; ++s) {
             mbar_init(bar(B_KFULL + s), 1);
-            mbar_init(bar(B_VFULL + s), 1);
             mbar_init(bar(B_KEMPTY + s), 1);
+        }
+        for (int s = 0; s < kVStages; ++s) {
+            mbar_init(bar(B_VFULL + s), 1);
             mbar_init(bar(B_VEMPTY + s), 1);
         }
         for (int w = 0; w < 2; ++w) {
@@ -543,23 +548,37 @@ __global__ void __launch_bounds__(kMode == kFused ? 512 : 384, 1)
             }
             // kFused: one filler for every stage, the converting warpgroup (codes for
             // cache tiles, TMA for current-segment tiles): with a single filler in
-            // tile order every parity wait on the stage ring is exact.
+            // tile order every parity wait on the stage ring is exact. Otherwise
+            // this thread fills the K ring and warp 2 the V ring, so that a K load
+            // never queues behind a V stage that is still in use.
             if (!kFill) {
-                int k_armed[kStages] = {-1, -1}, v_armed[kStages] = {-1, -1};
+                int k_armed[kKStages], v_armed[kVStages];
+                for (int st = 0; st < kKStages; ++st) k_armed[st] = -1;
+                for (int st = 0; st < kVStages; ++st) v_armed[st] = -1;
                 for (int i = 0; i < n; ++i) {
-                    const int st = i % kStages;
-                    const uint32_t free_ph = ((i / kStages) & 1) ^ 1;
-                    if (i >= kStages && !mbar_wait(bar(B_KEMPTY + st), free_ph, ctl)) break;
-                    load_k_tile(a, t_begin + i, head, sbase + kOffK + st * kTileBytes, bar(B_KFULL + st), &tm_kc,
+                    const int ks = i % kKStages;
+                    if (i >= kKStages && !mbar_wait(bar(B_KEMPTY + ks), ((i / kKStages) & 1) ^ 1, ctl)) break;
+                    load_k_tile(a, t_begin + i, head, sbase + kOffK + ks * kTileBytes, bar(B_KFULL + ks), &tm_kc,
                                 &tm_kcur);
-                    k_armed[st] = (i / kStages) & 1;
-                    if (i >= kStages && !mbar_wait(bar(B_VEMPTY + st), free_ph, ctl)) break;
-                    load_v_tile(a, t_begin + i, head, sbase + kOffV + st * kTileBytes, bar(B_VFULL + st), &tm_vc,
-                                &tm_vcur);
-                    v_armed[st] = (i / kStages) & 1;
+                    k_armed[ks] = (i / kKStages) & 1;
                 }
                 drain_armed(k_armed, v_armed, bar(B_KFULL), bar(B_VFULL));
             }
+        }
+      } else if (warp == 2) {
+        // ================================================================ V producer
+        if (!kFill && lane == 0) {
+            int k_armed[kKStages], v_armed[kVStages];
+            for (int st = 0; st < kKStages; ++st) k_armed[st] = -1;
+            for (int st = 0; st < kVStages; ++st) v_armed[st] = -1;
+            for (int i = 0; i < n; ++i) {
+                const int vs = i % kVStages;
+                if (i >= kVStages && !mbar_wait(bar(B_VEMPTY + vs), ((i / kVStages) & 1) ^ 1, ctl)) break;
+                load_v_tile(a, t_begin + i, head, sbase + kOffV + vs * kTileBytes, bar(B_VFULL + vs), &tm_vc,
+                            &tm_vcur);
+                v_armed[vs] = (i / kVStages) & 1;
+            }
+            drain_armed(k_armed, v_armed, bar(B_KFULL), bar(B_VFULL));
         }
       } else if (warp == 1) {
         // ================================================================ MMA issuer
@@ -578,13 +597,16 @@ __global__ void __launch_bounds__(kMode == kFused ? 512 : 384, 1)
         tc_fence_after();
         // k-step-0 descriptors of the Q tiles and of the K and V stages (scalars:
         // selected, not indexed, so they stay in registers)
-        static_assert(kStages == 2, "the stage descriptors below assume two stages");
+        // a K stage's descriptor is stage 0's plus the stage offset in the
+        // 16-byte address field (shared addresses < 256 KB: no carry)
+        static_assert(kVStages == 2, "the V stage descriptors below assume two stages");
         const uint64_t q_desc0 = desc_kmajor(sbase + kOffQ, 0), q_desc1 = desc_kmajor(sbase + kOffQ + kTileBytes, 0);
-        const uint64_t k_desc0 = desc_kmajor(sbase + kOffK, 0), k_desc1 = desc_kmajor(sbase + kOffK + kTileBytes, 0);
+        const uint64_t k_desc0 = desc_kmajor(sbase + kOffK, 0);
         const uint64_t v_desc0 = desc_mnmajor(sbase + kOffV, 0);
         const uint64_t v_desc1 = desc_mnmajor(sbase + kOffV + kTileBytes, 0);
         auto issue_s = [&](int w, int st) {
-            const uint64_t qd = w ? q_desc1 : q_desc0, kd = st ? k_desc1 : k_desc0;
+            const uint64_t qd = w ? q_desc1 : q_desc0;
+            const uint64_t kd = k_desc0 + static_cast<uint64_t>(st) * (kTileBytes >> 4);
 #pragma unroll
             for (int kk = 0; kk < kD / 16; ++kk)
                 I::ss(tm_s(w), qd + kstep_kmajor(kk), kd + kstep_kmajor(kk), idesc_qk, kk > 0 ? 1u : 0u);
@@ -602,38 +624,42 @@ __global__ void __launch_bounds__(kMode == kFused ? 512 : 384, 1)
                 issue_s(w, 0);
                 I::commit(bar(B_SFULL + w));
             }
-            // K of tile 0 is free once these S MMAs finish (a fill of tile 2 waits for it)
-            if (kStages < n) I::commit(bar(B_KEMPTY + 0));
+            // K of tile 0 is free once these S MMAs finish (a later fill waits for it)
+            if (kKStages < n) I::commit(bar(B_KEMPTY + 0));
         }
+        // Loads are awaited right after a group of MMAs has been issued (the tensor
+        // core has queued work meanwhile), never between two groups: V of the next
+        // tile and K of the tile after it at the end of each tile, so within a tile
+        // only the two P waits separate the groups.
+        if (ok) ok = I::wait(bar(B_VFULL + 0), 0, ctl);
+        if (ok && n > 1) ok = I::wait(bar(B_KFULL + 1 % kKStages), (1 / kKStages) & 1, ctl);
+        tc_fence_after();
         for (int i = 0; ok && i < n; ++i) {
-            const int st = i % kStages;
-            const uint32_t ph = (i / kStages) & 1;
-            const int st1 = (i + 1) % kStages;
-            const uint32_t ph1 = ((i + 1) / kStages) & 1;
+            const int st = i % kVStages;            // V stage of tile i
+            const int st1 = (i + 1) % kKStages;     // K stage of tile i + 1
             const bool last = (i + 1 == n);
             const uint32_t idesc_pv = i < nci ? idesc_pv_c : idesc_pv_q;
-            if (!(ok = I::wait(bar(B_VFULL + st), ph, ctl))) break;
             for (int w = 0; w < nq_tiles; ++w) {
                 if (!(ok = I::wait(bar(B_PFULL + w), i & 1, ctl))) break;
                 tc_fence_after();
                 issue_pv(w, st, i == 0, idesc_pv);
                 // each release is committed only when a later fill waits for it,
                 // so no arrival is left pending at exit
-                if (w == nq_tiles - 1 && i + kStages < n) I::commit(bar(B_VEMPTY + st));
+                if (w == nq_tiles - 1 && i + kVStages < n) I::commit(bar(B_VEMPTY + st));
                 if (!last) {
-                    // K of tile i + 1 is needed from here on only: P.V of Q tile 0
-                    // never waits for it
-                    if (w == 0) {
-                        if (!(ok = I::wait(bar(B_KFULL + st1), ph1, ctl))) break;
-                        tc_fence_after();
-                    }
                     issue_s(w, st1);
                     I::commit(bar(B_SFULL + w));
-                    if (w == nq_tiles - 1 && i + 1 + kStages < n) I::commit(bar(B_KEMPTY + st1));
+                    if (w == nq_tiles - 1 && i + 1 + kKStages < n) I::commit(bar(B_KEMPTY + st1));
                 } else {
                     I::commit(bar(B_OFULL + w));
                 }
             }
+            if (!ok) break;
+            if (i + 1 < n && !(ok = I::wait(bar(B_VFULL + (i + 1) % kVStages), ((i + 1) / kVStages) & 1, ctl)))
+                break;
+            if (i + 2 < n && !(ok = I::wait(bar(B_KFULL + (i + 2) % kKStages), ((i + 2) / kKStages) & 1, ctl)))
+                break;
+            tc_fence_after();
         }
         // drain: every MMA issued above has completed before teardown
         I::commit(bar(B_DRAIN));
@@ -797,7 +823,9 @@ __global__ void __launch_bounds__(kMode == kFused ? 512 : 384, 1)
             named_bar_sync(1, 128);
             return *dq_go != 0;
         };
-        int k_armed[kStages] = {-1, -1}, v_armed[kStages] = {-1, -1};
+        int k_armed[kKStages], v_armed[kVStages];
+        for (int st = 0; st < kKStages; ++st) k_armed[st] = -1;
+        for (int st = 0; st < kVStages; ++st) v_armed[st] = -1;
         if (nci > 0) {
             load_codes(a.kc8, t_begin, kb);
             load_codes(a.vc8, t_begin, vb);
@@ -805,32 +833,31 @@ __global__ void __launch_bounds__(kMode == kFused ? 512 : 384, 1)
         }
         for (int i = 0; i < n; ++i) {
             const int t = t_begin + i;
-            const int st = i % kStages;
-            const uint32_t free_ph = ((i / kStages) & 1) ^ 1;
-            const uint32_t ktile = sbase + kOffK + st * kTileBytes;
-            const uint32_t vtile = sbase + kOffV + st * kTileBytes;
+            const int ks = i % kKStages, vs = i % kVStages;
+            const uint32_t ktile = sbase + kOffK + ks * kTileBytes;
+            const uint32_t vtile = sbase + kOffV + vs * kTileBytes;
             const bool cached = i < nci;
             const bool next_cached = i + 1 < nci;
-            // ---- K (freed early: right after the S MMAs of tile i - 2)
-            if (i >= kStages && !group_wait(bar(B_KEMPTY + st), free_ph)) break;
+            // ---- K (freed early: right after the S MMAs of tile i - kKStages)
+            if (i >= kKStages && !group_wait(bar(B_KEMPTY + ks), ((i / kKStages) & 1) ^ 1)) break;
             if (!cached) {
                 if (elected) {
-                    load_k_tile(a, t, head, ktile, bar(B_KFULL + st), &tm_kc, &tm_kcur);
-                    k_armed[st] = (i / kStages) & 1;
+                    load_k_tile(a, t, head, ktile, bar(B_KFULL + ks), &tm_kc, &tm_kcur);
+                    k_armed[ks] = (i / kKStages) & 1;
                 }
             } else {
                 convert(ktile, kb, ks_own * rec.y);
                 if (next_cached) load_codes(a.kc8, t + 1, kb);
                 fence_proxy_async_smem();
                 named_bar_sync(1, 128);
-                if (elected) mbar_arrive(bar(B_KFULL + st));
+                if (elected) mbar_arrive(bar(B_KFULL + ks));
             }
-            // ---- V (freed after the P.V MMAs of tile i - 2)
-            if (i >= kStages && !group_wait(bar(B_VEMPTY + st), free_ph)) break;
+            // ---- V (freed after the P.V MMAs of tile i - kVStages)
+            if (i >= kVStages && !group_wait(bar(B_VEMPTY + vs), ((i / kVStages) & 1) ^ 1)) break;
             if (!cached) {
                 if (elected) {
-                    load_v_tile(a, t, head, vtile, bar(B_VFULL + st), &tm_vc, &tm_vcur);
-                    v_armed[st] = (i / kStages) & 1;
+                    load_v_tile(a, t, head, vtile, bar(B_VFULL + vs), &tm_vc, &tm_vcur);
+                    v_armed[vs] = (i / kVStages) & 1;
                 }
             } else {
                 convert(vtile, vb, vs_own * rec.w);
@@ -840,7 +867,7 @@ __global__ void __launch_bounds__(kMode == kFused ? 512 : 384, 1)
                 }
                 fence_proxy_async_smem();
                 named_bar_sync(1, 128);
-                if (elected) mbar_arrive(bar(B_VFULL + st));
+                if (elected) mbar_arrive(bar(B_VFULL + vs));
             }
         }
         if (elected) drain_armed(k_armed, v_armed, bar(B_KFULL), bar(B_VFULL));
