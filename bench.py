@@ -320,6 +320,7 @@ def run_extra(args, torch, nm, dev):
                           "roofline": {"bound": "hbm", "achieved": byts / (ms * 1e-3) / 1e9, "peak": hbm,
                                        "unit": "GB/s", "frac": byts / (ms * 1e-3) / 1e9 / hbm,
                                        "frac_of_nominal_8000": byts / (ms * 1e-3) / 1e9 / 8000.0,
+                                       "traffic": traffic_from_profile("commit_kernel<int8>"),
                                        "peak_kind": peak_src}}), flush=True)
         return 0
     if args.workload == "camera_xattn":
@@ -417,7 +418,7 @@ def run_extra(args, torch, nm, dev):
     if args.workload == "single_gpu_bf16_18f":
         # the headline shape (16 heads, 3 frames + 256 text over 18 history frames)
         # with the history kept in BF16: the same attention without the INT8 form's
-        # window copy and K-scale coefficients
+        # FP16 window copy and per-tile exponents
         cache = nm.KVCache("bf16", 16, 22, 40, 0, 18, device=dev)
         for s_ in range(6):
             k, v = synth.history_kv(geo, 3, 1, s_)
@@ -729,7 +730,7 @@ def main():
     # copy stream) overlaps step i+1; inputs and outputs are double-buffered and
     # ordered by events. The timed region spans all steps, from the first
     # upload to the last readback. L2 is not flushed here: each step streams
-    # ~330 MB (inputs, the INT8 window, its BF16 copy, split partials) through
+    # ~330 MB (inputs, the INT8 window, its FP16 copy, split partials) through
     # the 126 MB L2. The serial form (one step at a time, L2 flushed before
     # each) is reported too, as e2e_serial.
     Ke = args.e2e_steps or min(K, 100)
@@ -864,7 +865,6 @@ def main():
         # per step: the commit, the RoPE prep, the window copy and the attention
         # kernel (which merges its KV splits itself)
         "gpu_launches": K * 4,
-        "commit_traffic_profile": traffic_from_profile("commit_kernel<int8>"),
         "clocks": clocks,
     }
     if world == 1 and not args.no_cpu_baseline:

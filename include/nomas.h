@@ -15,7 +15,10 @@
  *    across segments"; cached keys and values are reused; full history
  *    (max_cache_segments=null) in the standard configuration.
  *  - same card, "Single-GPU Low-Memory Inference": INT8 KV storage with
- *    BF16 attention computation; a GPU history budget of 18 latent frames.
+ *    16-bit attention computation (the card names BF16; an INT8 cache is
+ *    attended to here in FP16 with power-of-two exponents per query row and
+ *    per 128-key tile, see nomas_seg_attn); a GPU history budget of 18
+ *    latent frames.
  *  - "Hy-Nomas Explained" blog, "Segment-wise causal joint attention" and
  *    "Step 3: The Video Latent ...": 22 x 40 = 880 tokens per latent frame.
  *
@@ -234,18 +237,20 @@ int nomas_kv_archive_evicted(const nomas_cache *c, int32_t n_frames, void *host_
                              int64_t *first_frame, void *stream);
 
 /*
- * nomas_seg_attn_workspace_bytes -- device workspace for the fastest form of
+ * nomas_seg_attn_workspace_bytes -- device workspace of the fastest plan of
  * nomas_seg_attn for this cache state and segment shape (0 on invalid
- * arguments). For an INT8 cache it includes a BF16 copy of the visible window
- * (2 * heads * visible_tokens * 256 bytes): the window is then dequantised
- * once per call and read by the BF16 attention kernel, instead of being
- * converted in shared memory by every CTA that reads a tile.
+ * arguments): the rotated Q and K, the KV-split partials, and for an INT8
+ * cache the tile exponent records, the Q row factors and an FP16 copy of the
+ * visible window (2 * heads * visible_tokens * 256 bytes), which is then
+ * converted once per call instead of in shared memory by every CTA that
+ * reads a tile.
  * nomas_seg_attn_workspace_min_bytes -- the smallest workspace nomas_seg_attn
- * accepts: without the copy, so an INT8 window is converted tile by tile
- * inside the attention kernel (same results up to rounding order, slower).
- * Both are equal for a BF16 cache. The first 256 bytes of a workspace are a
- * status header: zero them once before first use; the library only sets
- * error bits in it.
+ * accepts: one KV split and no copy (an INT8 window is converted tile by
+ * tile inside the attention kernel, to the same FP16 values).
+ * Any size in between is accepted; nomas_seg_attn then runs the fastest plan
+ * that fits (the copy first, then fewer KV splits). The first 256 bytes of a
+ * workspace are a status header: zero them once before first use; the
+ * library only sets error bits in it.
  */
 size_t nomas_seg_attn_workspace_bytes(const nomas_cache *c, int32_t n_video_frames, int32_t n_text);
 size_t nomas_seg_attn_workspace_min_bytes(const nomas_cache *c, int32_t n_video_frames, int32_t n_text);
@@ -267,11 +272,17 @@ size_t nomas_seg_attn_workspace_min_bytes(const nomas_cache *c, int32_t n_video_
  * For each head and query i: out_i = sum_j softmax_j(<R(p_i) q_i, k_j> / sqrt(128)) v_j
  * over the visible cached tokens (INT8 mode: code * scale) and all Nq
  * tokens of the current segment (keys rotated with their own positions).
- * The cache is read only. Q and current K are rounded to BF16 after RoPE,
- * probabilities are BF16 for the P.V product, accumulation is fp32.
- * workspace : device, >= nomas_seg_attn_workspace_min_bytes(...) bytes
- *             (>= nomas_seg_attn_workspace_bytes(...) selects the
- *             dequantise-once form for an INT8 cache), 256-byte aligned, not
+ * The cache is read only; accumulation is fp32. BF16 cache: Q and current K
+ * are rounded to BF16 after RoPE and the probabilities are BF16 for the P.V
+ * product. INT8 cache: every tensor-core operand is FP16 times a power of
+ * two held in fp32 -- Q per row, the current K per 128-key tile, the cache
+ * K and V as code * RN16(scale * 2^-e) with one exponent e per 128-key tile
+ * -- and the probabilities are FP16 for cache tiles and BF16 for the current
+ * segment's tiles (whose V is the caller's BF16). Per-token scales more than
+ * 2^100 apart within a head are outside this path's range.
+ * workspace : device, >= nomas_seg_attn_workspace_min_bytes(...) bytes (a
+ *             larger one selects a faster plan, up to
+ *             nomas_seg_attn_workspace_bytes(...)), 256-byte aligned, not
  *             shared with a call running concurrently.
  * Errors: NOMAS_ERR_ARG, NOMAS_ERR_ALIGN, NOMAS_ERR_STATE,
  * NOMAS_ERR_WORKSPACE, NOMAS_ERR_DEVICE, NOMAS_ERR_CUDA.
@@ -301,11 +312,10 @@ int nomas_device_status(void *workspace, void *stream);
  *
  * Arguments, layouts, results and errors are those of nomas_seg_attn, minus
  * the workspace. The fixed array serves as a workspace of
- * NOMAS_STATIC_SCRATCH_BYTES: the dequantise-once form runs when
- * nomas_seg_attn_workspace_bytes fits in it, the fused form when only
- * nomas_seg_attn_workspace_min_bytes does, and a shape whose minimum exceeds
- * it is rejected with NOMAS_ERR_WORKSPACE before anything is enqueued. The
- * call allocates and frees nothing.
+ * NOMAS_STATIC_SCRATCH_BYTES: the call runs the fastest plan that fits in it
+ * (as nomas_seg_attn does for any workspace size), and a shape whose minimum
+ * exceeds it is rejected with NOMAS_ERR_WORKSPACE before anything is
+ * enqueued. The call allocates and frees nothing.
  * The first call in a CUDA context (with that context current) sets the
  * array up: it looks up its device address and clears its status header
  * with an asynchronous memset on `stream`, ahead of the call's kernels; make

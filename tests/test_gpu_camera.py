@@ -8,7 +8,7 @@ import pytest
 
 import oracle
 import synth
-from harness import MAX_ABS, REL_L2, errors, to_dev, to_f64
+from harness import MAX_ABS, REL_L2, Guards, errors, to_dev, to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -25,11 +25,14 @@ def test_one_camera_token_gives_its_value_exactly(n_frames, chunk):
     torch = __import__("torch")
     import segment_causal_kv_b200 as nm
     q, kc, vc, F = inputs(16, 22, 40, n_frames, 1, chunk, seed=31)
-    out = nm.camera_attn(to_dev(q), to_dev(kc), to_dev(vc), n_frames, F, chunk)
+    g = Guards()  # canary bands around the output
+    out = g.alloc(q.shape, torch.bfloat16, fill=0.0)
+    nm.camera_attn(to_dev(q), to_dev(kc), to_dev(vc), n_frames, F, chunk, out=out)
     torch.cuda.synchronize()
     got = out.view(torch.int16).cpu().numpy().view(np.uint16)
     want = vc[(np.arange(n_frames * F) // F) // chunk, 0]
     assert np.array_equal(got, want)
+    g.check()
 
 
 @pytest.mark.parametrize("heads,gh,gw,n_frames,n_cam,chunk,q_std", [
@@ -42,13 +45,16 @@ def test_camera_attn_matches_the_oracle(heads, gh, gw, n_frames, n_cam, chunk, q
     torch = __import__("torch")
     import segment_causal_kv_b200 as nm
     q, kc, vc, F = inputs(heads, gh, gw, n_frames, n_cam, chunk, seed=heads + n_cam, q_std=q_std)
-    out = nm.camera_attn(to_dev(q), to_dev(kc), to_dev(vc), n_frames, F, chunk)
+    g = Guards()
+    out = g.alloc(q.shape, torch.bfloat16, fill=float("nan"))
+    nm.camera_attn(to_dev(q), to_dev(kc), to_dev(vc), n_frames, F, chunk, out=out)
     torch.cuda.synchronize()
     ref = oracle.camera_attn(q, n_frames, F, kc, vc, chunk)
     got = to_f64(out)
     assert np.isfinite(got).all()
     mx, rel = errors(got, ref)
     assert mx <= MAX_ABS and rel <= REL_L2, (mx, rel)
+    g.check()
 
 
 def test_padded_strides_touch_only_their_rows():

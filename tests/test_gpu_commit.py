@@ -7,7 +7,7 @@ import pytest
 
 import oracle
 import synth
-from harness import make_caches, to_dev
+from harness import Guards, make_caches, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -29,9 +29,11 @@ def assert_cache_equal(gpu, orc):
 
 def test_commit_int8_eighteen_frame_history_bit_exact():
     w = synth.WORKLOADS["single_gpu_int8_18f"]
-    gpu, orc = make_caches(w)
+    g = Guards()  # canary bands around the cache tensors
+    gpu, orc = make_caches(w, guards=g)
     assert_cache_equal(gpu, orc)
     assert gpu.valid_frames == 18 and gpu.head_slot == 0
+    g.check()
 
 
 @pytest.mark.parametrize("mode", ["int8", "bf16"])
@@ -39,7 +41,8 @@ def test_commit_ring_wraps_and_long_commits(mode):
     W = 4
     geo = synth.Geometry(3, 5, 7)
     import segment_causal_kv_b200 as nm
-    gpu = nm.KVCache(mode, 3, 5, 7, W, W)
+    g = Guards()
+    gpu = nm.KVCache(mode, 3, 5, 7, W, W, alloc=g.zeros)
     orc = oracle.OracleCache(oracle.MODE_INT8 if mode == "int8" else oracle.MODE_BF16, 3, 5, 7, W, W)
     for s, nf in enumerate([3, 2, 5, 1, 9, 4]):
         k, v = synth.history_kv(geo, nf, 90, s)
@@ -47,6 +50,7 @@ def test_commit_ring_wraps_and_long_commits(mode):
         orc.commit(k, v, nf)
         assert_cache_equal(gpu, orc)
         assert gpu.head_slot == gpu.frames_committed % W
+    g.check()
 
 
 def test_commit_bf16_full_history_and_capacity():
@@ -147,15 +151,17 @@ def test_layered_commit_matches_per_layer_commits(mode, n_layers):
     H, gh, gw, W = 2, 3, 5, 4
     geo = synth.Geometry(H, gh, gw)
     om = oracle.MODE_INT8 if mode == "int8" else oracle.MODE_BF16
-    gpus = [nm.KVCache(mode, H, gh, gw, W, W) for _ in range(n_layers)]
+    g = Guards()
+    gpus = [nm.KVCache(mode, H, gh, gw, W, W, alloc=g.zeros) for _ in range(n_layers)]
     orcs = [oracle.OracleCache(om, H, gh, gw, W, W) for _ in range(n_layers)]
     for s, nf in enumerate([3, 2, 4]):  # wraps the 4-frame ring
         kv = [synth.history_kv(geo, nf, 200 + layer, s) for layer in range(n_layers)]
         nm.commit_layers(gpus, [to_dev(k) for k, _ in kv], [to_dev(v) for _, v in kv], nf)
         for o, (k, v) in zip(orcs, kv):
             o.commit(k, v, nf)
-        for g, o in zip(gpus, orcs):
-            assert_cache_equal(g, o)
+        for gc, o in zip(gpus, orcs):
+            assert_cache_equal(gc, o)
+    g.check()
 
 
 
@@ -201,7 +207,8 @@ def test_commit_int8_round_half_even_ties():
     F = gh * gw
     geo = synth.Geometry(H, gh, gw)
     rng = np.random.default_rng(33)
-    gpu = nm.KVCache("int8", H, gh, gw, W, W)
+    g = Guards()
+    gpu = nm.KVCache("int8", H, gh, gw, W, W, alloc=g.zeros)
     orc = oracle.OracleCache(oracle.MODE_INT8, H, gh, gw, W, W)
     want = {}  # (tensor, head, slot row) -> (expected codes, expected scale)
     frame0 = 0
@@ -235,3 +242,4 @@ def test_commit_int8_round_half_even_ties():
     assert checked == H * W * (1 + F)
     # np.rint rounds half to even: the fixed ties landed on even codes
     assert np.all(codes["k"][0, F, 18:36] % 2 == 0)
+    g.check()
