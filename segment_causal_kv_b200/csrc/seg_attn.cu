@@ -24,8 +24,8 @@
 // contiguous range of 128-key KV tiles: cache tiles first, then the current
 // segment's tiles):
 //   warp 0      TMA producer: Q tiles once, then (kBf16, kWindow) every K
-//               tile into a 3-stage ring
-//   warp 2      (kBf16, kWindow) TMA producer of every V tile, 2-stage ring
+//               tile into a 2-stage ring
+//   warp 2      (kBf16, kWindow) TMA producer of every V tile, 3-stage ring
 //   warp 1      TMEM allocator + tcgen05.mma issuer
 //   warps 4-7   softmax warpgroup for Q tile 0 (one thread per query row)
 //   warps 8-11  softmax warpgroup for Q tile 1
@@ -61,8 +61,8 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BN = 128;
-constexpr int kKStages = 3;                   // K ring (a K stage is free again after the S MMAs)
-constexpr int kVStages = 2;                   // V ring (free after the P.V MMAs)
+constexpr int kKStages = 2;                   // K ring (a K stage is free again after the S MMAs)
+constexpr int kVStages = 3;                   // V ring (free only after the P.V MMAs: one more stage)
 constexpr uint32_t kTileBytes = BM * kD * 2;  // one 16-bit 128x128 tile
 constexpr uint32_t kHalfBytes = kTileBytes / 2;
 constexpr float kRescaleThreshold = 8.0f;     // P <= 2^8 between rescales
@@ -449,9 +449,9 @@ __device__ __forceinline__ void load_v_tile(const AttnArgs& a, int t, int head, 
 // still be in flight when the CTA exits (matters only after an abort).
 __device__ __forceinline__ void drain_armed(const int (&k_armed)[kKStages], const int (&v_armed)[kVStages],
                                             uint32_t kfull0, uint32_t vfull0) {
-    for (int st = 0; st < kKStages; ++st) {
+    for (int st = 0; st < (kKStages > kVStages ? kKStages : kVStages); ++st) {
         const uint64_t t0 = global_timer_ns();
-        while ((k_armed[st] >= 0 && !mbar_try_wait(kfull0 + 8u * st, k_armed[st])) ||
+        while ((st < kKStages && k_armed[st] >= 0 && !mbar_try_wait(kfull0 + 8u * st, k_armed[st])) ||
                (st < kVStages && v_armed[st] >= 0 && !mbar_try_wait(vfull0 + 8u * st, v_armed[st]))) {
             if (global_timer_ns() - t0 > NOMAS_WAIT_NS) break;
         }
@@ -597,13 +597,11 @@ __global__ void __launch_bounds__(kMode == kFused ? 512 : 384, 1)
         tc_fence_after();
         // k-step-0 descriptors of the Q tiles and of the K and V stages (scalars:
         // selected, not indexed, so they stay in registers)
-        // a K stage's descriptor is stage 0's plus the stage offset in the
+        // a K or V stage's descriptor is stage 0's plus the stage offset in the
         // 16-byte address field (shared addresses < 256 KB: no carry)
-        static_assert(kVStages == 2, "the V stage descriptors below assume two stages");
         const uint64_t q_desc0 = desc_kmajor(sbase + kOffQ, 0), q_desc1 = desc_kmajor(sbase + kOffQ + kTileBytes, 0);
         const uint64_t k_desc0 = desc_kmajor(sbase + kOffK, 0);
         const uint64_t v_desc0 = desc_mnmajor(sbase + kOffV, 0);
-        const uint64_t v_desc1 = desc_mnmajor(sbase + kOffV + kTileBytes, 0);
         auto issue_s = [&](int w, int st) {
             const uint64_t qd = w ? q_desc1 : q_desc0;
             const uint64_t kd = k_desc0 + static_cast<uint64_t>(st) * (kTileBytes >> 4);
@@ -612,7 +610,7 @@ __global__ void __launch_bounds__(kMode == kFused ? 512 : 384, 1)
                 I::ss(tm_s(w), qd + kstep_kmajor(kk), kd + kstep_kmajor(kk), idesc_qk, kk > 0 ? 1u : 0u);
         };
         auto issue_pv = [&](int w, int st, bool first_tile, uint32_t idesc_pv) {
-            const uint64_t vd = st ? v_desc1 : v_desc0;
+            const uint64_t vd = v_desc0 + static_cast<uint64_t>(st) * (kTileBytes >> 4);
 #pragma unroll
             for (int kk = 0; kk < BN / 16; ++kk)
                 I::ts(tm_o(w), tm_s(w) + kk * 8, vd + kstep_mnmajor(kk), idesc_pv, (first_tile && kk == 0) ? 0u : 1u);
