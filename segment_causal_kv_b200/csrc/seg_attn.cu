@@ -115,24 +115,18 @@ __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, co
     return __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
 }
 
-// How the MMA issuer issues: kWarp = the whole warp runs the loop and one
-// elected lane issues each instruction; otherwise lane 0 alone runs it.
-template <bool kWarp>
+// The MMA issuer: the whole warp runs the loop (warp-uniform waits and
+// conditions) and an elected lane issues each instruction inside the asm.
 struct Issuer {
     static __device__ __forceinline__ void ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
-        if (kWarp) mma_ss_warp(d, a, b, idesc, acc);
-        else mma_ss(d, a, b, idesc, acc);
+        mma_ss_warp(d, a, b, idesc, acc);
     }
     static __device__ __forceinline__ void ts(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
-        if (kWarp) mma_ts_warp(d, a, b, idesc, acc);
-        else mma_ts(d, a, b, idesc, acc);
+        mma_ts_warp(d, a, b, idesc, acc);
     }
-    static __device__ __forceinline__ void commit(uint32_t bar) {
-        if (kWarp) mma_commit_warp(bar);
-        else mma_commit(bar);
-    }
+    static __device__ __forceinline__ void commit(uint32_t bar) { mma_commit_warp(bar); }
     static __device__ __forceinline__ bool wait(uint32_t bar, uint32_t parity, const WaitCtl& ctl) {
-        return kWarp ? mbar_wait_warp(bar, parity, ctl) : mbar_wait(bar, parity, ctl);
+        return mbar_wait_warp(bar, parity, ctl);
     }
 };
 
@@ -586,7 +580,7 @@ __global__ void __launch_bounds__(kMode == kFused ? 512 : 384, 1)
         // one elected lane issues each MMA and commit; MMAs issued by a single
         // lane in a divergent branch run at little more than half the
         // tensor-core rate whenever a branch separates two groups of them.
-        using I = Issuer<true>;
+        using I = Issuer;
         constexpr uint32_t idesc_qk = idesc_f32(BM, BN, false, false, kInt8);
         constexpr uint32_t idesc_pv_c = idesc_f32(BM, kD, false, true, kInt8); // cache tiles
         constexpr uint32_t idesc_pv_q = idesc_f32(BM, kD, false, true, false); // current tiles: BF16 V
