@@ -177,8 +177,9 @@ bool window_copy_fits(int heads, int64_t nc) { return static_cast<int64_t>(heads
 // Workspace layout of a plan: status header, rotated Q and K (head-major; BF16,
 // or FP16 for an INT8 cache); for an INT8 cache the tile records
 // [heads][tiles_c + tiles_q] float4 and the Q row factors [heads][nq] fp32;
-// with splits > 1 the split partials [splits][units][32][256] float4, their
-// (max, sum) pairs [splits][units][256] and one arrival counter per unit; with
+// with splits > 1 the split partials [splits][units][16][256] (8 FP16 dims per
+// 16-byte word), their (max, sum, 2^e) records [splits][units][256] float4 and
+// one arrival counter per unit; with
 // the window form the FP16 copy of the visible window, K then V [heads][nc][128].
 Plan make_plan(const nomas_cache* c, int32_t n_video_frames, int32_t n_text, int max_splits, bool window) {
     Plan p{};
@@ -201,8 +202,8 @@ Plan make_plan(const nomas_cache* c, int32_t n_video_frames, int32_t n_text, int
     p.off_te = round_up(p.off_kt + qk_bytes, 256);
     p.off_qs = round_up(p.off_te + (int8 ? static_cast<size_t>(c->heads) * (p.tiles_c + p.tiles_q) * 16 : 0), 256);
     p.off_po = round_up(p.off_qs + (int8 ? static_cast<size_t>(c->heads) * p.nq * 4 : 0), 256);
-    p.off_pml = p.off_po + (sp ? prow * kD * sizeof(float) : 0);
-    p.off_cnt = round_up(p.off_pml + (sp ? prow * sizeof(float2) : 0), 256);
+    p.off_pml = p.off_po + (sp ? prow * kD * 2 : 0);
+    p.off_cnt = round_up(p.off_pml + (sp ? prow * 16 : 0), 256);
     p.off_kd = p.off_vd = p.total = round_up(p.off_cnt + (sp ? static_cast<size_t>(units) * sizeof(unsigned) : 0), 256);
     if (window) {
         const size_t copy = round_up(static_cast<size_t>(c->heads) * p.nc * kD * 2, 256);
@@ -598,8 +599,8 @@ int nomas_seg_attn(const nomas_cache* c, const void* q, const void* k, const voi
     a.vsc = c->v_scale;
     a.out = static_cast<uint16_t*>(out);
     a.lse = lse;
-    a.part_o = reinterpret_cast<float4*>(ws + p.off_po);
-    a.part_ml = reinterpret_cast<float2*>(ws + p.off_pml);
+    a.part_o = reinterpret_cast<uint4*>(ws + p.off_po);
+    a.part_ml = reinterpret_cast<float4*>(ws + p.off_pml);
     a.counters = counters;
     a.err = reinterpret_cast<unsigned*>(ws);
     a.scale_log2 = static_cast<float>(1.4426950408889634 / sqrt(static_cast<double>(kD)));

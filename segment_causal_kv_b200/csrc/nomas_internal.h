@@ -141,8 +141,8 @@ struct AttnArgs {
     const float* vsc;
     uint16_t* out;          // [nq][heads][128] BF16
     float* lse;             // [heads][nq] or null
-    float4* part_o;         // splits > 1: [splits][units][32][256] unnormalised O, 4 dims per float4
-    float2* part_ml;        // splits > 1: [splits][units][256] (reference max in log2 units, sum)
+    uint4* part_o;          // splits > 1: [splits][units][16][256] O / l * 2^-e in FP16, 8 dims per word
+    float4* part_ml;        // splits > 1: [splits][units][256] (reference max in log2 units, sum, 2^e, 0)
     unsigned* counters;     // splits > 1: [units] arrivals; the last CTA of a unit merges the splits
     unsigned* err;          // workspace status word
     float scale_log2;       // log2(e) / sqrt(128)

@@ -352,24 +352,51 @@ __device__ __noinline__ void store_out_row(uint32_t t_o, float inv_l, uint16_t* 
     }
 }
 
-// Partial row of one split: unnormalised fp32 O, 4 dims per float4, laid out
-// [32 chunks][256 rows] so that consecutive rows (threads) touch consecutive
-// 16-byte words.
-__device__ __noinline__ void store_partial_row(uint32_t t_o, float4* dst) {
+// Partial row of one split: O / l times 2^-e in FP16, with e from the row's
+// largest |O / l| (nomas_f16.cuh: that element lies in [2^14, 2^15), so no value
+// leaves FP16's range whatever the magnitude of V), 8 dims per 16-byte word,
+// laid out [16 chunks][256 rows] so that consecutive rows (threads) touch
+// consecutive words. Returns 2^e, which the merge multiplies back.
+__device__ __noinline__ float store_partial_row(uint32_t t_o, float inv_l, uint4* dst) {
+    float mx = 0.0f;
 #pragma unroll 1
     for (int c = 0; c < 4; ++c) {
         uint32_t o[32];
         tmem_ld32(t_o + c * 32, o);
 #pragma unroll
-        for (int e = 0; e < 8; ++e)
-            dst[(c * 8 + e) * 256] = make_float4(__uint_as_float(o[4 * e]), __uint_as_float(o[4 * e + 1]),
-                                                 __uint_as_float(o[4 * e + 2]), __uint_as_float(o[4 * e + 3]));
+        for (int e = 0; e < 32; e += 2) mx = max3(mx, fabsf(__uint_as_float(o[e])), fabsf(__uint_as_float(o[e + 1])));
     }
+    const int ex = pow2_exponent(mx * inv_l, kTopFloat);
+    const float f = inv_l * exp2_int(-ex);
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+        uint32_t o[32];
+        tmem_ld32(t_o + c * 32, o);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const uint32_t* q = o + 8 * e;
+            dst[(c * 4 + e) * 256] =
+                make_uint4(pack_f16x2(__uint_as_float(q[0]) * f, __uint_as_float(q[1]) * f),
+                           pack_f16x2(__uint_as_float(q[2]) * f, __uint_as_float(q[3]) * f),
+                           pack_f16x2(__uint_as_float(q[4]) * f, __uint_as_float(q[5]) * f),
+                           pack_f16x2(__uint_as_float(q[6]) * f, __uint_as_float(q[7]) * f));
+        }
+    }
+    return exp2_int(ex);
+}
+
+__device__ __forceinline__ float2 f16x2_to_f32x2(uint32_t w) {
+    float lo, hi;
+    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\tcvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, h;\n\t}"
+        : "=f"(lo), "=f"(hi)
+        : "r"(w));
+    return make_float2(lo, hi);
 }
 
 // Merge of the splits of one row (run by the last CTA of a unit to arrive):
-// O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s with M = max_s m_s. Eight
-// 16-byte loads per split are in flight at a time.
+// O = sum_s 2^(m_s - M) l_s O^_s 2^e_s / sum_s 2^(m_s - M) l_s with M = max_s m_s
+// and O^_s the stored FP16 row of split s. Four 16-byte loads per split are in
+// flight at a time.
 __device__ __noinline__ void merge_row(const AttnArgs& a, int unit, int row, uint16_t* dst, float* lse_dst) {
     const int units = a.heads * a.pairs;
     float mmax = -INFINITY;
@@ -377,37 +404,44 @@ __device__ __noinline__ void merge_row(const AttnArgs& a, int unit, int row, uin
         mmax = fmaxf(mmax, __ldcg(&a.part_ml[(static_cast<int64_t>(s) * units + unit) * 256 + row]).x);
     float L = 0.0f;
     for (int s = 0; s < a.splits; ++s) {
-        const float2 ml = __ldcg(&a.part_ml[(static_cast<int64_t>(s) * units + unit) * 256 + row]);
+        const float4 ml = __ldcg(&a.part_ml[(static_cast<int64_t>(s) * units + unit) * 256 + row]);
         L += ml.y * exp2f(ml.x - mmax);
     }
     const float inv = 1.0f / L;
 #pragma unroll 1
-    for (int c0 = 0; c0 < 32; c0 += 8) {
-        float4 acc[8];
+    for (int c0 = 0; c0 < 16; c0 += 4) {
+        float2 acc[4][4];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int k = 0; k < 4; ++k)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[k][e] = make_float2(0.0f, 0.0f);
 #pragma unroll 1
         for (int s = 0; s < a.splits; ++s) {
             const int64_t pu = static_cast<int64_t>(s) * units + unit;
-            const float g = exp2f(__ldcg(&a.part_ml[pu * 256 + row]).x - mmax);
-            const float4* base = a.part_o + pu * 32 * 256 + row;
-            float4 o[8];
+            const float4 ml = __ldcg(&a.part_ml[pu * 256 + row]);
+            const float g = exp2f(ml.x - mmax) * ml.y * ml.z;
+            const uint4* base = a.part_o + pu * 16 * 256 + row;
+            uint4 o[4];
 #pragma unroll
-            for (int k = 0; k < 8; ++k) o[k] = __ldcg(base + (c0 + k) * 256);
+            for (int k = 0; k < 4; ++k) o[k] = __ldcg(base + (c0 + k) * 256);
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                acc[k].x += o[k].x * g;
-                acc[k].y += o[k].y * g;
-                acc[k].z += o[k].z * g;
-                acc[k].w += o[k].w * g;
+            for (int k = 0; k < 4; ++k) {
+                const uint32_t w[4] = {o[k].x, o[k].y, o[k].z, o[k].w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 x = f16x2_to_f32x2(w[e]);
+                    acc[k][e].x = fmaf(x.x, g, acc[k][e].x);
+                    acc[k][e].y = fmaf(x.y, g, acc[k][e].y);
+                }
             }
         }
 #pragma unroll
-        for (int k = 0; k < 8; k += 2)
-            reinterpret_cast<uint4*>(dst)[(c0 + k) >> 1] =
-                make_uint4(pack_bf16x2(acc[k].x * inv, acc[k].y * inv), pack_bf16x2(acc[k].z * inv, acc[k].w * inv),
-                           pack_bf16x2(acc[k + 1].x * inv, acc[k + 1].y * inv),
-                           pack_bf16x2(acc[k + 1].z * inv, acc[k + 1].w * inv));
+        for (int k = 0; k < 4; ++k)
+            reinterpret_cast<uint4*>(dst)[c0 + k] =
+                make_uint4(pack_bf16x2(acc[k][0].x * inv, acc[k][0].y * inv),
+                           pack_bf16x2(acc[k][1].x * inv, acc[k][1].y * inv),
+                           pack_bf16x2(acc[k][2].x * inv, acc[k][2].y * inv),
+                           pack_bf16x2(acc[k][3].x * inv, acc[k][3].y * inv));
     }
     if (lse_dst) *lse_dst = (mmax + log2f(L)) * 0.69314718055994531f;
 }
@@ -735,8 +769,8 @@ __global__ void __launch_bounds__(kMode == kFused ? 512 : 384, 1)
             const int prow = w * BM + r;
             if (active && ok) {
                 tc_fence_after();
-                store_partial_row(t_o, a.part_o + pu * 32 * 256 + prow);
-                a.part_ml[pu * 256 + prow] = make_float2(m_ref, l);
+                const float sc = store_partial_row(t_o, 1.0f / l, a.part_o + pu * 16 * 256 + prow);
+                a.part_ml[pu * 256 + prow] = make_float4(m_ref, l, sc, 0.0f);
             }
             __threadfence();
             named_bar_sync(2, 256);

@@ -177,9 +177,9 @@ def test_workspace_plans_between_the_minimum_and_the_full_size():
     assert low == 256 + 2 * qk + up(16 * (124 + 23) * 16) + up(16 * 2896 * 4)
     # the full plan adds the FP16 copy of the INT8 window (2 x 16 heads x 15,840 tokens x
     # 256 B) and the KV-split partials: per split, 16 heads x 12 Q-tile pairs x 256 rows
-    # of 128 fp32 values and an fp32 (max, sum) pair, and one counter per unit
+    # of 128 FP16 values and an fp32 (max, sum, 2^e, 0) record, and one counter per unit
     copy = 2 * 16 * 18 * 880 * 256
-    per_split = 16 * 12 * 256 * (128 * 4 + 8)
+    per_split = 16 * 12 * 256 * (128 * 2 + 16)
     assert full - low >= copy + 2 * per_split and full % 256 == 0
     call = lambda wsb: nm.nomas_seg_attn(d, FAKE, FAKE, FAKE, 2048, 3, 256, FAKE, None, FAKE, wsb, None)
     assert call(low - 1) == nm.NOMAS_ERR_WORKSPACE
