@@ -526,9 +526,13 @@ def run_extra(args, torch, nm, dev):
         b.record(stream)
         b.synchronize()
         ms = a.elapsed_time(b) / reps
-        # the batched commit alone, L2 flushed before each: 54 x 32.8 MB
+        # the batched commit alone, L2 flushed before each: 54 x 32.8 MB. A short
+        # device-side delay ahead of the flush keeps the GPU busy while the host
+        # marshals the 54 cache descriptors, so that the events bracket the
+        # launch and not host time
         cm = []
         for _ in range(10):
+            torch.cuda._sleep(2_000_000)
             flush.zero_()
             a, b = device_events(torch, 2)
             a.record(stream)

@@ -176,8 +176,10 @@ __device__ __forceinline__ uint2 quantize8(const float (&y)[8], float& scale_out
     return r;
 }
 
+// At most 64 registers a thread, so that the persistent grid (two blocks per
+// SM) is resident in one wave.
 template <bool kGrouped, bool kInt8, int kF, int kL>
-__global__ void __launch_bounds__(kThreads) commit_kernel(const __grid_constant__ CommitArgs a,
+__global__ void __launch_bounds__(kThreads, 2) commit_kernel(const __grid_constant__ CommitArgs a,
                                                           const __grid_constant__ CommitLayersT<kL> L,
                                                           const __grid_constant__ RopeTabT<kF> tab) {
     // A warp task is one layer's token and a group of `head_group` of its heads; the
@@ -566,11 +568,12 @@ void commit_variant(const CommitArgs& a, int grid, const CommitLayersT<kL>& L, c
 
 cudaError_t launch_commit(const CommitArgs& a_in, const CommitLayers& layers, const RopeTab& tab, cudaStream_t s) {
     // heads per warp task: all of a token's heads when there are enough tokens
-    // to give every resident warp several tasks, else halves of that, down to 2,
-    // so that small commits still spread over the GPU
+    // to give every resident warp (two 512-thread blocks per SM) two tasks, else
+    // halves of that, down to 2, so that small commits still spread over the
+    // GPU (a 3-frame commit of 16 heads: 4 heads per task)
     CommitArgs a = a_in;
     const int64_t tokens = static_cast<int64_t>(a.n_frames) * a.tpf * a.n_layers;
-    const int64_t want = 4ll * 148 * 2 * (kThreads / 32);
+    const int64_t want = 2ll * 148 * 2 * (kThreads / 32);
     int hg = a.heads;
     while (hg > 2 && tokens * ((a.heads + hg - 1) / hg) < want) hg = (hg + 1) / 2;
     a.head_group = hg;
