@@ -395,53 +395,74 @@ __device__ __forceinline__ float2 f16x2_to_f32x2(uint32_t w) {
 
 // Merge of the splits of one row (run by the last CTA of a unit to arrive):
 // O = sum_s 2^(m_s - M) l_s O^_s 2^e_s / sum_s 2^(m_s - M) l_s with M = max_s m_s
-// and O^_s the stored FP16 row of split s. Four 16-byte loads per split are in
-// flight at a time.
+// and O^_s the stored FP16 row of split s. Splits are taken four at a time,
+// with all their loads issued before any is used: a pass over four chunks
+// (32 dims) of up to four splits has 20 loads in flight, so a row costs about
+// six L2 round trips instead of one per split and chunk group. Absent splits
+// of a group load nothing and weigh 0.
 __device__ __noinline__ void merge_row(const AttnArgs& a, int unit, int row, uint16_t* dst, float* lse_dst) {
-    const int units = a.heads * a.pairs;
+    const int64_t stride = static_cast<int64_t>(a.heads) * a.pairs * 256; // records between splits
+    const float4* ml = a.part_ml + static_cast<int64_t>(unit) * 256 + row;
+    const uint4* po = a.part_o + static_cast<int64_t>(unit) * 16 * 256 + row;
+    auto load_ml = [&](int s) { return s < a.splits ? __ldcg(ml + s * stride) : make_float4(-INFINITY, 0.f, 0.f, 0.f); };
     float mmax = -INFINITY;
-    for (int s = 0; s < a.splits; ++s)
-        mmax = fmaxf(mmax, __ldcg(&a.part_ml[(static_cast<int64_t>(s) * units + unit) * 256 + row]).x);
+    for (int s0 = 0; s0 < a.splits; s0 += 4) {
+        float4 r[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) r[k] = load_ml(s0 + k);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) mmax = fmaxf(mmax, r[k].x);
+    }
     float L = 0.0f;
-    for (int s = 0; s < a.splits; ++s) {
-        const float4 ml = __ldcg(&a.part_ml[(static_cast<int64_t>(s) * units + unit) * 256 + row]);
-        L += ml.y * exp2f(ml.x - mmax);
+    for (int s0 = 0; s0 < a.splits; s0 += 4) {
+        float4 r[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) r[k] = load_ml(s0 + k);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) L += r[k].y * exp2f(r[k].x - mmax);
     }
     const float inv = 1.0f / L;
 #pragma unroll 1
     for (int c0 = 0; c0 < 16; c0 += 4) {
         float2 acc[4][4];
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
+        for (int j = 0; j < 4; ++j)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) acc[k][e] = make_float2(0.0f, 0.0f);
+            for (int e = 0; e < 4; ++e) acc[j][e] = make_float2(0.0f, 0.0f);
 #pragma unroll 1
-        for (int s = 0; s < a.splits; ++s) {
-            const int64_t pu = static_cast<int64_t>(s) * units + unit;
-            const float4 ml = __ldcg(&a.part_ml[pu * 256 + row]);
-            const float g = exp2f(ml.x - mmax) * ml.y * ml.z;
-            const uint4* base = a.part_o + pu * 16 * 256 + row;
-            uint4 o[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) o[k] = __ldcg(base + (c0 + k) * 256);
+        for (int s0 = 0; s0 < a.splits; s0 += 4) {
+            float4 r[4];
+            uint4 o[4][4];
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-                const uint32_t w[4] = {o[k].x, o[k].y, o[k].z, o[k].w};
+                const bool on = s0 + k < a.splits;
+                r[k] = load_ml(s0 + k);
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 x = f16x2_to_f32x2(w[e]);
-                    acc[k][e].x = fmaf(x.x, g, acc[k][e].x);
-                    acc[k][e].y = fmaf(x.y, g, acc[k][e].y);
+                for (int j = 0; j < 4; ++j)
+                    o[k][j] = on ? __ldcg(po + (s0 + k) * stride * 16 + (c0 + j) * 256) : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float g = exp2f(r[k].x - mmax) * r[k].y * r[k].z;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const uint32_t w[4] = {o[k][j].x, o[k][j].y, o[k][j].z, o[k][j].w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 x = f16x2_to_f32x2(w[e]);
+                        acc[j][e].x = fmaf(x.x, g, acc[j][e].x);
+                        acc[j][e].y = fmaf(x.y, g, acc[j][e].y);
+                    }
                 }
             }
         }
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-            reinterpret_cast<uint4*>(dst)[c0 + k] =
-                make_uint4(pack_bf16x2(acc[k][0].x * inv, acc[k][0].y * inv),
-                           pack_bf16x2(acc[k][1].x * inv, acc[k][1].y * inv),
-                           pack_bf16x2(acc[k][2].x * inv, acc[k][2].y * inv),
-                           pack_bf16x2(acc[k][3].x * inv, acc[k][3].y * inv));
+        for (int j = 0; j < 4; ++j)
+            reinterpret_cast<uint4*>(dst)[c0 + j] =
+                make_uint4(pack_bf16x2(acc[j][0].x * inv, acc[j][0].y * inv),
+                           pack_bf16x2(acc[j][1].x * inv, acc[j][1].y * inv),
+                           pack_bf16x2(acc[j][2].x * inv, acc[j][2].y * inv),
+                           pack_bf16x2(acc[j][3].x * inv, acc[j][3].y * inv));
     }
     if (lse_dst) *lse_dst = (mmax + log2f(L)) * 0.69314718055994531f;
 }
