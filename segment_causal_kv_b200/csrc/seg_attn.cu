@@ -528,23 +528,11 @@ __global__ void __launch_bounds__(kMode == kFused ? 512 : 384, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    // ---- work unit: units with two Q tiles first, then (when the Q tile count
-    // is odd) the heads' last units of one Q tile, which take about half as long
-    // and so fill the last wave (the in-shared-memory form keeps the plain
-    // order, measured faster there); the splits of a unit are consecutive CTAs
-    const int full_pairs = kFill ? a.pairs : a.tiles_q / 2;
-    const int uo = blockIdx.x / a.splits;
+    // ---- work unit
+    const int unit = blockIdx.x / a.splits;
     const int split = blockIdx.x % a.splits;
-    const int n_full = a.heads * full_pairs;
-    int head, pair;
-    if (uo < n_full) { // then full_pairs >= 1
-        head = uo / full_pairs;
-        pair = uo - head * full_pairs;
-    } else {
-        head = uo - n_full;
-        pair = full_pairs;
-    }
-    const int unit = head * a.pairs + pair;
+    const int head = unit / a.pairs;
+    const int pair = unit % a.pairs;
     const int qt0 = 2 * pair;
     const bool has_q1 = (qt0 + 1) < a.tiles_q;
     const int nq_tiles = has_q1 ? 2 : 1;
