@@ -46,9 +46,9 @@
 // the reference follows x + c_T (x the log2-scaled score, c_T the V exponent
 // of its tile): P' = 2^(x + c_T - m) times V^ is 2^(x - m) times V, and the
 // row sum adds P' * 2^-c_T.
-// Split-KV: with splits > 1 each CTA leaves (O unnormalised, max, sum) in the
-// workspace and counts itself in per unit; the last CTA of a unit to arrive
-// merges the splits and writes the output (the partials are still in L2).
+// Split-KV: with splits > 1 each CTA leaves O/l in FP16 (times a per-row 2^-e)
+// and (max, sum, 2^e) in the workspace and counts itself in per unit; the last
+// CTA of a unit merges the splits and writes the output (partials still in L2).
 #include "nomas_f16.cuh"
 #include "nomas_internal.h"
 #include "nomas_ptx.cuh"
